@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark of block generation with the denoising-step library.
+
+One bench step = one block: a 256-token random canvas denoised until the
+mean-entropy stop (or the step budget), then its causal hand-off into the KV
+cache.  Workload full_b1 (default): 30 full-width layers, batch 1, an 8192-token
+prompt already in the cache, up to 48 steps, linear keep over 48, stop 0.1 nats,
+logit scale 1.5^(t-1).  Before every block the request's cache length is reset
+to the prompt, so every step does the same work.  Weights (49 GB) exceed L2.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (one per GPU, no data-path collective; the
+only collectives are the timing barrier and a max-reduction of the times).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["full_b1", "full_b16"], default="full_b1")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help=argparse.SUPPRESS)  # debugging only (0 = as specified)
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------- distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(backend):
+    import datetime
+
+    import torch.distributed as dist
+    world, rank, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    return dist if world > 1 else None
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def aggregate(dist, elapsed_ms: float, units: float, device=None):
+    """Max elapsed over ranks and the sum of the units all ranks processed."""
+    import torch
+    if dist is None:
+        return elapsed_ms, units
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload(name, layers_override=0):
+    from discrete_text_diffusion_b200 import synth
+    W = dict(synth.WORKLOADS[name])
+    W["model"] = dict(W["model"])
+    if layers_override:
+        W["model"]["n_layers"] = layers_override
+    return W
+
+
+def moe_up_bytes(model, n_rows, touched):
+    """Algorithmic bytes of one grouped gate/up launch: the touched experts' gate
+    and up weights (bf16), the permuted token rows read, the bf16 output written."""
+    d, f = model["d_model"], model["d_ff"]
+    return touched * 2 * f * d * 2 + n_rows * d * 2 + n_rows * f * 2
+
+
+# -------------------------------------------------------------------- ours
+
+def run_ours(args):
+    import torch
+
+    import discrete_text_diffusion_b200 as m
+    from discrete_text_diffusion_b200 import synth
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = init_dist("nccl")
+    dev = torch.device("cuda", local)
+    W = workload(args.workload, args.layers)
+    model, S = W["model"], W["sampler"]
+    B, n, P0 = W["batch"], model["canvas"], W["prompt_len"]
+    blocks = W.get("blocks", 1)
+    max_ctx = ((P0 + blocks * n + 63) // 64) * 64
+    max_tokens = max(B * n, min(8192, B * P0))
+    w = synth.make_weights(model, seed=W["seed"], dtype=W["dtype"], router_bias=W["router_bias"], device=dev)
+    h = m.dg_create(model, w, dtype=W["dtype"], max_batch=B, max_ctx=max_ctx, max_tokens=max_tokens)
+    req = list(range(B))
+    prompt = synth.uniform_tokens(P0, model["vocab"], seed=W["seed"] + 1, batch=B, device=dev)
+    t0 = time.time()
+    m.dg_prefill_prompt(h, req, prompt)
+    m.dg_synchronize(h)
+    prefill_s = time.time() - t0
+
+    # experts touched per layer on this workload's canvas (for the roofline bytes)
+    touched = torch.zeros(model["n_layers"], dtype=torch.int32, device=dev)
+    canvas = synth.uniform_tokens(n, model["vocab"], seed=W["seed"] + 2, batch=B, device=dev)
+    m.dg_denoise_step(h, req, canvas, None, 1, m.sampler_params(keep_k=1, seed=S["seed"]),
+                      m.step_out(experts_touched=touched))
+    m.dg_synchronize(h)
+    touched_mean = float(touched.float().mean().item())
+
+    out = torch.zeros((B, n), dtype=torch.int32, device=dev)
+    out_host = torch.zeros((B, n), dtype=torch.int32).pin_memory()
+    steps_seen = []
+
+    def one_step(host=False):
+        total = 0
+        for blk in range(blocks):
+            if blk == 0:
+                for r in req:
+                    m.dg_set_length(h, r, P0)
+            a = m.block_args(req, S["max_steps"], S["schedule_steps"], temperature=S["temperature"],
+                             logit_scale_growth=S["logit_scale_growth"], stop_threshold=S["stop_threshold"],
+                             seed=S["seed"], block=blk)
+            if host:
+                total += m.dg_generate_block_host(h, a, out_host)
+            else:
+                total += m.dg_generate_block(h, a, out)
+        steps_seen.append(total)
+
+    for _ in range(args.warmup):
+        one_step()
+    m.dg_synchronize(h)
+
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    m.dg_profile_reset(h)
+    m.dg_profile_enable(h, True)
+    launches0 = m.dg_launch_count(h)
+    steps_seen.clear()
+    with ClockSampler(local) as clk:
+        barrier(dist)
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            one_step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dist)
+    elapsed = ev0.elapsed_time(ev1)
+    launches = m.dg_launch_count(h) - launches0
+    prof = m.dg_profile_read(h)
+    m.dg_profile_enable(h, False)
+    clocks = clk.summary()
+    denoise_steps = sum(steps_seen)
+    units = args.steps * blocks * B * n
+    elapsed_max, units_all = aggregate(dist, elapsed, units, device=dev)
+
+    # end to end: the same calls with the tokens landing in pinned host memory
+    steps_seen.clear()
+    barrier(dist)
+    torch.cuda.synchronize(dev)
+    e0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step(host=True)
+    torch.cuda.synchronize(dev)
+    e2e_ms = (time.perf_counter() - e0) * 1e3
+    e2e_max, _ = aggregate(dist, e2e_ms, units, device=dev)
+
+    peaks, peak_kind = load_peaks()
+    roof = None
+    if "moe_up" in prof:
+        nl, ms = prof["moe_up"]
+        per_launch_s = ms / nl / 1e3
+        byt = moe_up_bytes(model, B * n * model["top_k"], touched_mean)
+        ach = byt / per_launch_s / 1e9
+        roof = {"kernel": "gemm_tc_kernel (grouped gate/up + SwiGLU)", "bound": "hbm", "achieved": round(ach, 1),
+                "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
+                "bytes_per_launch": int(byt), "avg_launch_us": round(per_launch_s * 1e6, 2),
+                "experts_touched_mean": round(touched_mean, 2)}
+    line = {
+        "metric": "canvas tokens/s (block generation, adaptive stop)",
+        "value": round(units_all / (elapsed_max / 1e3), 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_max / args.steps, 3),
+        "us_per_denoise_step": round(elapsed_max * 1e3 / max(1, denoise_steps), 1),
+        "denoise_steps_per_block": round(denoise_steps / max(1, args.steps * blocks), 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded random weights N(0,0.02), uniform prompt tokens)",
+        "config": {"workload": args.workload, "batch": B, "canvas": n, "prompt_len": P0,
+                   "layers": model["n_layers"], "d_model": model["d_model"], "experts": model["n_experts"],
+                   "top_k": model["top_k"], "vocab": model["vocab"], "blocks_per_step": blocks,
+                   "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (49 GB of weights)"},
+        "e2e": {"value": round(units_all / (e2e_max / 1e3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": 4 * B * blocks, "d2h_bytes_per_step": 4 * B * n * blocks},
+        "gpu_launches": int(launches),
+        "roofline": roof,
+        "clocks": clocks,
+        "prefill_s": round(prefill_s, 2),
+        "kernel_ms": {k: round(v[1], 3) for k, v in prof.items()},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(W, line["denoise_steps_per_block"])
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    h.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ oracle
+
+def _blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [os.cpu_count() or 1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(W, head_rows=16, seed_off=0):
+    """Time the CPU oracle on a bounded sample of the workload: one full layer
+    over the whole canvas against a cache of prompt_len positions, and the LM
+    head + sampler for head_rows positions.  Returns (layer_s, head_s_per_row)."""
+    import numpy as np
+
+    from discrete_text_diffusion_b200 import synth
+    from oracle import dg_oracle as O
+    model = dict(W["model"])
+    n, P0 = model["canvas"], W["prompt_len"]
+    w = synth.make_weights(model, seed=W["seed"] + seed_off, dtype="bf16", router_bias=True, layers=[0])
+    om = O.OracleModel(model, synth.to_numpy_weights(w))
+    k, v = synth.normal_kv(model["n_kv_heads"], P0, model["head_dim"], seed=W["seed"] + 5, dtype="bf16")
+    om.set_kv(0, 0, k.float().numpy(), v.float().numpy())
+    canvas = synth.uniform_tokens(n, model["vocab"], seed=W["seed"] + 6).numpy()
+    t0 = time.perf_counter()
+    hx = om.embed_tokens(canvas)
+    h1, _, _ = om.layer(hx, 0, 0, P0 + np.arange(n), causal=False)
+    t1 = time.perf_counter()
+    x = O.rms_norm(h1[:head_rows], om.weights["final_norm"], model["rms_eps"])
+    logits = O.lm_head(x, om.weights["embed"])
+    O.sample_canvas(logits, seed=0, step=1, block=0, req=0, temperature=1.0, logit_scale=1.0,
+                    keep_k=head_rows // 2, stop_threshold=0.1)
+    t2 = time.perf_counter()
+    return t1 - t0, (t2 - t1) / head_rows
+
+
+def oracle_tokens_per_s(W, layer_s, head_row_s, steps_per_block):
+    """Extrapolate the sample to the workload: per denoise step all layers on
+    the canvas plus the head for all positions; per block the steps plus one
+    more layer stack for the hand-off."""
+    model = W["model"]
+    n, B, L = model["canvas"], W["batch"], model["n_layers"]
+    step_s = B * (L * layer_s + n * head_row_s)
+    block_s = steps_per_block * step_s + B * L * layer_s
+    return B * n / block_s, step_s, block_s
+
+
+def cpu_baseline(W, steps_per_block):
+    layer_s, head_row_s = oracle_sample(W)
+    tps, step_s, block_s = oracle_tokens_per_s(W, layer_s, head_row_s, steps_per_block)
+    return {"value": round(tps, 5), "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": (f"float64 numpy oracle: 1 of {W['model']['n_layers']} layers on the full "
+                       f"{W['model']['canvas']}-token canvas over a {W['prompt_len']}-position cache "
+                       f"({layer_s:.2f} s) and LM head + sampler for 16 positions ({head_row_s * 16:.2f} s); "
+                       f"extrapolated to {steps_per_block} steps/block: {step_s:.1f} s/step, "
+                       f"{block_s:.1f} s/block")}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    W = workload(args.workload)
+    steps_per_block = 13.0
+    rates = []
+    for i in range(args.warmup + args.steps):
+        layer_s, head_row_s = oracle_sample(W, seed_off=0)
+        tps, _, block_s = oracle_tokens_per_s(W, layer_s, head_row_s, steps_per_block)
+        if i >= args.warmup:
+            rates.append((tps, block_s))
+    value = statistics.median(r[0] for r in rates)
+    line = {
+        "impl": "reference",
+        "metric": "canvas tokens/s (block generation, adaptive stop)",
+        "value": round(value, 5), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(statistics.median(r[1] for r in rates) * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded random weights, uniform tokens)",
+        "config": {"workload": args.workload, "batch": W["batch"], "canvas": W["model"]["canvas"],
+                   "prompt_len": W["prompt_len"], "layers": W["model"]["n_layers"],
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": "per step: 1 layer on the full canvas + LM head/sampler for 16 positions, "
+                                   f"extrapolated at {steps_per_block} denoise steps per block"},
+        "e2e": {"value": round(value, 5), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

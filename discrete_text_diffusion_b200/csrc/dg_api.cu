@@ -1,0 +1,933 @@
+// C ABI of the denoising-step library (see include/dg.h) and the host-side
+// orchestration of the step: workspaces, KV cache, TMA descriptors, the layer
+// loop, the sampler and the block loop with its causal hand-off.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/dg.h"
+#include "kernels.h"
+
+using namespace dg;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+// ------------------------------------------------------------ TMA encode
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 map over a row-major [rows, cols] matrix, box (64 cols, box_rows rows), 128-byte swizzle.
+bool tmap_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_stride_elems,
+             uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 3D bf16 map over [n2, rows, cols], box (64, box_rows, 1).
+bool tmap_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t n2, uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, n2};
+  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+enum ProfClass {
+  PC_EMBED, PC_DENSE, PC_ROPE, PC_ATTN, PC_NORM, PC_ROUTER, PC_GATHER, PC_MOE_UP, PC_MOE_DOWN, PC_COMBINE,
+  PC_LMHEAD, PC_SAMPLER, PC_FINISH, PC_COUNT
+};
+const char* kProfNames[PC_COUNT] = {"embed",  "dense_gemm", "rope_scatter", "attention", "rmsnorm",
+                                    "router", "gather",     "moe_up",       "moe_down",  "combine",
+                                    "lm_head", "sampler_rows", "sampler_finish"};
+
+}  // namespace
+
+struct LayerMaps {
+  CUtensorMap wq, wk, wv, wo, router, gate, up, down;
+};
+
+struct dg_handle {
+  dg_config c{};
+  bool bf16 = false;
+  size_t esz = 4;
+  cudaStream_t stream = nullptr;
+  int num_sms = 148;
+  int dev = 0;
+  std::string err;
+  // weights (borrowed)
+  const void* embed = nullptr;
+  const void* w_sc = nullptr;
+  const float* final_norm = nullptr;
+  std::vector<dg_layer_weights> lw;
+  std::vector<LayerMaps> lmaps;
+  CUtensorMap m_embed{}, m_wsc{}, m_dummy{};
+  // KV cache (owned)
+  void* kc = nullptr;
+  void* vt = nullptr;
+  std::vector<int> len;
+  // workspace (owned)
+  int T_max = 0;
+  float* h = nullptr;
+  void* xn = nullptr;
+  void* eprev = nullptr;
+  float* qkv = nullptr;
+  void* q = nullptr;
+  void* attn = nullptr;
+  float* glog = nullptr;
+  int32_t* ids = nullptr;
+  float* wts = nullptr;
+  int32_t* cnt = nullptr;
+  int32_t* off = nullptr;
+  int32_t* perm = nullptr;
+  int32_t* work = nullptr;
+  int32_t* n_work = nullptr;
+  int n_work_max = 0;
+  int32_t* touched = nullptr;
+  void* xp = nullptr;
+  void* hb = nullptr;
+  float* y = nullptr;
+  float* logits = nullptr;
+  float2* rope = nullptr;
+  CUtensorMap m_xn{}, m_eprev{}, m_attn{}, m_xp{}, m_hb{};
+  // sampler workspace
+  void* sws = nullptr;
+  int32_t* xh[2] = {nullptr, nullptr};
+  float* pmax = nullptr;
+  float* ent = nullptr;
+  int32_t* keep = nullptr;
+  float* meanh = nullptr;
+  int32_t* stop = nullptr;
+  int32_t* done = nullptr;
+  int32_t* canvas = nullptr;
+  int32_t* out_tok = nullptr;
+  int32_t* req_dev = nullptr;
+  int32_t* tok_ws = nullptr;
+  int* d_err = nullptr;
+  int32_t* h_done = nullptr;  // pinned
+  // profiling
+  bool prof = false;
+  struct Rec { int cls; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t pool_used = 0;
+  uint64_t launches = 0;
+};
+
+namespace {
+
+int fail(dg_handle* H, int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  if (H) H->err = buf;
+  else g_create_error = buf;
+  return code;
+}
+
+int cuda_check(dg_handle* H, cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return DG_OK;
+  return fail(H, DG_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+cudaEvent_t pool_event(dg_handle* H) {
+  if (H->pool_used == H->pool.size()) {
+    cudaEvent_t e;
+    cudaEventCreate(&e);
+    H->pool.push_back(e);
+  }
+  return H->pool[H->pool_used++];
+}
+
+struct ProfScope {
+  dg_handle* H;
+  int cls;
+  cudaEvent_t b = nullptr;
+  int n;
+  ProfScope(dg_handle* h, int c, int n_launch = 1) : H(h), cls(c), n(n_launch) {
+    if (H->prof) {
+      cudaEvent_t a = pool_event(H);
+      b = pool_event(H);
+      cudaEventRecord(a, H->stream);
+      H->recs.push_back({cls, a, b});
+    }
+  }
+  ~ProfScope() {
+    if (H->prof) cudaEventRecord(b, H->stream);
+    H->launches += (uint64_t)n;
+  }
+};
+
+template <typename T>
+T* dalloc(size_t n, bool* ok) {
+  void* p = nullptr;
+  if (n == 0) n = 1;
+  if (cudaMalloc(&p, n * sizeof(T)) != cudaSuccess) { *ok = false; return nullptr; }
+  return reinterpret_cast<T*>(p);
+}
+
+inline size_t kv_layer_elems(const dg_config& c) {
+  return (size_t)c.max_batch * c.n_kv_heads * c.max_ctx * c.head_dim;
+}
+inline void* kc_layer(dg_handle* H, int l) {
+  return (char*)H->kc + (size_t)l * kv_layer_elems(H->c) * H->esz;
+}
+inline void* vt_layer(dg_handle* H, int l) {
+  return (char*)H->vt + (size_t)l * kv_layer_elems(H->c) * H->esz;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int pick_ntile(int n_mtiles, int T, int num_sms) {
+  int nt = 256;
+  const int tmax = std::max(32, ((T + 31) / 32) * 32);
+  while (nt > tmax && nt > 32) nt >>= 1;
+  while (nt > 32 && (long)n_mtiles * ((T + nt - 1) / nt) < num_sms) nt >>= 1;
+  return nt;
+}
+
+int grouped_tile(const dg_handle* H, int T) {
+  if (!H->bf16) return 64;
+  const double avg = (double)T * H->c.top_k / H->c.n_experts;
+  if (avg > 128) return 256;
+  if (avg > 48) return 128;
+  return 64;
+}
+
+// ------------------------------------------------------------ GEMM helpers
+// out = x[T, K] * W^T (W [n_out, K]) for the dense projections.
+void dense_gemm(dg_handle* H, int cls, const void* x, const CUtensorMap* mx, const void* w, const CUtensorMap* mw,
+                int T, int n_out, int K, Epi epi, void* out, int ld_out) {
+  ProfScope ps(H, cls);
+  if (!H->bf16) {
+    launch_gemm_simt<float>((const float*)x, (const float*)w, T, n_out, K, epi, out, ld_out, nullptr, H->stream);
+    return;
+  }
+  TcGemm g{};
+  g.mode = 0;
+  g.M = n_out;
+  g.K = K;
+  g.T = T;
+  g.ntile = pick_ntile((n_out + 127) / 128, T, H->num_sms);
+  g.seg1 = g.seg2 = INT_MAX;
+  g.epi = epi;
+  g.out = out;
+  g.ld_out = ld_out;
+  g.err = H->d_err;
+  launch_gemm_tc(*mw, H->m_dummy, H->m_dummy, *mx, g, H->num_sms, H->stream);
+}
+
+void qkv_gemm(dg_handle* H, int l, int T) {
+  const dg_config& c = H->c;
+  const dg_layer_weights& L = H->lw[l];
+  const int nq = c.n_heads * c.head_dim, nk = c.n_kv_heads * c.head_dim;
+  const int ld = nq + 2 * nk;
+  ProfScope ps(H, PC_DENSE, H->bf16 ? 1 : 3);
+  if (!H->bf16) {
+    const float* x = (const float*)H->xn;
+    launch_gemm_simt<float>(x, (const float*)L.wq, T, nq, c.d_model, EPI_STORE_F32, H->qkv, ld, nullptr, H->stream);
+    launch_gemm_simt<float>(x, (const float*)L.wk, T, nk, c.d_model, EPI_STORE_F32, H->qkv + nq, ld, nullptr,
+                            H->stream);
+    launch_gemm_simt<float>(x, (const float*)L.wv, T, nk, c.d_model, EPI_STORE_F32, H->qkv + nq + nk, ld, nullptr,
+                            H->stream);
+    return;
+  }
+  TcGemm g{};
+  g.mode = 0;
+  g.M = ld;
+  g.K = c.d_model;
+  g.T = T;
+  g.ntile = pick_ntile((ld + 127) / 128, T, H->num_sms);
+  g.seg1 = nq;
+  g.seg2 = nq + nk;
+  g.epi = EPI_STORE_F32;
+  g.out = H->qkv;
+  g.ld_out = ld;
+  g.err = H->d_err;
+  const LayerMaps& M = H->lmaps[l];
+  launch_gemm_tc(M.wq, M.wk, M.wv, H->m_xn, g, H->num_sms, H->stream);
+}
+
+void moe_gemms(dg_handle* H, int l, int T) {
+  const dg_config& c = H->c;
+  const dg_layer_weights& L = H->lw[l];
+  const int tile = grouped_tile(H, T);
+  const int n_work_max = c.n_experts + (T * c.top_k + tile - 1) / tile;
+  {
+    ProfScope ps(H, PC_MOE_UP);
+    if (!H->bf16) {
+      launch_grouped_simt<float>((const float*)H->xp, (const float*)L.w_gate, (const float*)L.w_up, c.d_ff,
+                                 c.d_model, H->work, H->n_work, n_work_max, H->perm, true, H->hb, c.d_ff, H->stream);
+    } else {
+      TcGemm g{};
+      g.mode = 1;
+      g.M = c.d_ff;
+      g.K = c.d_model;
+      g.ntile = tile;
+      g.seg1 = g.seg2 = INT_MAX;
+      g.work = H->work;
+      g.n_work = H->n_work;
+      g.n_work_max = n_work_max;
+      g.epi = EPI_SWIGLU_ACT;
+      g.out = H->hb;
+      g.ld_out = c.d_ff;
+      g.err = H->d_err;
+      launch_gemm_tc(H->lmaps[l].gate, H->lmaps[l].up, H->m_dummy, H->m_xp, g, H->num_sms, H->stream);
+    }
+  }
+  {
+    ProfScope ps(H, PC_MOE_DOWN);
+    if (!H->bf16) {
+      launch_grouped_simt<float>((const float*)H->hb, (const float*)L.w_down, nullptr, c.d_model, c.d_ff, H->work,
+                                 H->n_work, n_work_max, H->perm, false, H->y, c.d_model, H->stream);
+    } else {
+      TcGemm g{};
+      g.mode = 2;
+      g.M = c.d_model;
+      g.K = c.d_ff;
+      g.ntile = tile;
+      g.seg1 = g.seg2 = INT_MAX;
+      g.work = H->work;
+      g.n_work = H->n_work;
+      g.n_work_max = n_work_max;
+      g.epi = EPI_SCATTER_F32;
+      g.out = H->y;
+      g.ld_out = c.d_model;
+      g.row_map = H->perm;
+      g.err = H->d_err;
+      launch_gemm_tc(H->lmaps[l].down, H->m_dummy, H->m_dummy, H->m_hb, g, H->num_sms, H->stream);
+    }
+  }
+}
+
+void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
+  const dg_config& c = H->c;
+  AttnArgs a{};
+  a.B = bi.B;
+  a.nq = nq;
+  a.hq = c.n_heads;
+  a.hkv = c.n_kv_heads;
+  a.hd = c.head_dim;
+  a.max_ctx = c.max_ctx;
+  a.causal = causal ? 1 : 0;
+  a.bi = bi;
+  ProfScope ps(H, PC_ATTN);
+  if (!H->bf16)
+    launch_attn_simt<float>((const float*)H->q, (const float*)kc_layer(H, l), (const float*)vt_layer(H, l),
+                            (float*)H->attn, a, H->stream);
+  else
+    launch_attn_simt<__nv_bfloat16>((const __nv_bfloat16*)H->q, (const __nv_bfloat16*)kc_layer(H, l),
+                                    (const __nv_bfloat16*)vt_layer(H, l), (__nv_bfloat16*)H->attn, a, H->stream);
+}
+
+template <typename T>
+void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const int32_t* tokens,
+                  const int32_t* prev, bool head, float* logits, float* hidden_out) {
+  const dg_config& c = H->c;
+  const int Tn = bi.B * nq;
+  const float eps = (float)c.rms_eps;
+  T* xn = (T*)H->xn;
+  {
+    ProfScope ps(H, PC_EMBED);
+    launch_embed<T>(tokens, prev, (const T*)H->embed, H->h, (T*)H->eprev, Tn, c.d_model, c.vocab, H->d_err,
+                    H->stream);
+  }
+  if (prev) dense_gemm(H, PC_DENSE, H->eprev, &H->m_eprev, H->w_sc, &H->m_wsc, Tn, c.d_model, c.d_model,
+                       EPI_ADD_F32, H->h, c.d_model);
+  {
+    ProfScope ps(H, PC_NORM);
+    const float* w0 = c.n_layers > 0 ? H->lw[0].attn_norm : H->final_norm;
+    launch_rmsnorm<T>(H->h, w0, xn, Tn, c.d_model, eps, H->stream);
+  }
+  const int ldqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_layer_weights& L = H->lw[l];
+    qkv_gemm(H, l, Tn);
+    {
+      ProfScope ps(H, PC_ROPE);
+      launch_rope_scatter<T>(H->qkv, (T*)H->q, (T*)kc_layer(H, l), (T*)vt_layer(H, l), (const float*)H->rope, bi,
+                             nq, c.n_heads, c.n_kv_heads, c.head_dim, c.max_ctx, H->stream);
+    }
+    (void)ldqkv;
+    attention(H, l, bi, nq, causal);
+    dense_gemm(H, PC_DENSE, H->attn, &H->m_attn, L.wo, &H->lmaps[l].wo, Tn, c.d_model, c.n_heads * c.head_dim,
+               EPI_ADD_F32, H->h, c.d_model);
+    {
+      ProfScope ps(H, PC_NORM);
+      launch_rmsnorm<T>(H->h, L.ffn_norm, xn, Tn, c.d_model, eps, H->stream);
+    }
+    dense_gemm(H, PC_ROUTER, H->xn, &H->m_xn, L.router_w, &H->lmaps[l].router, Tn, c.n_experts, c.d_model,
+               EPI_STORE_F32, H->glog, c.n_experts);
+    {
+      ProfScope ps(H, PC_ROUTER, 2);
+      launch_router_topk(H->glog, L.router_b, H->ids, H->wts, Tn, c.n_experts, c.top_k, H->stream);
+      launch_router_permute(H->ids, Tn * c.top_k, c.n_experts, grouped_tile(H, Tn), H->cnt, H->off, H->perm,
+                            H->work, H->n_work, H->touched + l, H->stream);
+    }
+    {
+      ProfScope ps(H, PC_GATHER);
+      launch_gather_rows<T>(xn, H->perm, (T*)H->xp, Tn * c.top_k, c.top_k, c.d_model, H->stream);
+    }
+    moe_gemms(H, l, Tn);
+    {
+      ProfScope ps(H, PC_COMBINE);
+      const float* nw = (l + 1 < c.n_layers) ? H->lw[l + 1].attn_norm : (head ? H->final_norm : nullptr);
+      if (hidden_out && l + 1 == c.n_layers) nw = nullptr;
+      launch_combine<T>(H->h, H->y, H->wts, c.top_k, nw, xn, Tn, c.d_model, eps, H->stream);
+    }
+  }
+  if (hidden_out) {
+    cudaMemcpyAsync(hidden_out, H->h, (size_t)Tn * c.d_model * sizeof(float), cudaMemcpyDeviceToDevice, H->stream);
+    if (head) {
+      ProfScope ps(H, PC_NORM);
+      launch_rmsnorm<T>(H->h, H->final_norm, xn, Tn, c.d_model, eps, H->stream);
+    }
+  }
+  if (head) dense_gemm(H, PC_LMHEAD, H->xn, &H->m_xn, H->embed, &H->m_embed, Tn, c.vocab, c.d_model, EPI_STORE_F32,
+                       logits, c.vocab);
+}
+
+void run_layers(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const int32_t* tokens, const int32_t* prev,
+                bool head, float* logits, float* hidden_out) {
+  if (H->bf16) run_layers_t<__nv_bfloat16>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out);
+  else run_layers_t<float>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out);
+}
+
+int make_batch(dg_handle* H, int batch, const int* req, BatchInfo* bi) {
+  if (batch < 1 || batch > H->c.max_batch || !req) return fail(H, DG_EINVAL, "batch %d out of range [1,%d]", batch,
+                                                               H->c.max_batch);
+  bi->B = batch;
+  for (int b = 0; b < batch; ++b) {
+    if (req[b] < 0 || req[b] >= H->c.max_batch) return fail(H, DG_EINVAL, "request slot %d out of range", req[b]);
+    for (int x = 0; x < b; ++x)
+      if (req[x] == req[b]) return fail(H, DG_EINVAL, "request slot %d repeated in a batch", req[b]);
+    bi->slot[b] = req[b];
+    bi->len[b] = H->len[req[b]];
+  }
+  return DG_OK;
+}
+
+int upload_req(dg_handle* H, const BatchInfo& bi) {
+  int32_t tmp[kMaxBatch];
+  for (int b = 0; b < bi.B; ++b) tmp[b] = bi.slot[b];
+  // pageable copy: the staging buffer is on the stack, so the runtime copies synchronously
+  return cuda_check(H, cudaMemcpyAsync(H->req_dev, tmp, bi.B * sizeof(int32_t), cudaMemcpyHostToDevice, H->stream),
+                    "upload request ids");
+}
+
+int check_launch(dg_handle* H, const char* what) {
+  return cuda_check(H, cudaGetLastError(), what);
+}
+
+SamplerArgs sampler_args(const dg_sampler_params& sp, int step) {
+  SamplerArgs a;
+  a.temperature = sp.temperature;
+  a.logit_scale = sp.logit_scale;
+  a.stop_threshold = sp.stop_threshold;
+  a.keep_k = sp.keep_k;
+  a.seed = sp.seed;
+  a.block = sp.block;
+  a.step = (uint32_t)step;
+  return a;
+}
+
+int check_sampler_params(dg_handle* H, const dg_sampler_params* sp) {
+  if (!sp) return fail(H, DG_EINVAL, "null sampler params");
+  if (!(sp->temperature >= 0.f) || !std::isfinite(sp->temperature))
+    return fail(H, DG_EINVAL, "temperature must be finite and >= 0");
+  if (!(sp->logit_scale > 0.f) || !std::isfinite(sp->logit_scale)) return fail(H, DG_EINVAL, "logit_scale must be > 0");
+  if (sp->keep_k < 0 || sp->keep_k > H->c.canvas) return fail(H, DG_EINVAL, "keep_k out of [0, N]");
+  return DG_OK;
+}
+
+// sampler over logits rows of the batch, then keep / re-noise / stop
+void run_sampler(dg_handle* H, const float* logits, const BatchInfo& bi, const SamplerArgs& a, int32_t* canvas,
+                 int32_t* xh, float* pmax, float* ent, int32_t* keep, float* meanh, int32_t* stop, int32_t* done,
+                 int32_t* out_tokens, int final_step) {
+  const int n = H->c.canvas;
+  {
+    ProfScope ps(H, PC_SAMPLER, 2);
+    launch_sampler_rows(logits, bi.B * n, n, H->c.vocab, H->req_dev, a, H->sws, xh, pmax, ent, H->stream);
+  }
+  {
+    ProfScope ps(H, PC_FINISH);
+    launch_sampler_finish(xh, pmax, ent, bi.B, n, H->c.vocab, H->req_dev, a, canvas, keep, meanh, stop, done,
+                          out_tokens, final_step, H->stream);
+  }
+}
+
+int read_device_error(dg_handle* H) {
+  int e = 0;
+  if (cudaMemcpy(&e, H->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail(H, DG_ECUDA, "reading the device error flag: %s", cudaGetErrorString(cudaGetLastError()));
+  if (e != 0) {
+    cudaMemset(H->d_err, 0, sizeof(int));
+    if (e == 5) return fail(H, DG_EINVAL, "a token outside [0, vocab) reached the embedding (replaced by 0)");
+    return fail(H, DG_ETIMEOUT, "a bounded device wait gave up (code %d)", e);
+  }
+  return DG_OK;
+}
+
+int encode_causal(dg_handle* H, const BatchInfo& bi0, const int32_t* tokens, int n, int src_pitch) {
+  // chunked causal encode: B * chunk <= T_max
+  BatchInfo bi = bi0;
+  const int chunk = std::max(1, std::min(n, H->T_max / bi.B));
+  for (int p0 = 0; p0 < n; p0 += chunk) {
+    const int m = std::min(chunk, n - p0);
+    if (cudaMemcpy2DAsync(H->tok_ws, m * sizeof(int32_t), tokens + p0, src_pitch * sizeof(int32_t),
+                          m * sizeof(int32_t), bi.B, cudaMemcpyDeviceToDevice, H->stream) != cudaSuccess)
+      return fail(H, DG_ECUDA, "token staging copy failed");
+    run_layers(H, bi, m, true, H->tok_ws, nullptr, false, nullptr, nullptr);
+    int rc = check_launch(H, "causal encode");
+    if (rc) return rc;
+    for (int b = 0; b < bi.B; ++b) {
+      bi.len[b] += m;
+      H->len[bi.slot[b]] += m;
+    }
+  }
+  return DG_OK;
+}
+
+}  // namespace
+
+// ======================================================================= ABI
+
+extern "C" {
+
+const char* dg_last_error(const dg_handle* h) { return h ? h->err.c_str() : g_create_error.c_str(); }
+
+int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle** out) {
+  g_create_error.clear();
+  if (!cfg || !out) return fail(nullptr, DG_EINVAL, "null config or output pointer");
+  *out = nullptr;
+  const dg_config& c = *cfg;
+  if (c.dtype != DG_FP32 && c.dtype != DG_BF16) return fail(nullptr, DG_EINVAL, "dtype must be DG_FP32 or DG_BF16");
+  if (c.n_layers < 0 || c.canvas < 1 || c.canvas > 1024 || c.vocab < 1 || c.max_batch < 1 ||
+      c.max_batch > kMaxBatch)
+    return fail(nullptr, DG_EINVAL, "bad layers/canvas/vocab/max_batch");
+  const bool model = c.n_layers > 0;
+  if (model) {
+    if (c.d_model < 1 || c.n_heads < 1 || c.n_kv_heads < 1 || c.n_heads % c.n_kv_heads || c.head_dim < 2 ||
+        c.head_dim % 2 || c.head_dim > 256 || c.n_experts < 1 || c.n_experts > 256 || c.top_k < 1 ||
+        c.top_k > 16 || c.top_k > c.n_experts || c.d_ff < 1)
+      return fail(nullptr, DG_EINVAL, "bad model shape");
+    if (8 % (c.n_heads / c.n_kv_heads) != 0) return fail(nullptr, DG_EINVAL, "Hq/Hkv must divide 8");
+    if (c.max_ctx < c.canvas || c.max_ctx % 64) return fail(nullptr, DG_EINVAL, "max_ctx must be a multiple of 64 >= canvas");
+    if (!(c.rms_eps > 0) || !(c.rope_base > 1)) return fail(nullptr, DG_EINVAL, "bad rms_eps / rope_base");
+    if (c.dtype == DG_BF16 && (c.d_model % 64 || c.d_ff % 64 || c.head_dim % 64))
+      return fail(nullptr, DG_EINVAL, "bf16 needs d_model, d_ff, head_dim multiples of 64");
+    if (!w || !w->embed || !w->w_sc || !w->final_norm || !w->layers)
+      return fail(nullptr, DG_EINVAL, "null weight pointer");
+    for (int l = 0; l < c.n_layers; ++l) {
+      const dg_layer_weights& L = w->layers[l];
+      const void* ps[] = {L.attn_norm, L.wq, L.wk, L.wv, L.wo, L.ffn_norm, L.router_w, L.w_gate, L.w_up, L.w_down};
+      for (const void* p : ps)
+        if (!p || !aligned16(p)) return fail(nullptr, DG_EINVAL, "layer %d: null or unaligned weight", l);
+    }
+    if (!aligned16(w->embed) || !aligned16(w->w_sc)) return fail(nullptr, DG_EINVAL, "unaligned embed / w_sc");
+  }
+  dg_handle* H = new dg_handle();
+  H->c = c;
+  if (H->c.max_tokens <= 0) H->c.max_tokens = c.max_batch * c.canvas;
+  if (H->c.max_tokens < c.max_batch * c.canvas) {
+    delete H;
+    return fail(nullptr, DG_EINVAL, "max_tokens < max_batch * canvas");
+  }
+  H->bf16 = c.dtype == DG_BF16;
+  H->esz = H->bf16 ? 2 : 4;
+  H->stream = (cudaStream_t)stream;
+  cudaGetDevice(&H->dev);
+  cudaDeviceGetAttribute(&H->num_sms, cudaDevAttrMultiProcessorCount, H->dev);
+  H->len.assign(c.max_batch, 0);
+  H->T_max = H->c.max_tokens;
+  bool ok = true;
+  const int T = H->T_max;
+  const int nrow = c.max_batch * c.canvas;
+  if (model) {
+    H->embed = w->embed;
+    H->w_sc = w->w_sc;
+    H->final_norm = w->final_norm;
+    H->lw.assign(w->layers, w->layers + c.n_layers);
+    const size_t kvn = kv_layer_elems(c) * c.n_layers;
+    H->kc = dalloc<char>(kvn * H->esz, &ok);
+    H->vt = dalloc<char>(kvn * H->esz, &ok);
+    const int qw = c.n_heads * c.head_dim;
+    const int ldqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+    H->h = dalloc<float>((size_t)T * c.d_model, &ok);
+    H->xn = dalloc<char>((size_t)T * c.d_model * H->esz, &ok);
+    H->eprev = dalloc<char>((size_t)T * c.d_model * H->esz, &ok);
+    H->qkv = dalloc<float>((size_t)T * ldqkv, &ok);
+    H->q = dalloc<char>((size_t)T * qw * H->esz, &ok);
+    H->attn = dalloc<char>((size_t)T * qw * H->esz, &ok);
+    H->glog = dalloc<float>((size_t)T * c.n_experts, &ok);
+    H->ids = dalloc<int32_t>((size_t)T * c.top_k, &ok);
+    H->wts = dalloc<float>((size_t)T * c.top_k, &ok);
+    H->cnt = dalloc<int32_t>(c.n_experts, &ok);
+    H->off = dalloc<int32_t>(c.n_experts + 1, &ok);
+    H->perm = dalloc<int32_t>((size_t)T * c.top_k, &ok);
+    H->n_work_max = c.n_experts + (T * c.top_k + 63) / 64;
+    H->work = dalloc<int32_t>((size_t)3 * H->n_work_max, &ok);
+    H->n_work = dalloc<int32_t>(1, &ok);
+    H->touched = dalloc<int32_t>(c.n_layers, &ok);
+    H->xp = dalloc<char>((size_t)T * c.top_k * c.d_model * H->esz, &ok);
+    H->hb = dalloc<char>((size_t)T * c.top_k * c.d_ff * H->esz, &ok);
+    H->y = dalloc<float>((size_t)T * c.top_k * c.d_model, &ok);
+    H->logits = dalloc<float>((size_t)nrow * c.vocab, &ok);
+    H->rope = dalloc<float2>((size_t)c.max_ctx * (c.head_dim / 2), &ok);
+    H->tok_ws = dalloc<int32_t>((size_t)T, &ok);
+  }
+  H->sws = dalloc<char>(sampler_workspace_bytes(nrow, c.vocab), &ok);
+  H->xh[0] = dalloc<int32_t>(nrow, &ok);
+  H->xh[1] = dalloc<int32_t>(nrow, &ok);
+  H->pmax = dalloc<float>(nrow, &ok);
+  H->ent = dalloc<float>(nrow, &ok);
+  H->keep = dalloc<int32_t>(nrow, &ok);
+  H->meanh = dalloc<float>(c.max_batch, &ok);
+  H->stop = dalloc<int32_t>(c.max_batch, &ok);
+  H->done = dalloc<int32_t>(c.max_batch, &ok);
+  H->canvas = dalloc<int32_t>(nrow, &ok);
+  H->out_tok = dalloc<int32_t>(nrow, &ok);
+  H->req_dev = dalloc<int32_t>(c.max_batch, &ok);
+  H->d_err = dalloc<int>(1, &ok);
+  if (cudaMallocHost(&H->h_done, c.max_batch * sizeof(int32_t)) != cudaSuccess) ok = false;
+  if (!ok) {
+    dg_destroy(H);
+    cudaGetLastError();
+    return fail(nullptr, DG_ENOMEM, "device allocation failed");
+  }
+  cudaMemset(H->d_err, 0, sizeof(int));
+  if (model) {
+    const size_t kvn = kv_layer_elems(c) * c.n_layers;
+    cudaMemset(H->kc, 0, kvn * H->esz);
+    cudaMemset(H->vt, 0, kvn * H->esz);
+    // RoPE table: (cos, sin) of pos * base^(-2j/hd), in double on the host
+    const int half = c.head_dim / 2;
+    std::vector<float2> tab((size_t)c.max_ctx * half);
+    for (int p = 0; p < c.max_ctx; ++p)
+      for (int j = 0; j < half; ++j) {
+        const double th = std::pow(c.rope_base, -2.0 * j / c.head_dim);
+        const double ang = (double)p * th;
+        tab[(size_t)p * half + j] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      }
+    cudaMemcpy(H->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+    if (H->bf16) {
+      const int d = c.d_model, F = c.d_ff, E = c.n_experts;
+      const int qw = c.n_heads * c.head_dim, kw = c.n_kv_heads * c.head_dim;
+      bool tm = true;
+      H->lmaps.resize(c.n_layers);
+      for (int l = 0; l < c.n_layers; ++l) {
+        const dg_layer_weights& L = H->lw[l];
+        LayerMaps& M = H->lmaps[l];
+        tm &= tmap_2d(&M.wq, L.wq, d, qw, d, 128);
+        tm &= tmap_2d(&M.wk, L.wk, d, kw, d, 128);
+        tm &= tmap_2d(&M.wv, L.wv, d, kw, d, 128);
+        tm &= tmap_2d(&M.wo, L.wo, qw, d, qw, 128);
+        tm &= tmap_2d(&M.router, L.router_w, d, E, d, 128);
+        tm &= tmap_3d(&M.gate, L.w_gate, d, F, E, 128);
+        tm &= tmap_3d(&M.up, L.w_up, d, F, E, 128);
+        tm &= tmap_3d(&M.down, L.w_down, F, d, E, 128);
+      }
+      tm &= tmap_2d(&H->m_embed, H->embed, d, c.vocab, d, 128);
+      tm &= tmap_2d(&H->m_wsc, H->w_sc, d, d, d, 128);
+      H->m_dummy = H->m_wsc;
+      tm &= tmap_2d(&H->m_xn, H->xn, d, T, d, 32);
+      tm &= tmap_2d(&H->m_eprev, H->eprev, d, T, d, 32);
+      tm &= tmap_2d(&H->m_attn, H->attn, qw, T, qw, 32);
+      tm &= tmap_2d(&H->m_xp, H->xp, d, (uint64_t)T * c.top_k, d, 32);
+      tm &= tmap_2d(&H->m_hb, H->hb, F, (uint64_t)T * c.top_k, F, 32);
+      if (!tm) {
+        dg_destroy(H);
+        return fail(nullptr, DG_ECUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
+      }
+    }
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    const char* m = cudaGetErrorString(cudaGetLastError());
+    dg_destroy(H);
+    return fail(nullptr, DG_ECUDA, "create: %s", m);
+  }
+  *out = H;
+  return DG_OK;
+}
+
+void dg_destroy(dg_handle* H) {
+  if (!H) return;
+  if (H->stream || true) cudaStreamSynchronize(H->stream);
+  void* ps[] = {H->kc, H->vt, H->h, H->xn, H->eprev, H->qkv, H->q, H->attn, H->glog, H->ids, H->wts, H->cnt,
+                H->off, H->perm, H->work, H->n_work, H->touched, H->xp, H->hb, H->y, H->logits, H->rope, H->sws,
+                H->xh[0], H->xh[1], H->pmax, H->ent, H->keep, H->meanh, H->stop, H->done, H->canvas, H->out_tok,
+                H->req_dev, H->tok_ws, H->d_err};
+  for (void* p : ps)
+    if (p) cudaFree(p);
+  if (H->h_done) cudaFreeHost(H->h_done);
+  for (cudaEvent_t e : H->pool) cudaEventDestroy(e);
+  delete H;
+}
+
+int dg_set_length(dg_handle* H, int req, int length) {
+  if (!H) return DG_EINVAL;
+  if (req < 0 || req >= H->c.max_batch) return fail(H, DG_EINVAL, "request slot out of range");
+  if (length < 0 || length > H->c.max_ctx) return fail(H, DG_ECAPACITY, "length %d exceeds max_ctx", length);
+  H->len[req] = length;
+  return DG_OK;
+}
+
+int dg_get_length(const dg_handle* H, int req, int* length) {
+  if (!H || !length || req < 0 || req >= H->c.max_batch) return DG_EINVAL;
+  *length = H->len[req];
+  return DG_OK;
+}
+
+int dg_set_kv(dg_handle* H, int req, int layer, const void* k, const void* v, int n) {
+  if (!H) return DG_EINVAL;
+  const dg_config& c = H->c;
+  if (c.n_layers == 0) return fail(H, DG_ESTATE, "sampler-only handle");
+  if (req < 0 || req >= c.max_batch || layer < 0 || layer >= c.n_layers || !k || !v || n < 0)
+    return fail(H, DG_EINVAL, "bad set_kv arguments");
+  if (n > c.max_ctx) return fail(H, DG_ECAPACITY, "n exceeds max_ctx");
+  const size_t slot_off = (size_t)req * c.n_kv_heads * c.max_ctx * c.head_dim * H->esz;
+  char* kc = (char*)kc_layer(H, layer) + slot_off;
+  char* vt = (char*)vt_layer(H, layer) + slot_off;
+  if (H->bf16)
+    launch_set_kv<__nv_bfloat16>((const __nv_bfloat16*)k, (const __nv_bfloat16*)v, (__nv_bfloat16*)kc,
+                                 (__nv_bfloat16*)vt, c.n_kv_heads, n, c.head_dim, c.max_ctx, H->stream);
+  else
+    launch_set_kv<float>((const float*)k, (const float*)v, (float*)kc, (float*)vt, c.n_kv_heads, n, c.head_dim,
+                         c.max_ctx, H->stream);
+  H->launches += 1;
+  return check_launch(H, "set_kv");
+}
+
+int dg_prefill_prompt(dg_handle* H, int batch, const int* req, const int32_t* tokens, int n) {
+  if (!H) return DG_EINVAL;
+  if (H->c.n_layers == 0) return fail(H, DG_ESTATE, "sampler-only handle");
+  if (!tokens || n < 0) return fail(H, DG_EINVAL, "bad tokens");
+  BatchInfo bi;
+  int rc = make_batch(H, batch, req, &bi);
+  if (rc) return rc;
+  for (int b = 0; b < batch; ++b)
+    if (bi.len[b] + n > H->c.max_ctx) return fail(H, DG_ECAPACITY, "prefill of %d exceeds max_ctx", n);
+  if (n == 0) return DG_OK;
+  return encode_causal(H, bi, tokens, n, n);
+}
+
+int dg_sample(dg_handle* H, const float* logits, int batch, const int* req, int step, const dg_sampler_params* sp,
+              int32_t* canvas, const dg_step_out* o) {
+  if (!H) return DG_EINVAL;
+  BatchInfo bi;
+  int rc = make_batch(H, batch, req, &bi);
+  if (rc) return rc;
+  if ((rc = check_sampler_params(H, sp))) return rc;
+  if (!logits || !canvas) return fail(H, DG_EINVAL, "null logits or canvas");
+  if ((rc = upload_req(H, bi))) return rc;
+  const SamplerArgs a = sampler_args(*sp, step);
+  run_sampler(H, logits, bi, a, canvas, (o && o->x_hat) ? o->x_hat : H->xh[0], (o && o->pmax) ? o->pmax : H->pmax,
+              (o && o->entropy) ? o->entropy : H->ent, o ? o->keep : nullptr, o ? o->mean_entropy : nullptr,
+              o ? o->stop : nullptr, nullptr, nullptr, 0);
+  return check_launch(H, "sample");
+}
+
+int dg_denoise_step(dg_handle* H, const dg_step_args* a, const dg_step_out* o) {
+  if (!H || !a) return DG_EINVAL;
+  const dg_config& c = H->c;
+  if (c.n_layers == 0) return fail(H, DG_ESTATE, "sampler-only handle");
+  BatchInfo bi;
+  int rc = make_batch(H, a->batch, a->req, &bi);
+  if (rc) return rc;
+  if ((rc = check_sampler_params(H, &a->sp))) return rc;
+  if (!a->canvas) return fail(H, DG_EINVAL, "null canvas");
+  if (a->step < 1) return fail(H, DG_EINVAL, "step must be >= 1");
+  for (int b = 0; b < bi.B; ++b)
+    if (bi.len[b] + c.canvas > c.max_ctx) return fail(H, DG_ECAPACITY, "cache + canvas exceeds max_ctx");
+  if ((rc = upload_req(H, bi))) return rc;
+  float* logits = a->logits_out ? a->logits_out : H->logits;
+  run_layers(H, bi, c.canvas, false, a->canvas, a->prev_pred, true, logits, a->hidden_out);
+  const SamplerArgs sa = sampler_args(a->sp, a->step);
+  run_sampler(H, logits, bi, sa, a->canvas, (o && o->x_hat) ? o->x_hat : H->xh[0],
+              (o && o->pmax) ? o->pmax : H->pmax, (o && o->entropy) ? o->entropy : H->ent, o ? o->keep : nullptr,
+              o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0);
+  if (o && o->experts_touched)
+    cudaMemcpyAsync(o->experts_touched, H->touched, c.n_layers * sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                    H->stream);
+  return check_launch(H, "denoise step");
+}
+
+static int generate_block_impl(dg_handle* H, const dg_block_args* a, int32_t* out_dev, int* steps_used) {
+  const dg_config& c = H->c;
+  if (c.n_layers == 0) return fail(H, DG_ESTATE, "sampler-only handle");
+  BatchInfo bi;
+  int rc = make_batch(H, a->batch, a->req, &bi);
+  if (rc) return rc;
+  if (a->max_steps < 1 || a->schedule_steps < 1) return fail(H, DG_EINVAL, "max_steps and schedule_steps must be >= 1");
+  if (!(a->temperature >= 0.f) || !(a->logit_scale_growth > 0.f)) return fail(H, DG_EINVAL, "bad temperature / growth");
+  for (int b = 0; b < bi.B; ++b)
+    if (bi.len[b] + c.canvas > c.max_ctx) return fail(H, DG_ECAPACITY, "cache + canvas exceeds max_ctx");
+  if ((rc = upload_req(H, bi))) return rc;
+  const int n = c.canvas;
+  {
+    ProfScope ps(H, PC_FINISH);
+    launch_init_canvas(H->canvas, bi, H->req_dev, n, c.vocab, a->seed, a->block, H->stream);
+  }
+  cudaMemsetAsync(H->done, 0, bi.B * sizeof(int32_t), H->stream);
+  const int32_t* prev = nullptr;
+  int steps = 0;
+  for (int t = 1; t <= a->max_steps; ++t) {
+    dg_sampler_params sp;
+    sp.temperature = a->temperature;
+    sp.logit_scale = (float)std::pow((double)a->logit_scale_growth, (double)(t - 1));
+    sp.stop_threshold = a->stop_threshold;
+    sp.keep_k = std::min(n, (int)(((long long)n * t + a->schedule_steps - 1) / a->schedule_steps));
+    sp.seed = a->seed;
+    sp.block = a->block;
+    run_layers(H, bi, n, false, H->canvas, prev, true, H->logits, nullptr);
+    int32_t* xh = H->xh[t & 1];
+    run_sampler(H, H->logits, bi, sampler_args(sp, t), H->canvas, xh, H->pmax, H->ent, H->keep, H->meanh, H->stop,
+                H->done, out_dev, t == a->max_steps ? 1 : 0);
+    if ((rc = check_launch(H, "block step"))) return rc;
+    steps = t;
+    cudaMemcpyAsync(H->h_done, H->done, bi.B * sizeof(int32_t), cudaMemcpyDeviceToHost, H->stream);
+    if ((rc = cuda_check(H, cudaStreamSynchronize(H->stream), "block step sync"))) return rc;
+    if ((rc = read_device_error(H))) return rc;
+    bool all = true;
+    for (int b = 0; b < bi.B; ++b) all &= H->h_done[b] != 0;
+    if (all) break;
+    prev = xh;
+  }
+  // causal hand-off of the finished block into the cache ([P2 架构基础], [P3])
+  if ((rc = encode_causal(H, bi, out_dev, n, n))) return rc;
+  if (steps_used) *steps_used = steps;
+  return DG_OK;
+}
+
+int dg_generate_block(dg_handle* H, const dg_block_args* a, int32_t* out_tokens, int* steps_used) {
+  if (!H || !a || !out_tokens) return H ? fail(H, DG_EINVAL, "null argument") : DG_EINVAL;
+  return generate_block_impl(H, a, out_tokens, steps_used);
+}
+
+int dg_generate_block_host(dg_handle* H, const dg_block_args* a, int32_t* out_tokens_host, int* steps_used) {
+  if (!H || !a || !out_tokens_host) return H ? fail(H, DG_EINVAL, "null argument") : DG_EINVAL;
+  int rc = generate_block_impl(H, a, H->out_tok, steps_used);
+  if (rc) return rc;
+  rc = cuda_check(H,
+                  cudaMemcpyAsync(out_tokens_host, H->out_tok, (size_t)a->batch * H->c.canvas * sizeof(int32_t),
+                                  cudaMemcpyDeviceToHost, H->stream),
+                  "copy tokens to host");
+  if (rc) return rc;
+  return cuda_check(H, cudaStreamSynchronize(H->stream), "sync");
+}
+
+int dg_synchronize(dg_handle* H) {
+  if (!H) return DG_EINVAL;
+  int rc = cuda_check(H, cudaStreamSynchronize(H->stream), "synchronize");
+  if (rc) return rc;
+  return read_device_error(H);
+}
+
+uint64_t dg_launch_count(const dg_handle* H) { return H ? H->launches : 0; }
+
+int dg_profile_enable(dg_handle* H, int on) {
+  if (!H) return DG_EINVAL;
+  H->prof = on != 0;
+  return DG_OK;
+}
+
+int dg_profile_reset(dg_handle* H) {
+  if (!H) return DG_EINVAL;
+  cudaStreamSynchronize(H->stream);
+  H->recs.clear();
+  H->pool_used = 0;
+  return DG_OK;
+}
+
+int dg_profile_read(dg_handle* H, dg_profile_entry* out, int max_entries, int* n_entries) {
+  if (!H || !n_entries) return DG_EINVAL;
+  int rc = cuda_check(H, cudaStreamSynchronize(H->stream), "profile sync");
+  if (rc) return rc;
+  double ms[PC_COUNT] = {0};
+  int cnt[PC_COUNT] = {0};
+  for (const auto& r : H->recs) {
+    float t = 0.f;
+    cudaEventElapsedTime(&t, r.a, r.b);
+    ms[r.cls] += t;
+    cnt[r.cls] += 1;
+  }
+  int n = 0;
+  for (int k = 0; k < PC_COUNT; ++k) {
+    if (cnt[k] == 0) continue;
+    if (out && n < max_entries) {
+      out[n].name = kProfNames[k];
+      out[n].launches = cnt[k];
+      out[n].ms = ms[k];
+    }
+    ++n;
+  }
+  *n_entries = n;
+  return DG_OK;
+}
+
+int dg_selftest_philox(dg_handle* H, const uint32_t* ctr, const uint32_t* key, uint32_t* out, uint32_t* out_curand,
+                       int n) {
+  if (!H || !ctr || !key || !out || n < 0) return DG_EINVAL;
+  launch_philox_selftest(ctr, key, out, out_curand, n, H->stream);
+  H->launches += 1;
+  return check_launch(H, "philox selftest");
+}
+
+int dg_selftest_gemm(dg_handle* H, const void* x, const void* w, int T, int M, int K, float* out) {
+  if (!H || !x || !w || !out || T < 1 || M < 1 || K < 64 || K % 64) return H ? fail(H, DG_EINVAL, "bad gemm args") : DG_EINVAL;
+  if (!aligned16(x) || !aligned16(w)) return fail(H, DG_EINVAL, "unaligned operands");
+  CUtensorMap mx, mw;
+  if (!tmap_2d(&mx, x, K, T, K, 32) || !tmap_2d(&mw, w, K, M, K, 128))
+    return fail(H, DG_ECUDA, "tensor map encode failed");
+  TcGemm g{};
+  g.mode = 0;
+  g.M = M;
+  g.K = K;
+  g.T = T;
+  g.ntile = pick_ntile((M + 127) / 128, T, H->num_sms);
+  g.seg1 = g.seg2 = INT_MAX;
+  g.epi = EPI_STORE_F32;
+  g.out = out;
+  g.ld_out = M;
+  g.err = H->d_err;
+  launch_gemm_tc(mw, mw, mw, mx, g, H->num_sms, H->stream);
+  H->launches += 1;
+  return check_launch(H, "selftest gemm");
+}
+
+}  // extern "C"

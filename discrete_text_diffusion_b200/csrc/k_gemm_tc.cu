@@ -1,0 +1,297 @@
+// tcgen05 GEMM for the bf16 model: out[token, m] = sum_k W[m, k] * X[token, k].
+//
+// The weight matrix is the 128-row M operand and the tokens are the N
+// operand (N = 32..256 per tile).  A canvas step has few tokens per expert
+// ([P1 五]: 256 tokens spread over ~84-128 experts), so putting the weights on
+// the M side keeps the tensor-core tile full while each weight tile streams
+// from HBM once per token tile.
+//
+// Persistent kernel, 192 threads:
+//   warp 0  lane 0: TMA producer (weights 128x64 + tokens Nx64 per stage,
+//           128-byte swizzle) into a ring of shared-memory stages
+//   warp 1  lane 0: issues tcgen05.mma (M=128, N, K=16) into a TMEM
+//           accumulator; tcgen05.commit frees stages / signals the epilogue
+//   warps 2-5: epilogue, each reading its 32-lane quarter of TMEM
+// Accumulators are double-buffered in TMEM when they fit, so the epilogue of
+// one tile overlaps the main loop of the next.
+//
+// Modes:
+//   0 dense: up to three weight maps stacked along M (the Q | K | V
+//     projections); epilogue store fp32, add fp32 (residual), or store bf16.
+//   1 grouped up: per work item (expert e, row0, rows) the gate and the up
+//     weights of expert e both multiply the same token tile into two
+//     accumulators; the epilogue writes silu(gate) * up as bf16.
+//   2 grouped down: expert e's down projection; the epilogue writes row r to
+//     out[row_map[r]] (the token-slot order), fp32.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "dg_common.cuh"
+#include "kernels.h"
+
+namespace dg {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kBoxN = 32;
+constexpr int kTcThreads = 192;
+constexpr int kABytes = kBM * kBK * 2;  // 16 KB
+constexpr int kMaxSmem = 232448;        // 227 KB opt-in limit per CTA
+
+struct TcLayout {
+  int n_a;          // weight operands per stage (1 or 2)
+  int stage_bytes;
+  int stages;
+  int acc_cols;     // TMEM columns of one accumulator buffer (all operands)
+  int n_acc_buf;
+  int tmem_cols;    // power of two >= 32
+  int smem_bytes;
+};
+
+static TcLayout tc_layout(const TcGemm& p) {
+  TcLayout L;
+  L.n_a = (p.mode == 1) ? 2 : 1;
+  L.stage_bytes = L.n_a * kABytes + p.ntile * kBK * 2;
+  const int overhead = 1024 /*align*/ + 1024 /*barriers*/;
+  L.stages = std::min(8, (kMaxSmem - overhead) / L.stage_bytes);
+  L.acc_cols = L.n_a * p.ntile;
+  L.n_acc_buf = (2 * L.acc_cols <= 512) ? 2 : 1;
+  int need = L.n_acc_buf * L.acc_cols;
+  L.tmem_cols = 32;
+  while (L.tmem_cols < need) L.tmem_cols <<= 1;
+  L.smem_bytes = overhead + L.stages * L.stage_bytes;
+  return L;
+}
+
+int gemm_tc_smem_bytes(const TcGemm& p, int* stages) {
+  TcLayout L = tc_layout(p);
+  if (stages) *stages = L.stages;
+  return L.smem_bytes;
+}
+
+struct TcKParams {
+  TcGemm g;
+  int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, n_ttiles;
+};
+
+__device__ __forceinline__ void tc_item(const TcKParams& P, int item, int& m0, int& e, int& row0, int& rows) {
+  const TcGemm& g = P.g;
+  if (g.mode == 0) {
+    const int tt = item % P.n_ttiles, mt = item / P.n_ttiles;
+    m0 = mt * kBM;
+    e = 0;
+    row0 = tt * g.ntile;
+    rows = min(g.ntile, g.T - row0);
+  } else {
+    const int mt = item % P.n_mtiles, w = item / P.n_mtiles;
+    m0 = mt * kBM;
+    e = g.work[3 * w];
+    row0 = g.work[3 * w + 1];
+    rows = g.work[3 * w + 2];
+  }
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap ta1,
+                   const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb,
+                   const TcKParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const TcGemm& g = P.g;
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* stage0 = base;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + P.stages * P.stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + P.stages;
+  uint64_t* acc_full = bars + 2 * P.stages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* err = g.err;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P.stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, (uint32_t)P.tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&ta0);
+    prefetch_tmap(&tb);
+    if (g.mode == 1) prefetch_tmap(&ta1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles : (*g.n_work) * P.n_mtiles;
+  const int nk = g.K / kBK;
+  const int n_a = (g.mode == 1) ? 2 : 1;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t kiter = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+      int m0, e, row0, rows;
+      tc_item(P, item, m0, e, row0, rows);
+      const int nb = (rows + kBoxN - 1) / kBoxN;
+      const uint32_t tx = (uint32_t)(n_a * kABytes + nb * kBoxN * kBK * 2);
+      const CUtensorMap* am = &ta0;
+      int am0 = m0;
+      if (g.mode == 0) {
+        if (m0 >= g.seg2) { am = &ta2; am0 = m0 - g.seg2; }
+        else if (m0 >= g.seg1) { am = &ta1; am0 = m0 - g.seg1; }
+      }
+      for (int kb = 0; kb < nk; ++kb, ++kiter) {
+        const int s = kiter % P.stages;
+        const uint32_t ph = (kiter / P.stages) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
+        uint8_t* st = stage0 + (size_t)s * P.stage_bytes;
+        mbar_expect_tx(&full[s], tx);
+        if (g.mode == 0) {
+          tma_load_2d(st, am, &full[s], kb * kBK, am0);
+        } else {
+          tma_load_3d(st, &ta0, &full[s], kb * kBK, m0, e);
+          if (g.mode == 1) tma_load_3d(st + kABytes, &ta1, &full[s], kb * kBK, m0, e);
+        }
+        uint8_t* sb = st + n_a * kABytes;
+        for (int i = 0; i < nb; ++i) tma_load_2d(sb + i * kBoxN * kBK * 2, &tb, &full[s], kb * kBK, row0 + i * kBoxN);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t kiter = 0;
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++it) {
+      int m0, e, row0, rows;
+      tc_item(P, item, m0, e, row0, rows);
+      const int n_mma = (rows + 15) & ~15;
+      const uint32_t idesc = idesc_bf16(kBM, n_mma);
+      const int ab = it % P.n_acc_buf;
+      const uint32_t use = (uint32_t)(it / P.n_acc_buf);
+      if (!mbar_wait(&acc_empty[ab], (use & 1u) ^ 1u, err, kErrTimeoutMma)) break;
+      tc_fence_after();
+      const uint32_t d0 = tmem_base + (uint32_t)(ab * P.acc_cols);
+      for (int kb = 0; kb < nk; ++kb, ++kiter) {
+        const int s = kiter % P.stages;
+        const uint32_t ph = (kiter / P.stages) & 1u;
+        if (!mbar_wait(&full[s], ph, err, kErrTimeoutMma)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(stage0 + (size_t)s * P.stage_bytes);
+        const uint32_t sb = sa + (uint32_t)(n_a * kABytes);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          const uint64_t bdesc = sdesc_k_sw128(sb + 32u * k);
+          const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+          umma_bf16(d0, sdesc_k_sw128(sa + 32u * k), bdesc, idesc, acc);
+          if (n_a == 2) umma_bf16(d0 + (uint32_t)g.ntile, sdesc_k_sw128(sa + kABytes + 32u * k), bdesc, idesc, acc);
+        }
+        umma_commit(&empty[s]);
+      }
+      if (!ok) break;
+      umma_commit(&acc_full[ab]);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;
+    int it = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
+      int m0, e, row0, rows;
+      tc_item(P, item, m0, e, row0, rows);
+      const int ab = it % P.n_acc_buf;
+      const uint32_t use = (uint32_t)(it / P.n_acc_buf);
+      if (!mbar_wait(&acc_full[ab], use & 1u, err, kErrTimeoutEpi)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * P.acc_cols);
+      const int m = m0 + r;
+      const bool mvalid = m < g.M;
+      for (int c0 = 0; c0 < rows; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tbase + (uint32_t)c0, v);
+        if (g.mode == 1) {
+          uint32_t u[32];
+          tmem_ld32(tbase + (uint32_t)(g.ntile + c0), u);
+          tmem_ld_wait();
+          if (mvalid) {
+            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c0 + j < rows) {
+                const float gt = __uint_as_float(v[j]), up = __uint_as_float(u[j]);
+                const float hv = gt / (1.f + expf(-gt)) * up;
+                o[(size_t)(row0 + c0 + j) * g.ld_out + m] = __float2bfloat16_rn(hv);
+              }
+            }
+          }
+        } else {
+          tmem_ld_wait();
+          if (mvalid) {
+            const float bv = g.bias ? g.bias[m] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c0 + j < rows) {
+                const float acc = __uint_as_float(v[j]) + bv;
+                if (g.mode == 2) {
+                  const int orow = g.row_map[row0 + c0 + j];
+                  reinterpret_cast<float*>(g.out)[(size_t)orow * g.ld_out + m] = acc;
+                } else if (g.epi == EPI_STORE_F32) {
+                  reinterpret_cast<float*>(g.out)[(size_t)(row0 + c0 + j) * g.ld_out + m] = acc;
+                } else if (g.epi == EPI_ADD_F32) {
+                  reinterpret_cast<float*>(g.out)[(size_t)(row0 + c0 + j) * g.ld_out + m] += acc;
+                } else {
+                  reinterpret_cast<__nv_bfloat16*>(g.out)[(size_t)(row0 + c0 + j) * g.ld_out + m] =
+                      __float2bfloat16_rn(acc);
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, (uint32_t)P.tmem_cols);
+  }
+}
+
+void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
+                    const TcGemm& g, int num_sms, cudaStream_t s) {
+  const TcLayout L = tc_layout(g);
+  TcKParams P;
+  P.g = g;
+  P.stages = L.stages;
+  P.stage_bytes = L.stage_bytes;
+  P.acc_cols = L.acc_cols;
+  P.n_acc_buf = L.n_acc_buf;
+  P.tmem_cols = L.tmem_cols;
+  P.n_mtiles = (g.M + kBM - 1) / kBM;
+  P.n_ttiles = (g.mode == 0) ? (g.T + g.ntile - 1) / g.ntile : 0;
+  const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles : g.n_work_max * P.n_mtiles;
+  if (total <= 0) return;
+  static int attr_bytes = 0;
+  if (attr_bytes < L.smem_bytes) {
+    cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    attr_bytes = kMaxSmem;
+  }
+  int per_sm = std::max(1, std::min(kMaxSmem / L.smem_bytes, 512 / L.tmem_cols));
+  per_sm = std::min(per_sm, 2);
+  const int grid = std::min(total, num_sms * per_sm);
+  gemm_tc_kernel<<<grid, kTcThreads, L.smem_bytes, s>>>(a0, a1, a2, b, P);
+}
+
+}  // namespace dg

@@ -1,0 +1,137 @@
+// MoE router ([P1 二]: 128 experts, 8 per token; [P1 五]: ~84 distinct experts
+// touched per 256-token canvas): warp-level top-k of the gate logits with a
+// softmax over the selected k, then a deterministic counting sort of the
+// (token, slot) items into expert order, the tile work list for the grouped
+// expert GEMMs and the count of distinct experts touched.
+#include "dg_common.cuh"
+#include "kernels.h"
+
+namespace dg {
+
+// One warp per token.  Lane l holds experts l, l+32, ...; k rounds of a warp
+// arg-max with (value desc, id asc) ordering pick the top-k.
+__global__ void router_topk_kernel(const float* __restrict__ glog, const float* __restrict__ bias,
+                                   int32_t* __restrict__ ids, float* __restrict__ wts, int n_tok, int e, int k) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_tok) return;
+  constexpr int kPer = 8;  // E <= 256
+  float v[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int ex = lane + 32 * j;
+    v[j] = (ex < e) ? glog[(size_t)warp * e + ex] + (bias ? bias[ex] : 0.f) : -INFINITY;
+  }
+  float sel_v[16];
+  int sel_i[16];
+  for (int r = 0; r < k; ++r) {
+    // best local candidate (lowest id wins ties: j ascending = id ascending)
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int ex = lane + 32 * j;
+      if (ex < e && (v[j] > bv || (v[j] == bv && ex < bi))) { bv = v[j]; bi = ex; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    sel_v[r] = bv;
+    sel_i[r] = bi;
+    // remove the winner
+#pragma unroll
+    for (int j = 0; j < kPer; ++j)
+      if (lane + 32 * j == bi) v[j] = -INFINITY;
+  }
+  if (lane == 0) {
+    const float m = sel_v[0];
+    float s = 0.f;
+    for (int r = 0; r < k; ++r) s += expf(sel_v[r] - m);
+    for (int r = 0; r < k; ++r) {
+      ids[(size_t)warp * k + r] = sel_i[r];
+      wts[(size_t)warp * k + r] = expf(sel_v[r] - m) / s;
+    }
+  }
+}
+
+void launch_router_topk(const float* glog, const float* bias, int32_t* ids, float* wts, int n_tok, int e, int k,
+                        cudaStream_t s) {
+  if (n_tok <= 0) return;
+  const int threads = 256;
+  const int blocks = (n_tok * 32 + threads - 1) / threads;
+  router_topk_kernel<<<blocks, threads, 0, s>>>(glog, bias, ids, wts, n_tok, e, k);
+}
+
+// Single-CTA counting sort.  Items i = t*k + s in order; inside an expert the
+// position of an item is the number of earlier items (smaller i) with the same
+// expert, so tokens are ascending and the result needs no atomics in its order.
+__global__ void __launch_bounds__(1024) router_permute_kernel(const int32_t* __restrict__ ids, int n_items, int e,
+                                                             int tile, int32_t* __restrict__ cnt_out,
+                                                             int32_t* __restrict__ off_out,
+                                                             int32_t* __restrict__ perm, int32_t* __restrict__ work,
+                                                             int32_t* __restrict__ n_work,
+                                                             int32_t* __restrict__ touched) {
+  __shared__ int cnt[256];
+  __shared__ int off[257];
+  __shared__ int running[256];
+  __shared__ int wc[32][256];  // per-warp per-expert counts of the current chunk
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int x = tid; x < e; x += blockDim.x) { cnt[x] = 0; running[x] = 0; }
+  __syncthreads();
+  for (int i = tid; i < n_items; i += blockDim.x) atomicAdd(&cnt[ids[i]], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0, nt = 0, nw = 0;
+    for (int x = 0; x < e; ++x) {
+      off[x] = acc;
+      acc += cnt[x];
+      if (cnt[x] > 0) ++nt;
+      for (int r0 = 0; r0 < cnt[x]; r0 += tile) {
+        work[3 * nw + 0] = x;
+        work[3 * nw + 1] = off[x] + r0;
+        work[3 * nw + 2] = min(tile, cnt[x] - r0);
+        ++nw;
+      }
+    }
+    off[e] = acc;
+    *n_work = nw;
+    *touched = nt;
+  }
+  __syncthreads();
+  for (int x = tid; x < e; x += blockDim.x) cnt_out[x] = cnt[x];
+  for (int x = tid; x <= e; x += blockDim.x) off_out[x] = off[x];
+  for (int base = 0; base < n_items; base += blockDim.x) {
+    for (int x = tid; x < 32 * 256; x += blockDim.x) (&wc[0][0])[x] = 0;
+    __syncthreads();
+    const int i = base + tid;
+    const bool valid = i < n_items;
+    const int ex = valid ? ids[i] : -1 - lane;  // invalid lanes never match a real expert
+    const unsigned peers = __match_any_sync(0xffffffffu, ex);
+    const int lane_rank = __popc(peers & ((1u << lane) - 1u));
+    if (valid && lane_rank == 0) wc[w][ex] = __popc(peers);
+    __syncthreads();
+    // exclusive scan over warps, per expert; advance the running totals
+    for (int x = tid; x < e; x += blockDim.x) {
+      int acc = running[x];
+      for (int ww = 0; ww < 32; ++ww) {
+        const int c = wc[ww][x];
+        wc[ww][x] = acc;
+        acc += c;
+      }
+      running[x] = acc;
+    }
+    __syncthreads();
+    if (valid) perm[off[ex] + wc[w][ex] + lane_rank] = i;
+    __syncthreads();
+  }
+}
+
+void launch_router_permute(const int32_t* ids, int n_items, int e, int tile, int32_t* cnt, int32_t* off,
+                           int32_t* perm, int32_t* work, int32_t* n_work, int32_t* touched, cudaStream_t s) {
+  router_permute_kernel<<<1, 1024, 0, s>>>(ids, n_items, e, tile, cnt, off, perm, work, n_work, touched);
+}
+
+}  // namespace dg

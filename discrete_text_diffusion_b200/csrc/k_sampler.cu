@@ -1,0 +1,336 @@
+// The sampler ([P1 四]: confidence, entropy, keep the confident positions,
+// re-randomise the rest, adaptive stop on mean entropy; [P1 五]: a softmax over
+// the full ~262k vocabulary per canvas position).
+//
+// Pass 1 (HBM-bound): each CTA reduces one 4096-logit chunk of one row to
+// (max, sum exp(z-max), sum exp(z-max)(z-max)) with 128-bit loads.
+// Pass 2: one CTA per row merges the chunk partials in chunk order, derives
+// pmax and the entropy, and draws the inverse-CDF sample: the chunk holding
+// u*S is found from the partials and only that chunk is re-read and scanned
+// in vocabulary order.
+// Pass 3: one CTA per canvas ranks positions by pmax, keeps the top-k,
+// re-noises the rest with Philox, and forms the mean entropy / stop flag.
+#include <curand_kernel.h>
+
+#include "dg_common.cuh"
+#include "kernels.h"
+
+namespace dg {
+
+constexpr int kChunk = 4096;
+constexpr int kThreads = 256;
+constexpr int kPerThread = kChunk / kThreads;  // 16
+
+struct Partial {
+  float m;   // chunk max of z (T > 0) / of the scaled logit (T == 0)
+  float s;   // sum exp(z - m)              | T == 0: bits of the first arg-max index
+  float a;   // sum exp(z - m) * (z - m)    | T == 0: bits of the count of maxima
+  float pad;
+};
+
+size_t sampler_workspace_bytes(int rows, int vocab) {
+  const size_t n_chunks = (vocab + kChunk - 1) / kChunk;
+  return (size_t)rows * n_chunks * sizeof(Partial);
+}
+
+__device__ __forceinline__ void load_chunk(const float* __restrict__ row, int c0, int vocab, float scale,
+                                           float (&z)[kPerThread], bool vec4) {
+  if (vec4) {
+#pragma unroll
+    for (int r = 0; r < kPerThread / 4; ++r) {
+      const int j = c0 + (threadIdx.x + r * kThreads) * 4;
+      float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (j < vocab) v = __ldcs(reinterpret_cast<const float4*>(row + j));  // j+3 < vocab since vocab % 4 == 0
+      z[4 * r + 0] = (j < vocab) ? v.x * scale : -INFINITY;
+      z[4 * r + 1] = (j < vocab) ? v.y * scale : -INFINITY;
+      z[4 * r + 2] = (j < vocab) ? v.z * scale : -INFINITY;
+      z[4 * r + 3] = (j < vocab) ? v.w * scale : -INFINITY;
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < kPerThread; ++r) {
+      const int j = c0 + threadIdx.x + r * kThreads;
+      z[r] = (j < vocab) ? row[j] * scale : -INFINITY;
+    }
+  }
+}
+
+// vocabulary index of register r of this thread in the load pattern above
+__device__ __forceinline__ int reg_index(int c0, int r, bool vec4) {
+  return vec4 ? c0 + (threadIdx.x + (r >> 2) * kThreads) * 4 + (r & 3) : c0 + threadIdx.x + r * kThreads;
+}
+
+__global__ void __launch_bounds__(kThreads) sampler_pass1(const float* __restrict__ logits, int vocab, float scale,
+                                                          int argmax_mode, Partial* __restrict__ part) {
+  __shared__ float red_m[kThreads / 32];
+  __shared__ float red_s[kThreads / 32];
+  __shared__ float red_a[kThreads / 32];
+  __shared__ int red_i[kThreads / 32];
+  __shared__ int red_c[kThreads / 32];
+  const int c = blockIdx.x, row = blockIdx.y;
+  const int n_chunks = gridDim.x;
+  const int c0 = c * kChunk;
+  const bool vec4 = (vocab % 4) == 0;
+  float z[kPerThread];
+  load_chunk(logits + (size_t)row * vocab, c0, vocab, scale, z, vec4);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  float m = -INFINITY;
+#pragma unroll
+  for (int r = 0; r < kPerThread; ++r) m = fmaxf(m, z[r]);
+  m = warp_max(m);
+  if (lane == 0) red_m[w] = m;
+  __syncthreads();
+  m = red_m[0];
+#pragma unroll
+  for (int x = 1; x < kThreads / 32; ++x) m = fmaxf(m, red_m[x]);
+  Partial p;
+  if (argmax_mode) {
+    int idx = 0x7fffffff, cntm = 0;
+#pragma unroll
+    for (int r = 0; r < kPerThread; ++r)
+      if (z[r] == m) { idx = min(idx, reg_index(c0, r, vec4)); ++cntm; }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      idx = min(idx, __shfl_xor_sync(0xffffffffu, idx, o));
+      cntm += __shfl_xor_sync(0xffffffffu, cntm, o);
+    }
+    if (lane == 0) { red_i[w] = idx; red_c[w] = cntm; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int x = 1; x < kThreads / 32; ++x) { idx = min(idx, red_i[x]); cntm += red_c[x]; }
+      p.m = m;
+      p.s = __int_as_float(idx);
+      p.a = __int_as_float(cntm);
+      p.pad = 0.f;
+      part[(size_t)row * n_chunks + c] = p;
+    }
+    return;
+  }
+  float s = 0.f, a = 0.f;
+  if (m > -INFINITY) {
+#pragma unroll
+    for (int r = 0; r < kPerThread; ++r) {
+      const float d = z[r] - m;
+      const float e = expf(d);      // exp(-inf) = 0 for padding
+      s += e;
+      a += (e > 0.f) ? e * d : 0.f;
+    }
+  }
+  s = warp_sum(s);
+  a = warp_sum(a);
+  if (lane == 0) { red_s[w] = s; red_a[w] = a; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s = 0.f; a = 0.f;
+    for (int x = 0; x < kThreads / 32; ++x) { s += red_s[x]; a += red_a[x]; }
+    p.m = m; p.s = s; p.a = a; p.pad = 0.f;
+    part[(size_t)row * n_chunks + c] = p;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) sampler_pass2(const float* __restrict__ logits, int n, int vocab,
+                                                          float scale, int argmax_mode, const int* __restrict__ req_ids,
+                                                          uint64_t seed, uint32_t step, uint32_t block,
+                                                          const Partial* __restrict__ part, int32_t* __restrict__ x_hat,
+                                                          float* __restrict__ pmax, float* __restrict__ ent) {
+  __shared__ float sh_M, sh_S, sh_target, sh_P0;
+  __shared__ int sh_c;
+  __shared__ float scan[kThreads];
+  __shared__ int sh_pick;
+  __shared__ int sh_last;
+  const int row = blockIdx.x;
+  if (threadIdx.x == 0) sh_last = 0;
+  const int b = row / n, i = row - b * n;
+  const int n_chunks = (vocab + kChunk - 1) / kChunk;
+  const Partial* pr = part + (size_t)row * n_chunks;
+  if (argmax_mode) {
+    if (threadIdx.x == 0) {
+      float M = -INFINITY;
+      for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pr[c].m);
+      int idx = -1, cntm = 0;
+      for (int c = 0; c < n_chunks; ++c)
+        if (pr[c].m == M) {
+          if (idx < 0) idx = __float_as_int(pr[c].s);
+          cntm += __float_as_int(pr[c].a);
+        }
+      x_hat[row] = idx;
+      pmax[row] = 1.0f / (float)cntm;
+      ent[row] = logf((float)cntm);
+    }
+    return;
+  }
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pr[c].m);
+    float S = 0.f, A = 0.f;
+    for (int c = 0; c < n_chunks; ++c) {
+      const float f = expf(pr[c].m - M);
+      S += pr[c].s * f;
+      A += (pr[c].a + (pr[c].m - M) * pr[c].s) * f;
+    }
+    const Philox4 w = sampler_words(seed, (uint32_t)i, step, block, (uint32_t)req_ids[b]);
+    const float target = unit_uniform(w.w[0]) * S;
+    // first chunk whose inclusive prefix exceeds the target (chunk order)
+    float P = 0.f;
+    int cs = -1, last_pos = 0;
+    float P0 = 0.f;
+    for (int c = 0; c < n_chunks; ++c) {
+      const float sc = pr[c].s * expf(pr[c].m - M);
+      if (sc > 0.f) last_pos = c;
+      if (cs < 0 && P + sc > target) { cs = c; P0 = P; }
+      P += sc;
+    }
+    if (cs < 0) { cs = last_pos; P0 = INFINITY; }  // rounding: no crossing -> last positive
+    sh_M = M; sh_S = S; sh_target = target; sh_P0 = P0; sh_c = cs;
+    pmax[row] = 1.0f / S;
+    ent[row] = logf(S) - A / S;
+  }
+  __syncthreads();
+  // scan chunk sh_c in vocabulary order: thread t owns 16 consecutive elements
+  const float M = sh_M, target = sh_target, P0 = sh_P0;
+  const int c0 = sh_c * kChunk;
+  const float* lrow = logits + (size_t)row * vocab;
+  float e[kPerThread];
+  float local = 0.f;
+  int lastpos = -1;
+#pragma unroll
+  for (int r = 0; r < kPerThread; ++r) {
+    const int j = c0 + threadIdx.x * kPerThread + r;
+    const float v = (j < vocab) ? expf(lrow[j] * scale - M) : 0.f;
+    e[r] = v;
+    local += v;
+    if (v > 0.f) lastpos = j;
+  }
+  // inclusive scan of the per-thread sums in thread order (Hillis-Steele)
+  scan[threadIdx.x] = local;
+  __syncthreads();
+  for (int o = 1; o < kThreads; o <<= 1) {
+    const float add = (threadIdx.x >= o) ? scan[threadIdx.x - o] : 0.f;
+    __syncthreads();
+    scan[threadIdx.x] += add;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) sh_pick = 0x7fffffff;
+  __syncthreads();
+  const float before = P0 + (scan[threadIdx.x] - local);
+  if (before <= target && before + local > target) {
+    float run = before;
+    int pick = -1;
+#pragma unroll
+    for (int r = 0; r < kPerThread; ++r) {
+      run += e[r];
+      if (pick < 0 && run > target) pick = c0 + threadIdx.x * kPerThread + r;
+    }
+    if (pick < 0) pick = lastpos;  // the thread sum crossed but the element walk fell short
+    atomicMin(&sh_pick, pick);
+  }
+  __syncthreads();
+  if (sh_pick == 0x7fffffff) {
+    // no crossing in this chunk (rounding): the last element with e > 0
+    if (lastpos >= 0) atomicMax(&sh_last, lastpos);
+    __syncthreads();
+    if (threadIdx.x == 0) x_hat[row] = sh_last;
+    return;
+  }
+  if (threadIdx.x == 0) x_hat[row] = sh_pick;
+}
+
+void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const int* req_ids, const SamplerArgs& a,
+                         void* ws, int32_t* x_hat, float* pmax, float* ent, cudaStream_t s) {
+  if (rows <= 0) return;
+  const int n_chunks = (vocab + kChunk - 1) / kChunk;
+  const int argmax_mode = a.temperature == 0.f;
+  const float scale = argmax_mode ? a.logit_scale : a.logit_scale / a.temperature;
+  Partial* part = reinterpret_cast<Partial*>(ws);
+  sampler_pass1<<<dim3(n_chunks, rows), kThreads, 0, s>>>(logits, vocab, scale, argmax_mode, part);
+  sampler_pass2<<<rows, kThreads, 0, s>>>(logits, n, vocab, scale, argmax_mode, req_ids, a.seed, a.step, a.block,
+                                          part, x_hat, pmax, ent);
+}
+
+// Pass 3: per canvas.  rank_i = #{j : pmax_j > pmax_i or (pmax_j == pmax_i and j < i)}.
+__global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const float* __restrict__ pmax,
+                                      const float* __restrict__ ent, int n, int vocab, const int* __restrict__ req_ids,
+                                      uint64_t seed, uint32_t step, uint32_t block, int keep_k, float stop_thr,
+                                      int32_t* __restrict__ canvas, int32_t* __restrict__ keep_out,
+                                      float* __restrict__ mean_h, int32_t* __restrict__ stop_out,
+                                      int32_t* __restrict__ done, int32_t* __restrict__ out_tokens, int final_step) {
+  extern __shared__ float pm[];
+  __shared__ float red[32];
+  __shared__ int sh_stop;
+  const int b = blockIdx.x;
+  const int req = req_ids[b];
+  const int i = threadIdx.x;
+  for (int j = i; j < n; j += blockDim.x) pm[j] = pmax[(size_t)b * n + j];
+  const int was_done = (done != nullptr) ? done[b] : 0;
+  __syncthreads();
+  float hsum = 0.f;
+  if (i < n) hsum = ent[(size_t)b * n + i];
+  // deterministic block sum over positions
+  hsum = warp_sum(hsum);
+  if ((i & 31) == 0) red[i >> 5] = hsum;
+  __syncthreads();
+  if (i == 0) {
+    float t = 0.f;
+    for (int x = 0; x < (int)((blockDim.x + 31) >> 5); ++x) t += red[x];
+    const float mh = t / (float)n;
+    const int st = (stop_thr >= 0.f && mh < stop_thr) ? 1 : 0;
+    if (mean_h) mean_h[b] = mh;
+    if (stop_out) stop_out[b] = st;
+    sh_stop = st;
+  }
+  __syncthreads();
+  if (i < n) {
+    const float p = pm[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const float q = pm[j];
+      rank += (q > p || (q == p && j < i)) ? 1 : 0;
+    }
+    const int kept = rank < keep_k;
+    const int32_t xh = x_hat[(size_t)b * n + i];
+    const Philox4 w = sampler_words(seed, (uint32_t)i, step, block, (uint32_t)req);
+    const int32_t tok = kept ? xh : uniform_token(w.w[1], (uint32_t)vocab);
+    canvas[(size_t)b * n + i] = tok;
+    if (keep_out) keep_out[(size_t)b * n + i] = kept;
+    if (out_tokens != nullptr && !was_done && (sh_stop || final_step)) out_tokens[(size_t)b * n + i] = xh;
+  }
+  __syncthreads();
+  if (i == 0 && done != nullptr && !was_done && (sh_stop || final_step)) done[b] = 1;
+}
+
+void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float* ent, int B, int n, int vocab,
+                           const int* req_ids, const SamplerArgs& a, int32_t* canvas, int32_t* keep, float* mean_h,
+                           int32_t* stop, int32_t* done, int32_t* out_tokens, int final_step, cudaStream_t s) {
+  if (B <= 0) return;
+  const int threads = ((n + 31) / 32) * 32;
+  sampler_finish_kernel<<<B, threads, n * sizeof(float), s>>>(x_hat, pmax, ent, n, vocab, req_ids, a.seed, a.step,
+                                                              a.block, a.keep_k, a.stop_threshold, canvas, keep,
+                                                              mean_h, stop, done, out_tokens, final_step);
+}
+
+// ------------------------------------------------------------ self test
+__global__ void philox_selftest_kernel(const uint32_t* ctr, const uint32_t* key, uint32_t* out,
+                                       uint32_t* out_curand, int n) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n) return;
+  const Philox4 o = philox4x32_10(ctr[4 * t], ctr[4 * t + 1], ctr[4 * t + 2], ctr[4 * t + 3], key[2 * t],
+                                  key[2 * t + 1]);
+  for (int j = 0; j < 4; ++j) out[4 * t + j] = o.w[j];
+  if (out_curand) {
+    const uint4 c = make_uint4(ctr[4 * t], ctr[4 * t + 1], ctr[4 * t + 2], ctr[4 * t + 3]);
+    const uint2 k = make_uint2(key[2 * t], key[2 * t + 1]);
+    const uint4 r = curand_Philox4x32_10(c, k);
+    out_curand[4 * t] = r.x;
+    out_curand[4 * t + 1] = r.y;
+    out_curand[4 * t + 2] = r.z;
+    out_curand[4 * t + 3] = r.w;
+  }
+}
+
+void launch_philox_selftest(const uint32_t* ctr, const uint32_t* key, uint32_t* out, uint32_t* out_curand, int n,
+                            cudaStream_t s) {
+  if (n <= 0) return;
+  philox_selftest_kernel<<<(n + 127) / 128, 128, 0, s>>>(ctr, key, out, out_curand, n);
+}
+
+}  // namespace dg

@@ -1,0 +1,144 @@
+// Host-side launchers of the device kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dg {
+
+constexpr int kMaxBatch = 64;
+
+// Per-launch description of the requests in a forward pass: row b of the
+// batch is request slot `slot[b]` whose cache holds `len[b]` positions before
+// this pass.
+struct BatchInfo {
+  int B;
+  int slot[kMaxBatch];
+  int len[kMaxBatch];
+};
+
+// ---- elementwise / small kernels (k_elementwise.cu)
+// h[t,:] = E[tok[t],:] (fp32); if prev != null, eprev[t,:] = E[prev[t],:] (act dtype)
+template <typename T>
+void launch_embed(const int32_t* tok, const int32_t* prev, const T* embed, float* h, T* eprev, int n_tok,
+                  int d, int vocab, int* err, cudaStream_t s);
+// xn[t,:] = h[t,:] * w / sqrt(mean(h^2) + eps)
+template <typename T>
+void launch_rmsnorm(const float* h, const float* w, T* xn, int n_tok, int d, float eps, cudaStream_t s);
+// h[t,:] += sum_s wts[t,s] * y[t*k+s,:] (slot order), then optional xn = rmsnorm(h, norm_w)
+template <typename T>
+void launch_combine(float* h, const float* y, const float* wts, int k, const float* norm_w, T* xn,
+                    int n_tok, int d, float eps, cudaStream_t s);
+// Split fp32 q|k|v rows into rotated Q [B,Hq,nq,hd], K cache rows and transposed V cache rows.
+template <typename T>
+void launch_rope_scatter(const float* qkv, T* q, T* kc, T* vt, const float* rope_cs, const BatchInfo& bi,
+                         int nq, int hq, int hkv, int hd, int max_ctx, cudaStream_t s);
+// xp[p,:] = xn[perm[p]/k,:] for p < n_rows
+template <typename T>
+void launch_gather_rows(const T* xn, const int32_t* perm, T* xp, int n_rows, int k, int d, cudaStream_t s);
+// canvas[b,i] = uniform token from Philox word 1 of counter (i, 0, block, req[b])
+void launch_init_canvas(int32_t* canvas, const BatchInfo& bi, const int* req_ids, int n, int vocab,
+                        uint64_t seed, uint32_t block, cudaStream_t s);
+// Copy a [Hkv, n, hd] K/V block into positions [0, n) of one request's cache.
+template <typename T>
+void launch_set_kv(const T* k, const T* v, T* kc, T* vt, int hkv, int n, int hd, int max_ctx,
+                   cudaStream_t s);
+
+// ---- router (k_router.cu)
+// Per token: g = glog + bias; top-k (ties -> lower id); softmax over the k.
+void launch_router_topk(const float* glog, const float* bias, int32_t* ids, float* wts, int n_tok, int e,
+                        int k, cudaStream_t s);
+// Deterministic counting sort of the n_tok*k (token, slot) items by expert
+// (tokens ascending inside an expert).  perm[pos] = t*k+s; cnt[E]; off[E+1];
+// work list of (expert, first row, rows) tiles of at most `tile` rows;
+// touched = number of experts with cnt > 0.
+void launch_router_permute(const int32_t* ids, int n_items, int e, int tile, int32_t* cnt, int32_t* off,
+                           int32_t* perm, int32_t* work, int32_t* n_work, int32_t* touched,
+                           cudaStream_t s);
+
+// ---- sampler (k_sampler.cu)
+struct SamplerArgs {
+  float temperature, logit_scale, stop_threshold;
+  int keep_k;
+  uint64_t seed;
+  uint32_t block;
+  uint32_t step;
+};
+size_t sampler_workspace_bytes(int rows, int vocab);
+// rows = B*N logits rows; writes x_hat, pmax, H (workspace-sized arrays).
+void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const int* req_ids,
+                         const SamplerArgs& a, void* ws, int32_t* x_hat, float* pmax, float* ent,
+                         cudaStream_t s);
+// Per canvas: keep set, re-noise, mean entropy, stop; optional block-loop outputs.
+void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float* ent, int B, int n,
+                           int vocab, const int* req_ids, const SamplerArgs& a, int32_t* canvas,
+                           int32_t* keep, float* mean_h, int32_t* stop, int32_t* done, int32_t* out_tokens,
+                           int final_step, cudaStream_t s);
+
+// ---- GEMMs
+enum Epi { EPI_STORE_F32 = 0, EPI_ADD_F32 = 1, EPI_STORE_ACT = 2, EPI_SWIGLU_ACT = 3, EPI_SCATTER_F32 = 4 };
+
+// SIMT fp32/generic path: out[t, n] (op)= sum_k x[t,k] w[n,k].
+template <typename T>
+void launch_gemm_simt(const T* x, const T* w, int n_tok, int n_out, int kdim, Epi epi, void* out, int ld_out,
+                      const float* bias, cudaStream_t s);
+// SIMT grouped expert GEMM over a work list (expert, row0, rows):
+// up:   out[r, f]  = silu(x[r] . wg[e,f]) * (x[r] . wu[e,f])      (act dtype)
+// down: y[perm[r], n] = x[r] . wd[e,n]                              (fp32)
+template <typename T>
+void launch_grouped_simt(const T* x, const T* wa, const T* wb, int n_out, int kdim, const int32_t* work,
+                         const int32_t* n_work, int n_work_max, const int32_t* perm, bool up, void* out,
+                         int ld_out, cudaStream_t s);
+
+// tcgen05 path (k_gemm_tc.cu): weights are the 128-row M side, tokens the N side.
+struct TcGemm {
+  int mode;          // 0 dense, 1 grouped up (gate+up, SwiGLU), 2 grouped down
+  int M, K;          // weight rows (dense: total; grouped: per expert), reduction dim
+  int T;             // dense: token rows
+  int ntile;         // token tile width (multiple of 32, <= 256)
+  int seg1, seg2;    // dense: first weight row served by map a1 / a2 (multiples of 128)
+  const int32_t* work;
+  const int32_t* n_work;
+  int n_work_max;
+  int epi;
+  void* out;
+  int ld_out;
+  const float* bias;
+  const int32_t* row_map;
+  int* err;
+};
+void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
+                    const TcGemm& p, int num_sms, cudaStream_t s);
+int gemm_tc_smem_bytes(const TcGemm& p, int* stages);
+
+// ---- attention
+struct AttnArgs {
+  int B, nq, hq, hkv, hd, max_ctx;
+  int causal;
+  BatchInfo bi;
+};
+// SIMT (any dtype): q [B,Hq,nq,hd]; kc [slots,Hkv,max_ctx,hd]; vt [slots,Hkv,hd,max_ctx];
+// out [B*nq, Hq*hd]
+template <typename T>
+void launch_attn_simt(const T* q, const T* kc, const T* vt, T* out, const AttnArgs& a, cudaStream_t s);
+
+// tcgen05 canvas/causal attention for bf16, hd == 256 (k_attn_tc.cu).
+struct AttnTcArgs {
+  AttnArgs a;
+  int n_split;       // KV splits per (b, head, q-tile)
+  float* part_o;     // [splits][B][Hq][nq_pad][hd] fp32 partial outputs (unnormalised)
+  float* part_ml;    // [splits][B][Hq][nq_pad][2] (max, sum)
+  int nq_pad;
+  int* err;
+};
+void launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    __nv_bfloat16* out, const AttnTcArgs& a, cudaStream_t s);
+size_t attn_tc_partial_floats(int n_split, int B, int hq, int nq_pad, int hd);
+
+// ---- self test
+void launch_philox_selftest(const uint32_t* ctr, const uint32_t* key, uint32_t* out, uint32_t* out_curand,
+                            int n, cudaStream_t s);
+
+}  // namespace dg

@@ -1,0 +1,278 @@
+"""Thin Python binding of the C ABI in include/dg.h (ctypes; argument
+marshalling only).  Every function here forwards to the function of the same
+name in libdg.so; tensors are passed as raw device pointers.
+
+The library must have been built (``python -m discrete_text_diffusion_b200.build``);
+importing this module without it raises -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdg.so")
+
+DG_OK, DG_EINVAL, DG_ENOMEM, DG_ECUDA, DG_ECAPACITY, DG_ESTATE, DG_ETIMEOUT = range(7)
+DG_FP32, DG_BF16 = 0, 1
+
+EXPORTS = (
+    "dg_create", "dg_destroy", "dg_last_error", "dg_prefill_prompt", "dg_set_kv", "dg_set_length",
+    "dg_get_length", "dg_denoise_step", "dg_sample", "dg_generate_block", "dg_generate_block_host",
+    "dg_synchronize", "dg_launch_count", "dg_profile_enable", "dg_profile_read", "dg_profile_reset",
+    "dg_selftest_philox", "dg_selftest_gemm",
+)
+
+
+class DgConfig(C.Structure):
+    _fields_ = [("n_layers", C.c_int), ("d_model", C.c_int), ("n_heads", C.c_int), ("n_kv_heads", C.c_int),
+                ("head_dim", C.c_int), ("n_experts", C.c_int), ("top_k", C.c_int), ("d_ff", C.c_int),
+                ("vocab", C.c_int), ("canvas", C.c_int), ("max_batch", C.c_int), ("max_ctx", C.c_int),
+                ("max_tokens", C.c_int), ("dtype", C.c_int), ("rope_base", C.c_double), ("rms_eps", C.c_double)]
+
+
+class DgLayerWeights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "router_w",
+                                          "router_b", "w_gate", "w_up", "w_down")]
+
+
+class DgWeights(C.Structure):
+    _fields_ = [("embed", C.c_void_p), ("w_sc", C.c_void_p), ("final_norm", C.c_void_p),
+                ("layers", C.POINTER(DgLayerWeights))]
+
+
+class DgSamplerParams(C.Structure):
+    _fields_ = [("temperature", C.c_float), ("logit_scale", C.c_float), ("stop_threshold", C.c_float),
+                ("keep_k", C.c_int), ("seed", C.c_uint64), ("block", C.c_uint32)]
+
+
+class DgStepOut(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("x_hat", "pmax", "entropy", "keep", "mean_entropy", "stop",
+                                          "experts_touched")]
+
+
+class DgStepArgs(C.Structure):
+    _fields_ = [("batch", C.c_int), ("req", C.POINTER(C.c_int)), ("canvas", C.c_void_p),
+                ("prev_pred", C.c_void_p), ("step", C.c_int), ("sp", DgSamplerParams),
+                ("logits_out", C.c_void_p), ("hidden_out", C.c_void_p)]
+
+
+class DgBlockArgs(C.Structure):
+    _fields_ = [("batch", C.c_int), ("req", C.POINTER(C.c_int)), ("max_steps", C.c_int),
+                ("schedule_steps", C.c_int), ("temperature", C.c_float), ("logit_scale_growth", C.c_float),
+                ("stop_threshold", C.c_float), ("seed", C.c_uint64), ("block", C.c_uint32)]
+
+
+class DgProfileEntry(C.Structure):
+    _fields_ = [("name", C.c_char_p), ("launches", C.c_int), ("ms", C.c_double)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libdg.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m discrete_text_diffusion_b200.build")
+        L = C.CDLL(LIB_PATH)
+        P = C.c_void_p
+        L.dg_create.argtypes = [C.POINTER(DgConfig), C.POINTER(DgWeights), P, C.POINTER(P)]
+        L.dg_destroy.argtypes = [P]
+        L.dg_destroy.restype = None
+        L.dg_last_error.argtypes = [P]
+        L.dg_last_error.restype = C.c_char_p
+        L.dg_prefill_prompt.argtypes = [P, C.c_int, C.POINTER(C.c_int), P, C.c_int]
+        L.dg_set_kv.argtypes = [P, C.c_int, C.c_int, P, P, C.c_int]
+        L.dg_set_length.argtypes = [P, C.c_int, C.c_int]
+        L.dg_get_length.argtypes = [P, C.c_int, C.POINTER(C.c_int)]
+        L.dg_denoise_step.argtypes = [P, C.POINTER(DgStepArgs), C.POINTER(DgStepOut)]
+        L.dg_sample.argtypes = [P, P, C.c_int, C.POINTER(C.c_int), C.c_int, C.POINTER(DgSamplerParams), P,
+                                C.POINTER(DgStepOut)]
+        L.dg_generate_block.argtypes = [P, C.POINTER(DgBlockArgs), P, C.POINTER(C.c_int)]
+        L.dg_generate_block_host.argtypes = [P, C.POINTER(DgBlockArgs), P, C.POINTER(C.c_int)]
+        L.dg_synchronize.argtypes = [P]
+        L.dg_launch_count.argtypes = [P]
+        L.dg_launch_count.restype = C.c_uint64
+        L.dg_profile_enable.argtypes = [P, C.c_int]
+        L.dg_profile_read.argtypes = [P, C.POINTER(DgProfileEntry), C.c_int, C.POINTER(C.c_int)]
+        L.dg_profile_reset.argtypes = [P]
+        L.dg_selftest_philox.argtypes = [P, P, P, P, P, C.c_int]
+        L.dg_selftest_gemm.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, P]
+        _lib = L
+    return _lib
+
+
+class DgError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"dg error {code}: {msg}")
+        self.code = code
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _ints(xs):
+    return (C.c_int * len(xs))(*[int(x) for x in xs])
+
+
+class Handle:
+    """Owns a dg_handle and keeps the borrowed weight tensors alive."""
+
+    def __init__(self, ptr, keep):
+        self.ptr = ptr
+        self._keep = keep
+
+    def check(self, rc):
+        if rc != DG_OK:
+            raise DgError(rc, lib().dg_last_error(self.ptr).decode())
+        return rc
+
+    def close(self):
+        if self.ptr:
+            lib().dg_destroy(self.ptr)
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _cfg(model: dict, *, dtype: str, max_batch: int, max_ctx: int, max_tokens: int = 0) -> DgConfig:
+    m = model
+    return DgConfig(m.get("n_layers", 0), m.get("d_model", 0), m.get("n_heads", 0), m.get("n_kv_heads", 0),
+                    m.get("head_dim", 0), m.get("n_experts", 0), m.get("top_k", 0), m.get("d_ff", 0),
+                    m["vocab"], m["canvas"], max_batch, max_ctx, max_tokens,
+                    DG_BF16 if dtype == "bf16" else DG_FP32, float(m.get("rope_base", 10000.0)),
+                    float(m.get("rms_eps", 1e-6)))
+
+
+def dg_create(model: dict, weights, *, dtype: str, max_batch: int, max_ctx: int, max_tokens: int = 0,
+              stream=None) -> Handle:
+    """dg_create.  weights: dict of device tensors (synth.make_weights layout) or None
+    for a sampler-only handle (model['n_layers'] == 0)."""
+    cfg = _cfg(model, dtype=dtype, max_batch=max_batch, max_ctx=max_ctx, max_tokens=max_tokens)
+    keep = [weights]
+    wp = None
+    if weights is not None:
+        lay = (DgLayerWeights * len(weights["layers"]))()
+        for i, L in enumerate(weights["layers"]):
+            for k in DgLayerWeights._fields_:
+                name = k[0]
+                setattr(lay[i], name, None if L.get(name) is None else L[name].data_ptr())
+        keep.append(lay)
+        wp = DgWeights(weights["embed"].data_ptr(), weights["w_sc"].data_ptr(), weights["final_norm"].data_ptr(),
+                       lay)
+        keep.append(wp)
+    out = C.c_void_p()
+    s = None if stream is None else C.c_void_p(stream.cuda_stream)
+    rc = lib().dg_create(C.byref(cfg), C.byref(wp) if wp is not None else None, s, C.byref(out))
+    if rc != DG_OK:
+        raise DgError(rc, lib().dg_last_error(None).decode())
+    return Handle(out, keep)
+
+
+def dg_destroy(h: Handle):
+    h.close()
+
+
+def dg_last_error(h: Handle | None = None) -> str:
+    return lib().dg_last_error(None if h is None else h.ptr).decode()
+
+
+def dg_prefill_prompt(h: Handle, req, tokens: torch.Tensor):
+    """tokens: int32 [B, n] on the device."""
+    return h.check(lib().dg_prefill_prompt(h.ptr, len(req), _ints(req), _ptr(tokens), tokens.shape[-1]))
+
+
+def dg_set_kv(h: Handle, req: int, layer: int, k: torch.Tensor, v: torch.Tensor):
+    return h.check(lib().dg_set_kv(h.ptr, req, layer, _ptr(k), _ptr(v), k.shape[1]))
+
+
+def dg_set_length(h: Handle, req: int, length: int):
+    return h.check(lib().dg_set_length(h.ptr, req, length))
+
+
+def dg_get_length(h: Handle, req: int) -> int:
+    v = C.c_int()
+    h.check(lib().dg_get_length(h.ptr, req, C.byref(v)))
+    return v.value
+
+
+def sampler_params(temperature=1.0, logit_scale=1.0, stop_threshold=-1.0, keep_k=0, seed=0, block=0):
+    return DgSamplerParams(temperature, logit_scale, stop_threshold, keep_k, seed, block)
+
+
+def step_out(x_hat=None, pmax=None, entropy=None, keep=None, mean_entropy=None, stop=None, experts_touched=None):
+    return DgStepOut(*[None if t is None else t.data_ptr() for t in
+                       (x_hat, pmax, entropy, keep, mean_entropy, stop, experts_touched)])
+
+
+def dg_denoise_step(h: Handle, req, canvas, prev_pred, step, sp: DgSamplerParams, out: DgStepOut,
+                    logits_out=None, hidden_out=None):
+    a = DgStepArgs(len(req), _ints(req), canvas.data_ptr(), None if prev_pred is None else prev_pred.data_ptr(),
+                   step, sp, None if logits_out is None else logits_out.data_ptr(),
+                   None if hidden_out is None else hidden_out.data_ptr())
+    return h.check(lib().dg_denoise_step(h.ptr, C.byref(a), C.byref(out)))
+
+
+def dg_sample(h: Handle, logits, req, step, sp: DgSamplerParams, canvas, out: DgStepOut):
+    return h.check(lib().dg_sample(h.ptr, _ptr(logits), len(req), _ints(req), step, C.byref(sp), _ptr(canvas),
+                                   C.byref(out)))
+
+
+def block_args(req, max_steps, schedule_steps, temperature=1.0, logit_scale_growth=1.0, stop_threshold=-1.0,
+               seed=0, block=0):
+    return DgBlockArgs(len(req), _ints(req), max_steps, schedule_steps, temperature, logit_scale_growth,
+                       stop_threshold, seed, block)
+
+
+def dg_generate_block(h: Handle, a: DgBlockArgs, out_tokens: torch.Tensor) -> int:
+    steps = C.c_int()
+    h.check(lib().dg_generate_block(h.ptr, C.byref(a), _ptr(out_tokens), C.byref(steps)))
+    return steps.value
+
+
+def dg_generate_block_host(h: Handle, a: DgBlockArgs, out_tokens_host: torch.Tensor) -> int:
+    steps = C.c_int()
+    h.check(lib().dg_generate_block_host(h.ptr, C.byref(a), _ptr(out_tokens_host), C.byref(steps)))
+    return steps.value
+
+
+def dg_synchronize(h: Handle):
+    return h.check(lib().dg_synchronize(h.ptr))
+
+
+def dg_launch_count(h: Handle) -> int:
+    return int(lib().dg_launch_count(h.ptr))
+
+
+def dg_profile_enable(h: Handle, on: bool):
+    return h.check(lib().dg_profile_enable(h.ptr, 1 if on else 0))
+
+
+def dg_profile_reset(h: Handle):
+    return h.check(lib().dg_profile_reset(h.ptr))
+
+
+def dg_profile_read(h: Handle) -> dict:
+    arr = (DgProfileEntry * 32)()
+    n = C.c_int()
+    h.check(lib().dg_profile_read(h.ptr, arr, 32, C.byref(n)))
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].ms) for i in range(min(n.value, 32))}
+
+
+def dg_selftest_philox(h: Handle, ctr, key, out, out_curand=None):
+    return h.check(lib().dg_selftest_philox(h.ptr, _ptr(ctr), _ptr(key), _ptr(out), _ptr(out_curand),
+                                            ctr.shape[0]))
+
+
+def dg_selftest_gemm(h: Handle, x, w, out):
+    """out[T, M] fp32 = x[T, K] @ w[M, K]^T through the tensor-core GEMM."""
+    return h.check(lib().dg_selftest_gemm(h.ptr, _ptr(x), _ptr(w), x.shape[0], w.shape[0], x.shape[1], _ptr(out)))

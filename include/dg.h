@@ -1,0 +1,259 @@
+/*
+ * dg.h -- C ABI of the B200 denoising-step library for block-autoregressive
+ * multinomial text diffusion with a top-k MoE (DiffusionGemma-style).
+ *
+ * Sources of the operations, cited by tag:
+ *   [P1] DiffusionGemma technical-report summary (animattoys.com):
+ *        section 一 (multinomial diffusion: noise replaces a token by a uniform
+ *        vocabulary token; a 256-token random canvas; ~12 rounds on average),
+ *        section 二 (Gemma-4 MoE, 128 experts / top-8; causal prompt encoding into
+ *        the KV cache and bidirectional canvas attention; self-conditioning on the
+ *        previous round's predictions with ~7.8M extra parameters),
+ *        section 四 (the sampler: confidence, entropy, re-randomising the
+ *        uncertain positions, temperature, adaptive stop on mean entropy, a
+ *        48-round budget), section 五 (per-step cost: MoE, softmax over the
+ *        262k vocabulary and the self-conditioning matmul, canvas attention).
+ *   [P2] DiffusionGemma overview (youleyou.com), 架构基础 (causal encoder into
+ *        the KV cache, bidirectional denoiser over the canvas, finished blocks
+ *        handed to the KV cache) and 离散文本扩散的运作机制 (canvas init,
+ *        iterative refinement, re-noising of low-confidence positions).
+ *   [P3] "Google 開源 DiffusionGemma" (akiraxclaw.com): a finished canvas is
+ *        encoded into the KV cache before the next one starts.
+ *   [Philox] Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless the comment says host.  The caller
+ *     owns every pointer it passes; the library never frees them.  Weights are
+ *     BORROWED: they must stay valid and unchanged until dg_destroy.
+ *   - Matrices are row-major [out, in] (the layout of a linear layer's weight).
+ *   - Work is ordered on the handle's stream.  Entry points that return results
+ *     on the host (steps_used, lengths) synchronise that stream.
+ *   - Return value: DG_OK or an error code; dg_last_error() gives the message.
+ *     All shape, alignment and capacity checks run on the host before any
+ *     launch; a failed check launches nothing and leaves state unchanged.
+ *     A device-side timeout in a kernel wait is reported as DG_ETIMEOUT by the
+ *     next call that synchronises.  No entry point traps the device.
+ *   - dtype DG_BF16: weights, activations between GEMMs and the KV cache are
+ *     bf16, accumulation and the residual stream fp32.  dtype DG_FP32: all fp32.
+ *     Norm weights and the router bias are fp32 in both.
+ */
+#ifndef DG_H
+#define DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  DG_OK = 0,
+  DG_EINVAL = 1,     /* bad argument, shape, alignment or null pointer */
+  DG_ENOMEM = 2,     /* device or pinned-host allocation failed */
+  DG_ECUDA = 3,      /* a CUDA runtime/driver call failed */
+  DG_ECAPACITY = 4,  /* KV cache or workspace capacity exceeded */
+  DG_ESTATE = 5,     /* call not valid in the handle's state */
+  DG_ETIMEOUT = 6    /* a bounded device-side wait gave up */
+};
+
+enum { DG_FP32 = 0, DG_BF16 = 1 };
+
+typedef struct dg_handle dg_handle;
+
+/* Model shape and capacities ([P1 二]). */
+typedef struct dg_config {
+  int n_layers;      /* transformer layers (0: sampler-only handle) */
+  int d_model;       /* d */
+  int n_heads;       /* Hq query heads */
+  int n_kv_heads;    /* Hkv KV heads; Hq % Hkv == 0 (GQA) */
+  int head_dim;      /* hd, even */
+  int n_experts;     /* E <= 256 */
+  int top_k;         /* k <= min(E, 16) */
+  int d_ff;          /* F, expert FFN width */
+  int vocab;         /* V */
+  int canvas;        /* N, canvas length (256 in [P1 一]) */
+  int max_batch;     /* request slots, 1..64 */
+  int max_ctx;       /* KV capacity per request in positions, multiple of 64 */
+  int max_tokens;    /* rows per forward pass (>= max_batch*canvas; 0 = that) */
+  int dtype;         /* DG_BF16 or DG_FP32 */
+  double rope_base;  /* RoPE base (10000) */
+  double rms_eps;    /* RMSNorm epsilon */
+} dg_config;
+
+/* One layer's weights (all borrowed device pointers). */
+typedef struct dg_layer_weights {
+  const float* attn_norm;  /* [d] fp32 */
+  const void* wq;          /* [Hq*hd, d] */
+  const void* wk;          /* [Hkv*hd, d] */
+  const void* wv;          /* [Hkv*hd, d] */
+  const void* wo;          /* [d, Hq*hd] */
+  const float* ffn_norm;   /* [d] fp32 */
+  const void* router_w;    /* [E, d] */
+  const float* router_b;   /* [E] fp32, or NULL for no bias */
+  const void* w_gate;      /* [E, F, d] */
+  const void* w_up;        /* [E, F, d] */
+  const void* w_down;      /* [E, d, F] */
+} dg_layer_weights;
+
+typedef struct dg_weights {
+  const void* embed;                /* [V, d]; also the tied LM head */
+  const void* w_sc;                 /* [d, d] self-conditioning projection */
+  const float* final_norm;          /* [d] fp32 */
+  const dg_layer_weights* layers;   /* HOST array of n_layers entries */
+} dg_weights;
+
+/* Sampler settings for one step ([P1 四]). */
+typedef struct dg_sampler_params {
+  float temperature;     /* T > 0; 0 = argmax (ties to the lower index) */
+  float logit_scale;     /* s: statistics use z = s * logit / T */
+  float stop_threshold;  /* stop when mean entropy (nats) < this; < 0 disables */
+  int keep_k;            /* positions kept this step (0..N) */
+  uint64_t seed;         /* Philox key */
+  uint32_t block;        /* Philox counter word 2 (block index) */
+} dg_sampler_params;
+
+/* Outputs of one sampler step; every pointer may be NULL (not written). */
+typedef struct dg_step_out {
+  int32_t* x_hat;            /* [B, N] sampled tokens */
+  float* pmax;               /* [B, N] max probability of z */
+  float* entropy;            /* [B, N] entropy of z, nats */
+  int32_t* keep;             /* [B, N] 1 = kept, 0 = re-noised */
+  float* mean_entropy;       /* [B] */
+  int32_t* stop;             /* [B] 1 = stop test passed */
+  int32_t* experts_touched;  /* [n_layers] distinct experts routed to */
+} dg_step_out;
+
+/* One denoising step ([P1 一/二/四]). */
+typedef struct dg_step_args {
+  int batch;                   /* B <= max_batch */
+  const int* req;              /* HOST [B] request slots, distinct */
+  int32_t* canvas;             /* [B, N] in: current canvas, out: re-noised canvas */
+  const int32_t* prev_pred;    /* [B, N] previous x_hat for self-conditioning, or NULL */
+  int step;                    /* t >= 1, Philox counter word 1 */
+  dg_sampler_params sp;
+  float* logits_out;           /* [B, N, V] fp32 to receive the logits, or NULL */
+  float* hidden_out;           /* [B*N, d] fp32 residual stream before the final
+                                  norm, or NULL */
+} dg_step_args;
+
+/* One block ([P1 一/四], [P2], [P3]). */
+typedef struct dg_block_args {
+  int batch;                  /* B <= max_batch */
+  const int* req;             /* HOST [B] request slots, distinct */
+  int max_steps;              /* step budget (48 in [P1 四]) */
+  int schedule_steps;         /* T of the keep schedule k_t = ceil(N t / T) */
+  float temperature;
+  float logit_scale_growth;   /* s_t = growth^(t-1) */
+  float stop_threshold;       /* < 0 disables the adaptive stop */
+  uint64_t seed;
+  uint32_t block;
+} dg_block_args;
+
+/* Kernel-class timing, filled when profiling is on. */
+typedef struct dg_profile_entry {
+  const char* name;   /* static string */
+  int launches;
+  double ms;          /* summed CUDA-event time on the handle's stream */
+} dg_profile_entry;
+
+/*
+ * dg_create: validate cfg, borrow w, allocate the KV cache
+ * ([layers][max_batch][Hkv][max_ctx][hd] for K and the transposed
+ * [layers][max_batch][Hkv][hd][max_ctx] for V, zero-filled) and the workspaces,
+ * and build the TMA descriptors.  stream: a cudaStream_t (NULL = legacy default).
+ * For n_layers == 0, w may be NULL (sampler-only handle for dg_sample).
+ * BF16 handles need d, hd, F multiples of 64 and weight pointers 16-byte aligned.
+ */
+int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle** out);
+
+/* Release everything the handle owns.  NULL is a no-op. */
+void dg_destroy(dg_handle* h);
+
+/* Message of the last failed call on h (NULL h: last failed dg_create). */
+const char* dg_last_error(const dg_handle* h);
+
+/*
+ * Causal encode of n tokens per request at positions P..P+n-1, appending their
+ * K/V to each request's cache (prompt prefill, [P1 二], [P2 架构基础]); then
+ * P += n.  tokens: [B, n] int32.  DG_ECAPACITY if any P + n > max_ctx.
+ */
+int dg_prefill_prompt(dg_handle* h, int batch, const int* req, const int32_t* tokens, int n);
+
+/*
+ * Test hook: write positions [0, n) of one layer's cache for request req.
+ * k, v: [Hkv, n, hd] in the handle's dtype.  Does not change P.
+ */
+int dg_set_kv(dg_handle* h, int req, int layer, const void* k, const void* v, int n);
+
+/* Set / read a request's cache length P (host-side state; set checks capacity). */
+int dg_set_length(dg_handle* h, int req, int length);
+int dg_get_length(const dg_handle* h, int req, int* length);
+
+/*
+ * One denoising step over B canvases: embed + self-conditioning, all layers
+ * (canvas attention over cache [0,P) + the canvas, no mask), final norm, tied
+ * LM head, then the sampler (dg_sample's definition).  The canvas K/V are
+ * written at cache positions [P, P+N) as scratch; P is not changed.
+ * DG_ECAPACITY if P + N > max_ctx.
+ */
+int dg_denoise_step(dg_handle* h, const dg_step_args* a, const dg_step_out* o);
+
+/*
+ * The sampler alone on caller logits [B, N, V] fp32 ([P1 四], [P1 五]):
+ * z = s*l/T; pmax = max softmax(z); H = entropy(softmax(z));
+ * x_hat = inverse-CDF sample in vocabulary order with u from Philox word 0 of
+ * counter (i, step, block, req[b]) under key seed (u = (w0 >> 8) * 2^-24);
+ * keep = top keep_k positions by pmax (ties to the lower index);
+ * canvas[b,i] = keep ? x_hat : (w1 * V) >> 32 (uniform re-noise from word 1);
+ * mean entropy and stop = mean < stop_threshold.
+ */
+int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int step,
+              const dg_sampler_params* sp, int32_t* canvas, const dg_step_out* o);
+
+/*
+ * One block per request: canvas from Philox word 1 of counter (i, 0, block,
+ * req); steps t = 1..max_steps with keep_k = ceil(N t / schedule_steps) and
+ * logit scale growth^(t-1), self-conditioning on the previous x_hat; a request
+ * finishes at its first stop (or at max_steps) with output x_hat; the loop ends
+ * when every request has finished.  Then the causal hand-off: the output tokens
+ * are encoded causally and their K/V appended (P += N) ([P2], [P3]).
+ * out_tokens: [B, N] device int32.  steps_used: HOST int, steps run.
+ */
+int dg_generate_block(dg_handle* h, const dg_block_args* a, int32_t* out_tokens, int* steps_used);
+
+/* dg_generate_block with HOST output: copies the [B, N] tokens to out_tokens_host. */
+int dg_generate_block_host(dg_handle* h, const dg_block_args* a, int32_t* out_tokens_host,
+                           int* steps_used);
+
+/* Synchronise the handle's stream and report device-side timeouts. */
+int dg_synchronize(dg_handle* h);
+
+/* Kernel launches issued by this handle since creation. */
+uint64_t dg_launch_count(const dg_handle* h);
+
+/* Per-kernel-class CUDA-event timing: enable/disable, read (synchronises), reset. */
+int dg_profile_enable(dg_handle* h, int on);
+int dg_profile_read(dg_handle* h, dg_profile_entry* out, int max_entries, int* n_entries);
+int dg_profile_reset(dg_handle* h);
+
+/*
+ * Test hook: Philox4x32-10 [Philox] on n counters.  ctr [n,4], key [n,2],
+ * out [n,4] (this library's generator), out_curand [n,4] (cuRAND's device
+ * Philox4_32_10 for the same key/counter, or NULL).  All device uint32.
+ * Uses the handle's stream; h may be a sampler-only handle.
+ */
+int dg_selftest_philox(dg_handle* h, const uint32_t* ctr, const uint32_t* key, uint32_t* out,
+                       uint32_t* out_curand, int n);
+
+/*
+ * Test hook: one dense bf16 GEMM through the tensor-core path,
+ * out[T, M] (fp32) = x[T, K] * w[M, K]^T.  x, w bf16 row-major, 16-byte aligned,
+ * K a multiple of 64.  Requires a bf16 handle (its stream and SM count are used).
+ */
+int dg_selftest_gemm(dg_handle* h, const void* x, const void* w, int T, int M, int K, float* out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_H */

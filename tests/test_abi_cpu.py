@@ -1,0 +1,117 @@
+"""The C ABI library loads, exports every function include/dg.h declares, the
+ctypes structures match the header's layout, and host-side validation rejects
+bad configurations before touching a GPU.  CPU only."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+import discrete_text_diffusion_b200 as dgm
+from discrete_text_diffusion_b200 import dg as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dg.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dg_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        from discrete_text_diffusion_b200 import build
+        build.build()
+    return B.lib()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.EXPORTS)
+
+
+def test_binding_has_same_names_as_abi():
+    for n in B.EXPORTS:
+        assert callable(getattr(B, n)), n
+
+
+_STRUCTS = {
+    "dg_config": B.DgConfig, "dg_layer_weights": B.DgLayerWeights, "dg_weights": B.DgWeights,
+    "dg_sampler_params": B.DgSamplerParams, "dg_step_out": B.DgStepOut, "dg_step_args": B.DgStepArgs,
+    "dg_block_args": B.DgBlockArgs, "dg_profile_entry": B.DgProfileEntry,
+}
+
+
+def test_struct_layouts_match_header(tmp_path):
+    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void) {"]
+    for cname, py in _STRUCTS.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'printf("{cname}.{fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-o", str(exe), str(src)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = dict(line.rsplit(" ", 1) for line in out if line)
+    for cname, py in _STRUCTS.items():
+        assert int(got[f"{cname} size"]) == C.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert int(got[f"{cname}.{fname}"]) == getattr(py, fname).offset, f"{cname}.{fname}"
+
+
+def _create_rc(**over):
+    m = dict(dgm.synth.WORKLOADS["tiny_fp32"]["model"])
+    m.update(over)
+    cfg = B._cfg(m, dtype="fp32", max_batch=1, max_ctx=128)
+    out = C.c_void_p()
+    rc = B.lib().dg_create(C.byref(cfg), None, None, C.byref(out))
+    return rc, B.lib().dg_last_error(None).decode()
+
+
+@pytest.mark.parametrize("over,word", [
+    (dict(n_kv_heads=3), "shape"),
+    (dict(head_dim=7), "shape"),
+    (dict(top_k=9), "shape"),
+    (dict(canvas=0), "canvas"),
+])
+def test_create_rejects_bad_shapes_on_host(lib, over, word):
+    rc, msg = _create_rc(**over)
+    assert rc == B.DG_EINVAL and word in msg
+
+
+def test_create_rejects_missing_weights_on_host(lib):
+    rc, msg = _create_rc()
+    assert rc == B.DG_EINVAL and "weight" in msg
+
+
+def test_create_rejects_bad_dtype_and_capacity(lib):
+    m = dgm.synth.WORKLOADS["tiny_fp32"]["model"]
+    cfg = B._cfg(m, dtype="fp32", max_batch=1, max_ctx=100)     # not a multiple of 64
+    out = C.c_void_p()
+    assert lib.dg_create(C.byref(cfg), None, None, C.byref(out)) == B.DG_EINVAL
+    cfg = B._cfg(m, dtype="fp32", max_batch=65, max_ctx=128)    # too many request slots
+    assert lib.dg_create(C.byref(cfg), None, None, C.byref(out)) == B.DG_EINVAL
+    cfg = B._cfg(m, dtype="fp32", max_batch=1, max_ctx=128)
+    cfg.dtype = 7
+    assert lib.dg_create(C.byref(cfg), None, None, C.byref(out)) == B.DG_EINVAL
+    cfg = B._cfg(dict(m, d_model=96), dtype="bf16", max_batch=1, max_ctx=128)
+    lw = (B.DgLayerWeights * 2)()
+    w = B.DgWeights(16, 16, 16, lw)
+    rc = lib.dg_create(C.byref(cfg), C.byref(w), None, C.byref(out))
+    assert rc == B.DG_EINVAL and "multiples of 64" in lib.dg_last_error(None).decode()
+
+
+def test_null_handle_calls_fail_cleanly(lib):
+    assert lib.dg_synchronize(None) == B.DG_EINVAL
+    assert lib.dg_set_length(None, 0, 0) == B.DG_EINVAL
+    assert lib.dg_launch_count(None) == 0
+    lib.dg_destroy(None)

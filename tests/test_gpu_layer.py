@@ -1,0 +1,73 @@
+"""Full-width bf16 layer (d 2816, 16/8 heads of 256, 128 experts top-8, FFN
+704, vocab 262144, router bias N(0,1), a 2048-position N(0,1) bf16 KV cache,
+canvas 256): one denoise step through the C ABI, checked layer-output-wise and
+on sampled logits against the float64 oracle (max-abs-rel 2e-2 for bf16).
+Plus the tensor-core GEMM alone against a float64 matmul of the same operands."""
+import numpy as np
+import pytest
+import torch
+
+from discrete_text_diffusion_b200 import synth
+from oracle import dg_oracle as O
+from tests._util import max_abs_rel, to_np
+
+W = synth.WORKLOADS["layer_bf16"]
+M = W["model"]
+TOL_BF16 = 2e-2
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,Mr,K", [(1, 128, 64), (31, 200, 128), (256, 384, 2816), (300, 4096, 2816),
+                                    (4096, 512, 704), (96, 262144 // 64, 2816)])
+def test_tc_gemm_matches_float64_matmul(dg, T, Mr, K):
+    g = torch.Generator(device="cuda").manual_seed(T * 7 + Mr)
+    x = torch.randn((T, K), generator=g, device="cuda").to(torch.bfloat16)
+    w = (torch.randn((Mr, K), generator=g, device="cuda") * 0.05).to(torch.bfloat16)
+    out = torch.full((T, Mr), float("nan"), device="cuda")
+    h = dg.dg_create(dict(vocab=8, canvas=4), None, dtype="bf16", max_batch=1, max_ctx=64)
+    dg.dg_selftest_gemm(h, x, w, out)
+    dg.dg_synchronize(h)
+    ref = x.double().cpu() @ w.double().cpu().T
+    err = max_abs_rel(to_np(out), ref.numpy())
+    assert err < 1e-3, err
+    h.close()
+
+
+def _layer_setup(dg):
+    w = synth.make_weights(M, seed=W["seed"], dtype="bf16", router_bias=True, device="cuda")
+    k, v = synth.normal_kv(M["n_kv_heads"], W["cache_len"], M["head_dim"], seed=W["seed"] + 50, dtype="bf16",
+                           device="cuda")
+    h = dg.dg_create(M, w, dtype="bf16", max_batch=1, max_ctx=W["cache_len"] + M["canvas"])
+    dg.dg_set_kv(h, 0, 0, k, v)
+    dg.dg_set_length(h, 0, W["cache_len"])
+    om = O.OracleModel(dict(M), synth.to_numpy_weights(w))
+    om.set_kv(0, 0, k.float().cpu().numpy(), v.float().cpu().numpy())
+    return w, h, om
+
+
+@pytest.mark.gpu
+def test_full_width_layer_step(dg):
+    w, h, om = _layer_setup(dg)
+    n, vocab, d = M["canvas"], M["vocab"], M["d_model"]
+    canvas = synth.uniform_tokens(n, vocab, seed=W["seed"] + 1)
+    prev = synth.uniform_tokens(n, vocab, seed=W["seed"] + 2)
+    rows = np.arange(0, n, 16)
+    for use_prev in (False, True):
+        logits = torch.zeros((1, n, vocab), device="cuda")
+        hid = torch.zeros((n, d), device="cuda")
+        touched = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sp = dg.sampler_params(temperature=1.0, keep_k=64, stop_threshold=0.1, seed=1)
+        dg.dg_denoise_step(h, [0], canvas[None].cuda(), prev[None].cuda() if use_prev else None, 1, sp,
+                           dg.step_out(experts_touched=touched), logits_out=logits, hidden_out=hid)
+        dg.dg_synchronize(h)
+        pos = W["cache_len"] + np.arange(n)
+        hx = om.embed_tokens(canvas.numpy(), prev.numpy() if use_prev else None)
+        ref_h, _, _ = om.layer(hx, 0, 0, pos, causal=False)
+        err_h = max_abs_rel(to_np(hid), ref_h)
+        assert err_h < TOL_BF16, f"layer output max-abs-rel {err_h} (self-cond={use_prev})"
+        x = O.rms_norm(ref_h[rows], om.weights["final_norm"], M["rms_eps"])
+        ref_l = O.lm_head(x, om.weights["embed"])
+        err_l = max_abs_rel(to_np(logits)[0][rows], ref_l)
+        assert err_l < TOL_BF16, f"logits max-abs-rel {err_l}"
+        assert 1 <= int(touched.item()) <= M["n_experts"]
+    h.close()
