@@ -123,6 +123,13 @@ struct dg_handle {
   float* logits = nullptr;
   float2* rope = nullptr;
   CUtensorMap m_xn{}, m_eprev{}, m_attn{}, m_xp{}, m_hb{};
+  // tensor-core attention (bf16, head dim 256)
+  bool attn_tc = false;
+  CUtensorMap m_q{};
+  std::vector<CUtensorMap> m_kc, m_vt;
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  size_t part_rows_cap = 0;   // split-rows capacity of part_o / part_ml
   // sampler workspace
   void* sws = nullptr;
   int32_t* xh[2] = {nullptr, nullptr};
@@ -346,6 +353,25 @@ void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
   a.max_ctx = c.max_ctx;
   a.causal = causal ? 1 : 0;
   a.bi = bi;
+  if (H->attn_tc) {
+    // split the keys so that the grid covers the SMs about twice
+    int max_len = 0;
+    for (int b = 0; b < bi.B; ++b) max_len = std::max(max_len, bi.len[b] + nq);
+    const int base = bi.B * c.n_heads * ((nq + 127) / 128);
+    const int tiles = (max_len + 63) / 64;
+    int n_split = std::max(1, std::min({(2 * H->num_sms + base - 1) / base, 16, std::max(1, tiles / 4)}));
+    if ((size_t)n_split * bi.B * c.n_heads * nq > H->part_rows_cap) n_split = 1;
+    AttnTcArgs t{};
+    t.a = a;
+    t.n_split = n_split;
+    t.part_o = H->part_o;
+    t.part_ml = H->part_ml;
+    t.nq_pad = nq;
+    t.err = H->d_err;
+    ProfScope ps(H, PC_ATTN, n_split > 1 ? 2 : 1);
+    launch_attn_tc(H->m_q, H->m_kc[l], H->m_vt[l], (__nv_bfloat16*)H->attn, t, H->stream);
+    return;
+  }
   ProfScope ps(H, PC_ATTN);
   if (!H->bf16)
     launch_attn_simt<float>((const float*)H->q, (const float*)kc_layer(H, l), (const float*)vt_layer(H, l),
@@ -610,6 +636,11 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
     H->logits = dalloc<float>((size_t)nrow * c.vocab, &ok);
     H->rope = dalloc<float2>((size_t)c.max_ctx * (c.head_dim / 2), &ok);
     H->tok_ws = dalloc<int32_t>((size_t)T, &ok);
+    if (c.dtype == DG_BF16 && c.head_dim == 256) {
+      H->part_rows_cap = (size_t)16 * c.canvas * c.n_heads;
+      H->part_o = dalloc<float>(H->part_rows_cap * c.head_dim, &ok);
+      H->part_ml = dalloc<float>(H->part_rows_cap * 2, &ok);
+    }
   }
   H->sws = dalloc<char>(sampler_workspace_bytes(nrow, c.vocab), &ok);
   H->xh[0] = dalloc<int32_t>(nrow, &ok);
@@ -670,6 +701,18 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
       tm &= tmap_2d(&H->m_attn, H->attn, qw, T, qw, 32);
       tm &= tmap_2d(&H->m_xp, H->xp, d, (uint64_t)T * c.top_k, d, 32);
       tm &= tmap_2d(&H->m_hb, H->hb, F, (uint64_t)T * c.top_k, F, 32);
+      if (c.head_dim == 256) {
+        H->attn_tc = true;
+        const uint64_t hd = (uint64_t)c.head_dim;
+        tm &= tmap_2d(&H->m_q, H->q, hd, (uint64_t)T * c.n_heads, hd, 128);
+        H->m_kc.resize(c.n_layers);
+        H->m_vt.resize(c.n_layers);
+        const uint64_t kv_rows = (uint64_t)c.max_batch * c.n_kv_heads;
+        for (int l = 0; l < c.n_layers; ++l) {
+          tm &= tmap_2d(&H->m_kc[l], kc_layer(H, l), hd, kv_rows * c.max_ctx, hd, 64);
+          tm &= tmap_2d(&H->m_vt[l], vt_layer(H, l), (uint64_t)c.max_ctx, kv_rows * hd, (uint64_t)c.max_ctx, 256);
+        }
+      }
       if (!tm) {
         dg_destroy(H);
         return fail(nullptr, DG_ECUDA, "cuTensorMapEncodeTiled failed (driver entry point or arguments)");
@@ -691,7 +734,7 @@ void dg_destroy(dg_handle* H) {
   void* ps[] = {H->kc, H->vt, H->h, H->xn, H->eprev, H->qkv, H->q, H->attn, H->glog, H->ids, H->wts, H->cnt,
                 H->off, H->perm, H->work, H->n_work, H->touched, H->xp, H->hb, H->y, H->logits, H->rope, H->sws,
                 H->xh[0], H->xh[1], H->pmax, H->ent, H->keep, H->meanh, H->stop, H->done, H->canvas, H->out_tok,
-                H->req_dev, H->tok_ws, H->d_err};
+                H->req_dev, H->tok_ws, H->d_err, H->part_o, H->part_ml};
   for (void* p : ps)
     if (p) cudaFree(p);
   if (H->h_done) cudaFreeHost(H->h_done);

@@ -1,0 +1,370 @@
+// tcgen05 attention for the bf16 model with head dim 256: the canvas step
+// (every canvas query sees the whole cache and the whole canvas, [P1 二],
+// [P2 架构基础]) and the causal encode of prompts / finished blocks.
+//
+// One CTA = (request b, query head h, 128-query tile, KV split).  GQA: head h
+// reads KV head h*Hkv/Hq.
+//   warp 0 lane 0: TMA producer.  Q tile (128 x 256) once; then per 64-key tile
+//     the K tile (64 keys x 256) and the transposed V tile (256 x 64 keys)
+//     into one of two stages.
+//   warp 1 lane 0: MMA issuer.  S_j = Q K_j^T (M 128, N 64, K 256) into one of
+//     two TMEM score buffers, one tile ahead of O += P_j V_j (M 128, N 256,
+//     K 64) with O resident in TMEM (256 columns).
+//   warps 2-5: softmax.  Thread = query row.  Scores are scaled to log2 units;
+//     the running max is only raised when a tile exceeds it by more than 8
+//     (then O and the running sum are rescaled through TMEM), so most tiles
+//     need no correction.  P (bf16) is written to one of two swizzled shared
+//     buffers for the PV MMA.  At the end O / l goes out as bf16, or O, max
+//     and sum go to the split workspace for the combine kernel.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "dg_common.cuh"
+#include "kernels.h"
+
+namespace dg {
+
+constexpr int kAttnThreads = 192;
+constexpr int kQTile = 128;
+constexpr int kKTile = 64;
+constexpr int kHd = 256;
+constexpr int kQBytes = kQTile * kHd * 2;   // 64 KB
+constexpr int kKBytes = kKTile * kHd * 2;   // 32 KB
+constexpr int kVBytes = kHd * kKTile * 2;   // 32 KB
+constexpr int kPBytes = kQTile * kKTile * 2;  // 16 KB
+constexpr int kAttnSmem = 1024 + kQBytes + 2 * kKBytes + 2 * kVBytes + 2 * kPBytes + 256;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+struct AttnTcParams {
+  AttnTcArgs t;
+  int n_qtiles;
+  float scale_log2;   // log2(e) / sqrt(hd)
+};
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                   const __grid_constant__ CUtensorMap tv, __nv_bfloat16* __restrict__ out, const AttnTcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const AttnArgs& a = P.t.a;
+  const int split = blockIdx.x % P.t.n_split;
+  const int qt = blockIdx.x / P.t.n_split;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h * a.hkv / a.hq;
+  const int slot = a.bi.slot[b], plen = a.bi.len[b];
+  const int q0 = qt * kQTile;
+  const int n_keys = plen + a.nq;
+  const int kmax = a.causal ? min(n_keys, plen + q0 + kQTile) : n_keys;
+  const int tiles_all = (kmax + kKTile - 1) / kKTile;
+  const int per = (tiles_all + P.t.n_split - 1) / P.t.n_split;
+  const int t_begin = split * per;
+  const int t_end = min(tiles_all, t_begin + per);
+  const int ntiles = max(0, t_end - t_begin);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t row_id = ((size_t)b * a.hq + h) * a.nq;   // first output row of this (b, h)
+
+  if (ntiles == 0) {
+    // empty split (causal tail): contributes nothing to the combine
+    if (warp >= 2) {
+      const int r = (warp & 3) * 32 + lane;
+      const int qi = q0 + r;
+      if (qi < a.nq && P.t.n_split > 1) {
+        const size_t pr = (size_t)split * a.B * a.hq * a.nq + row_id + qi;
+        P.t.part_ml[2 * pr] = -INFINITY;
+        P.t.part_ml[2 * pr + 1] = 0.f;
+        float* po = P.t.part_o + pr * kHd;
+        for (int d = 0; d < kHd; ++d) po[d] = 0.f;
+      }
+    }
+    return;
+  }
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sQ = base;
+  uint8_t* sK = sQ + kQBytes;            // [2][kKBytes]
+  uint8_t* sV = sK + 2 * kKBytes;        // [2][kVBytes]
+  uint8_t* sP = sV + 2 * kVBytes;        // [2][kPBytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;     // [2]
+  uint64_t* kv_empty = bars + 3;    // [2]
+  uint64_t* s_full = bars + 5;      // [2]
+  uint64_t* s_empty = bars + 7;     // [2]
+  uint64_t* p_full = bars + 9;      // [2]
+  uint64_t* pv_done = bars + 11;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  int* err = P.t.err;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem;          // two score buffers: columns [0, 64), [64, 128)
+  const uint32_t tO = tmem + 256;    // output accumulator: columns [256, 512)
+
+  if (warp == 0 && lane == 0) {
+    // ----------------------------------------------------------- producer
+    prefetch_tmap(&tq);
+    prefetch_tmap(&tk);
+    prefetch_tmap(&tv);
+    const int qrow = (int)row_id + q0;
+    mbar_expect_tx(q_full, kQBytes);
+    for (int c = 0; c < kHd / 64; ++c) tma_load_2d(sQ + c * (kQTile * 128), &tq, q_full, c * 64, qrow);
+    const int krow = (slot * a.hkv + g) * a.max_ctx;
+    const int vrow = (slot * a.hkv + g) * kHd;
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j & 1;
+      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+      if (!mbar_wait(&kv_empty[s], ph ^ 1u, err, kErrTimeoutAttn)) break;
+      const int key0 = (t_begin + j) * kKTile;
+      mbar_expect_tx(&kv_full[s], kKBytes + kVBytes);
+      uint8_t* k_dst = sK + s * kKBytes;
+      for (int c = 0; c < kHd / 64; ++c) tma_load_2d(k_dst + c * (kKTile * 128), &tk, &kv_full[s], c * 64, krow + key0);
+      tma_load_2d(sV + s * kVBytes, &tv, &kv_full[s], key0, vrow);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ----------------------------------------------------------- MMA issuer
+    const uint32_t idesc_s = idesc_bf16(kQTile, kKTile);
+    const uint32_t idesc_o = idesc_bf16(kQTile, kHd);
+    const uint32_t q_base = smem_u32(sQ);
+    bool ok = mbar_wait(q_full, 0, err, kErrTimeoutAttn);
+    auto issue_s = [&](int j) -> bool {
+      const int s = j & 1;
+      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+      if (!mbar_wait(&kv_full[s], ph, err, kErrTimeoutAttn)) return false;
+      if (!mbar_wait(&s_empty[s], ph ^ 1u, err, kErrTimeoutAttn)) return false;
+      tc_fence_after();
+      const uint32_t k_base = smem_u32(sK + s * kKBytes);
+#pragma unroll
+      for (int c = 0; c < kHd / 64; ++c)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(tS + (uint32_t)(s * kKTile), sdesc_k_sw128(q_base + c * (kQTile * 128) + 32u * k),
+                    sdesc_k_sw128(k_base + c * (kKTile * 128) + 32u * k), idesc_s, (c | k) ? 1u : 0u);
+      umma_commit(&s_full[s]);
+      return true;
+    };
+    if (ok) ok = issue_s(0);
+    for (int j = 0; j < ntiles && ok; ++j) {
+      if (j + 1 < ntiles && !issue_s(j + 1)) break;
+      const int s = j & 1;
+      if (!mbar_wait(&p_full[s], (uint32_t)(j >> 1) & 1u, err, kErrTimeoutAttn)) break;
+      tc_fence_after();
+      const uint32_t p_base = smem_u32(sP + s * kPBytes);
+      const uint32_t v_base = smem_u32(sV + s * kVBytes);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        umma_bf16(tO, sdesc_k_sw128(p_base + 32u * k), sdesc_k_sw128(v_base + 32u * k), idesc_o,
+                  (j > 0 || k > 0) ? 1u : 0u);
+      umma_commit(&pv_done[s]);
+      umma_commit(&kv_empty[s]);
+    }
+  } else if (warp >= 2) {
+    // ----------------------------------------------------------- softmax
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qi = q0 + r;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int row_lim = a.causal ? min(n_keys, plen + qi + 1) : n_keys;  // keys < row_lim are visible
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j & 1;
+      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+      if (!mbar_wait(&s_full[s], ph, err, kErrTimeoutAttn)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld32(tS + lane_off + (uint32_t)(s * kKTile), *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tS + lane_off + (uint32_t)(s * kKTile + 32), *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tc_fence_before();
+      mbar_arrive(&s_empty[s]);
+      const int key0 = (t_begin + j) * kKTile;
+      float x[64];
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float v = (key0 + c < row_lim) ? __uint_as_float(sv[c]) * P.scale_log2 : -INFINITY;
+        x[c] = v;
+        tmax = fmaxf(tmax, v);
+      }
+      // raise the running max only when this tile exceeds it by the threshold
+      const bool raise = tmax > m_run + kRescaleThreshold;
+      const float m_new = raise ? tmax : m_run;
+      const float alpha = (raise && m_run > -INFINITY) ? exp2f(m_run - m_new) : 1.f;
+      if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
+        // O of rows in this warp must be rescaled: wait until PV_{j-1} landed
+        if (!mbar_wait(&pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, err, kErrTimeoutAttn)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < kHd; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + lane_off + (uint32_t)c0, ov);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+          tmem_st32(tO + lane_off + (uint32_t)c0, ov);
+        }
+        tmem_st_wait();
+      }
+      l_run *= alpha;
+      m_run = m_new;
+      // P_j -> shared buffer s, once PV_{j-2} has finished reading it
+      if (j >= 2 && !mbar_wait(&pv_done[s], (uint32_t)((j - 2) >> 1) & 1u, err, kErrTimeoutAttn)) {
+        ok = false;
+        break;
+      }
+      uint8_t* prow = sP + s * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+      float lsum = 0.f;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = (m_run > -INFINITY) ? exp2f(x[c8 * 8 + 2 * e] - m_run) : 0.f;
+          const float p1 = (m_run > -INFINITY) ? exp2f(x[c8 * 8 + 2 * e + 1] - m_run) : 0.f;
+          const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+          lsum += __low2float(pp) + __high2float(pp);   // sum what the MMA will see
+          pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+        }
+        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l_run += lsum;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[s]);
+    }
+    if (ok) ok = mbar_wait(&pv_done[(ntiles - 1) & 1], (uint32_t)((ntiles - 1) >> 1) & 1u, err, kErrTimeoutAttn);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = qi < a.nq;
+      if (P.t.n_split == 1) {
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        __nv_bfloat16* op = out + ((size_t)b * a.nq + qi) * ((size_t)a.hq * kHd) + (size_t)h * kHd;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kHd; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + lane_off + (uint32_t)c0, ov);
+          if (valid) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(ov[c + 2 * e]) * inv,
+                                                                __uint_as_float(ov[c + 2 * e + 1]) * inv);
+                pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+              }
+              *reinterpret_cast<uint4*>(op + c0 + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      } else {
+        const size_t pr = (size_t)split * a.B * a.hq * a.nq + row_id + qi;
+        if (valid) {
+          P.t.part_ml[2 * pr] = m_run;
+          P.t.part_ml[2 * pr + 1] = l_run;
+        }
+        float* po = P.t.part_o + pr * kHd;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kHd; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO + lane_off + (uint32_t)c0, ov);
+          if (valid) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(po + c0 + c) =
+                  make_float4(__uint_as_float(ov[c]), __uint_as_float(ov[c + 1]), __uint_as_float(ov[c + 2]),
+                              __uint_as_float(ov[c + 3]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge the split partials of one (b, h, query) row: one warp per row.
+__global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                                    __nv_bfloat16* __restrict__ out, int n_split, int B, int hq, int nq) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rows = B * hq * nq;
+  if (row >= rows) return;
+  const size_t stride = (size_t)rows;
+  float M = -INFINITY;
+  for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[2 * (s * stride + row)]);
+  float L = 0.f;
+  float acc[8];
+#pragma unroll
+  for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+  for (int s = 0; s < n_split; ++s) {
+    const float ms = part_ml[2 * (s * stride + row)];
+    if (ms == -INFINITY) continue;
+    const float w = exp2f(ms - M);
+    L += part_ml[2 * (s * stride + row) + 1] * w;
+    const float* po = part_o + (s * stride + row) * kHd;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) acc[x] += w * po[lane + 32 * x];
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  // row = (b*hq + h)*nq + q  ->  out[(b*nq + q), h*hd + d]
+  const int q = row % nq;
+  const int bh = row / nq;
+  const int h = bh % hq, b = bh / hq;
+  __nv_bfloat16* op = out + ((size_t)b * nq + q) * ((size_t)hq * kHd) + (size_t)h * kHd;
+#pragma unroll
+  for (int x = 0; x < 8; ++x) op[lane + 32 * x] = __float2bfloat16_rn(acc[x] * inv);
+}
+
+size_t attn_tc_partial_floats(int n_split, int B, int hq, int nq_pad, int hd) {
+  return (size_t)n_split * B * hq * nq_pad * hd;
+}
+
+void launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, __nv_bfloat16* out,
+                    const AttnTcArgs& t, cudaStream_t s) {
+  const AttnArgs& a = t.a;
+  if (a.B <= 0 || a.nq <= 0) return;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+    attr = true;
+  }
+  AttnTcParams P;
+  P.t = t;
+  P.n_qtiles = (a.nq + kQTile - 1) / kQTile;
+  P.scale_log2 = 1.4426950408889634f / sqrtf((float)a.hd);
+  dim3 grid(P.n_qtiles * t.n_split, a.hq, a.B);
+  attn_tc_kernel<<<grid, kAttnThreads, kAttnSmem, s>>>(tq, tk, tv, out, P);
+  if (t.n_split > 1) {
+    const int rows = a.B * a.hq * a.nq;
+    attn_combine_kernel<<<(rows * 32 + 255) / 256, 256, 0, s>>>(t.part_o, t.part_ml, out, t.n_split, a.B, a.hq,
+                                                                 a.nq);
+  }
+}
+
+}  // namespace dg

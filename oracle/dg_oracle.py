@@ -340,13 +340,15 @@ class OracleModel:
             self.k_cache[req][l] = self.k_cache[req][l][:, :length]
             self.v_cache[req][l] = self.v_cache[req][l][:, :length]
 
-    def layer(self, h, li, req, pos, causal, n_layers_limit=None):
+    def layer(self, h, li, req, pos, causal, trace=None):
         """One transformer layer on the n rows of h at positions pos.
 
         Keys are the request's cache [0, P) followed by the n new rows.  With
         causal=True new row i sees cache + new rows <= i (prompt encoding and
         canvas hand-off, [P1 二], [P2 架构基础]); with causal=False every new row
         sees everything (the bidirectional canvas).  Returns (h_out, k_new, v_new).
+        If trace is a dict it receives the MoE input and the router margins
+        (recorded only; the arithmetic is unchanged).
         """
         c, L = self.cfg, self.weights["layers"][li]
         hq, hkv, hd = c["n_heads"], c["n_kv_heads"], c["head_dim"]
@@ -367,6 +369,9 @@ class OracleModel:
         o = attention(q, kk, vv, allowed).transpose(1, 0, 2).reshape(n, hq * hd)
         h = h + o @ L["wo"].T
         x = rms_norm(h, L["ffn_norm"], c["rms_eps"])
+        if trace is not None:
+            ids, _, g, margin = router(x, L["router_w"], L.get("router_b"), c["top_k"])
+            trace.update(moe_in=x, router_ids=ids, router_logits=g, router_margin=margin, h_attn=h)
         h = h + moe(x, L, c["top_k"])
         return h, k, v
 

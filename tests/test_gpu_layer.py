@@ -14,6 +14,9 @@ from tests._util import max_abs_rel, to_np
 W = synth.WORKLOADS["layer_bf16"]
 M = W["model"]
 TOL_BF16 = 2e-2
+# Router logits carry ~2^-8 relative error from the bf16 MoE input (~0.005 in
+# logit units here); decisions closer than 4x that are rounding-order ties.
+ROUTER_MARGIN = 0.02
 
 
 @pytest.mark.gpu
@@ -62,12 +65,21 @@ def test_full_width_layer_step(dg):
         dg.dg_synchronize(h)
         pos = W["cache_len"] + np.arange(n)
         hx = om.embed_tokens(canvas.numpy(), prev.numpy() if use_prev else None)
-        ref_h, _, _ = om.layer(hx, 0, 0, pos, causal=False)
-        err_h = max_abs_rel(to_np(hid), ref_h)
+        tr = {}
+        ref_h, _, _ = om.layer(hx, 0, 0, pos, causal=False, trace=tr)
+        # Tokens whose 8th/9th router logits are closer than the bf16 error of
+        # the router input may legitimately pick another expert: compare the
+        # rest, and require them to be the large majority.
+        safe = tr["router_margin"] > ROUTER_MARGIN
+        assert safe.mean() > 0.6, f"only {safe.mean():.2f} of tokens have a router margin > {ROUTER_MARGIN}"
+        got_h = to_np(hid)
+        den = np.max(np.abs(ref_h))
+        err_h = float(np.max(np.abs(got_h[safe] - ref_h[safe])) / den)
         assert err_h < TOL_BF16, f"layer output max-abs-rel {err_h} (self-cond={use_prev})"
-        x = O.rms_norm(ref_h[rows], om.weights["final_norm"], M["rms_eps"])
+        r = rows[safe[rows]]
+        x = O.rms_norm(ref_h[r], om.weights["final_norm"], M["rms_eps"])
         ref_l = O.lm_head(x, om.weights["embed"])
-        err_l = max_abs_rel(to_np(logits)[0][rows], ref_l)
+        err_l = max_abs_rel(to_np(logits)[0][r], ref_l)
         assert err_l < TOL_BF16, f"logits max-abs-rel {err_l}"
         assert 1 <= int(touched.item()) <= M["n_experts"]
     h.close()

@@ -37,7 +37,8 @@ def _compare(got, ref, b):
     low = check_decisions(got["x_hat"][b], ref["x_hat"], ref["sample_margin"], "x_hat")
     if ref["keep_margin"] > 1e-5:
         assert np.array_equal(got["keep"][b].astype(bool), ref["keep"])
-        assert np.array_equal(got["canvas"][b], ref["x_new"])
+        same = got["x_hat"][b] == ref["x_hat"]     # low-margin samples may differ
+        assert np.array_equal(got["canvas"][b][same], ref["x_new"][same])
     # whatever the keep set, re-noised positions hold the Philox token
     rn = got["keep"][b] == 0
     assert np.array_equal(got["canvas"][b][rn], ref["renoise"][rn])
