@@ -22,10 +22,10 @@ constexpr int kThreads = 256;
 constexpr int kPerThread = kChunk / kThreads;  // 16
 
 struct Partial {
-  float m;   // chunk max of z (T > 0) / of the scaled logit (T == 0)
-  float s;   // sum exp(z - m)              | T == 0: bits of the first arg-max index
-  float a;   // sum exp(z - m) * (z - m)    | T == 0: bits of the count of maxima
-  float pad;
+  float m;    // chunk max of z (T > 0) / of the scaled logit (T == 0)
+  int idx;    // T == 0: first arg-max index in the chunk
+  double s;   // sum exp(z - m)             | T == 0: count of maxima
+  double a;   // sum exp(z - m) * (z - m)
 };
 
 size_t sampler_workspace_bytes(int rows, int vocab) {
@@ -60,11 +60,20 @@ __device__ __forceinline__ int reg_index(int c0, int r, bool vec4) {
   return vec4 ? c0 + (threadIdx.x + (r >> 2) * kThreads) * 4 + (r & 3) : c0 + threadIdx.x + r * kThreads;
 }
 
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// The exponentials are fp32 (expf); every sum over the vocabulary is carried
+// in fp64 so the CDF that decides the sample is not limited by fp32 rounding
+// of 262144-term sums.
 __global__ void __launch_bounds__(kThreads) sampler_pass1(const float* __restrict__ logits, int vocab, float scale,
                                                           int argmax_mode, Partial* __restrict__ part) {
   __shared__ float red_m[kThreads / 32];
-  __shared__ float red_s[kThreads / 32];
-  __shared__ float red_a[kThreads / 32];
+  __shared__ double red_s[kThreads / 32];
+  __shared__ double red_a[kThreads / 32];
   __shared__ int red_i[kThreads / 32];
   __shared__ int red_c[kThreads / 32];
   const int c = blockIdx.x, row = blockIdx.y;
@@ -99,31 +108,31 @@ __global__ void __launch_bounds__(kThreads) sampler_pass1(const float* __restric
     if (threadIdx.x == 0) {
       for (int x = 1; x < kThreads / 32; ++x) { idx = min(idx, red_i[x]); cntm += red_c[x]; }
       p.m = m;
-      p.s = __int_as_float(idx);
-      p.a = __int_as_float(cntm);
-      p.pad = 0.f;
+      p.idx = idx;
+      p.s = (double)cntm;
+      p.a = 0.0;
       part[(size_t)row * n_chunks + c] = p;
     }
     return;
   }
-  float s = 0.f, a = 0.f;
+  double s = 0.0, a = 0.0;
   if (m > -INFINITY) {
 #pragma unroll
     for (int r = 0; r < kPerThread; ++r) {
       const float d = z[r] - m;
       const float e = expf(d);      // exp(-inf) = 0 for padding
-      s += e;
-      a += (e > 0.f) ? e * d : 0.f;
+      s += (double)e;
+      a += (e > 0.f) ? (double)e * (double)d : 0.0;
     }
   }
-  s = warp_sum(s);
-  a = warp_sum(a);
+  s = warp_sum_d(s);
+  a = warp_sum_d(a);
   if (lane == 0) { red_s[w] = s; red_a[w] = a; }
   __syncthreads();
   if (threadIdx.x == 0) {
-    s = 0.f; a = 0.f;
+    s = 0.0; a = 0.0;
     for (int x = 0; x < kThreads / 32; ++x) { s += red_s[x]; a += red_a[x]; }
-    p.m = m; p.s = s; p.a = a; p.pad = 0.f;
+    p.m = m; p.idx = 0; p.s = s; p.a = a;
     part[(size_t)row * n_chunks + c] = p;
   }
 }
@@ -133,9 +142,10 @@ __global__ void __launch_bounds__(kThreads) sampler_pass2(const float* __restric
                                                           uint64_t seed, uint32_t step, uint32_t block,
                                                           const Partial* __restrict__ part, int32_t* __restrict__ x_hat,
                                                           float* __restrict__ pmax, float* __restrict__ ent) {
-  __shared__ float sh_M, sh_S, sh_target, sh_P0;
+  __shared__ float sh_M;
+  __shared__ double sh_target, sh_P0;
   __shared__ int sh_c;
-  __shared__ float scan[kThreads];
+  __shared__ double scan[kThreads];
   __shared__ int sh_pick;
   __shared__ int sh_last;
   const int row = blockIdx.x;
@@ -147,78 +157,79 @@ __global__ void __launch_bounds__(kThreads) sampler_pass2(const float* __restric
     if (threadIdx.x == 0) {
       float M = -INFINITY;
       for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pr[c].m);
-      int idx = -1, cntm = 0;
+      int idx = -1;
+      double cntm = 0.0;
       for (int c = 0; c < n_chunks; ++c)
         if (pr[c].m == M) {
-          if (idx < 0) idx = __float_as_int(pr[c].s);
-          cntm += __float_as_int(pr[c].a);
+          if (idx < 0) idx = pr[c].idx;
+          cntm += pr[c].s;
         }
       x_hat[row] = idx;
-      pmax[row] = 1.0f / (float)cntm;
-      ent[row] = logf((float)cntm);
+      pmax[row] = (float)(1.0 / cntm);
+      ent[row] = (float)log(cntm);
     }
     return;
   }
   if (threadIdx.x == 0) {
     float M = -INFINITY;
     for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pr[c].m);
-    float S = 0.f, A = 0.f;
+    double S = 0.0, A = 0.0;
     for (int c = 0; c < n_chunks; ++c) {
-      const float f = expf(pr[c].m - M);
+      const double f = exp((double)pr[c].m - (double)M);
       S += pr[c].s * f;
-      A += (pr[c].a + (pr[c].m - M) * pr[c].s) * f;
+      A += (pr[c].a + ((double)pr[c].m - (double)M) * pr[c].s) * f;
     }
     const Philox4 w = sampler_words(seed, (uint32_t)i, step, block, (uint32_t)req_ids[b]);
-    const float target = unit_uniform(w.w[0]) * S;
+    const double target = (double)unit_uniform(w.w[0]) * S;
     // first chunk whose inclusive prefix exceeds the target (chunk order)
-    float P = 0.f;
+    double P = 0.0, P0 = 0.0;
     int cs = -1, last_pos = 0;
-    float P0 = 0.f;
     for (int c = 0; c < n_chunks; ++c) {
-      const float sc = pr[c].s * expf(pr[c].m - M);
-      if (sc > 0.f) last_pos = c;
+      const double sc = pr[c].s * exp((double)pr[c].m - (double)M);
+      if (sc > 0.0) last_pos = c;
       if (cs < 0 && P + sc > target) { cs = c; P0 = P; }
       P += sc;
     }
     if (cs < 0) { cs = last_pos; P0 = INFINITY; }  // rounding: no crossing -> last positive
-    sh_M = M; sh_S = S; sh_target = target; sh_P0 = P0; sh_c = cs;
-    pmax[row] = 1.0f / S;
-    ent[row] = logf(S) - A / S;
+    sh_M = M; sh_target = target; sh_P0 = P0; sh_c = cs;
+    pmax[row] = (float)(1.0 / S);
+    ent[row] = (float)(log(S) - A / S);
   }
   __syncthreads();
   // scan chunk sh_c in vocabulary order: thread t owns 16 consecutive elements
-  const float M = sh_M, target = sh_target, P0 = sh_P0;
+  const float M = sh_M;
+  const double target = sh_target, P0 = sh_P0;
   const int c0 = sh_c * kChunk;
   const float* lrow = logits + (size_t)row * vocab;
   float e[kPerThread];
-  float local = 0.f;
+  double local = 0.0;
   int lastpos = -1;
 #pragma unroll
   for (int r = 0; r < kPerThread; ++r) {
     const int j = c0 + threadIdx.x * kPerThread + r;
     const float v = (j < vocab) ? expf(lrow[j] * scale - M) : 0.f;
     e[r] = v;
-    local += v;
+    local += (double)v;
     if (v > 0.f) lastpos = j;
   }
   // inclusive scan of the per-thread sums in thread order (Hillis-Steele)
   scan[threadIdx.x] = local;
   __syncthreads();
   for (int o = 1; o < kThreads; o <<= 1) {
-    const float add = (threadIdx.x >= o) ? scan[threadIdx.x - o] : 0.f;
+    const double add = (threadIdx.x >= o) ? scan[threadIdx.x - o] : 0.0;
     __syncthreads();
     scan[threadIdx.x] += add;
     __syncthreads();
   }
   if (threadIdx.x == 0) sh_pick = 0x7fffffff;
   __syncthreads();
-  const float before = P0 + (scan[threadIdx.x] - local);
+  const double before = P0 + (scan[threadIdx.x] - local);
   if (before <= target && before + local > target) {
-    float run = before;
+    double run = before;
     int pick = -1;
 #pragma unroll
     for (int r = 0; r < kPerThread; ++r) {
-      run += e[r];
+      run += (double)e[r];
       if (pick < 0 && run > target) pick = c0 + threadIdx.x * kPerThread + r;
     }
     if (pick < 0) pick = lastpos;  // the thread sum crossed but the element walk fell short
