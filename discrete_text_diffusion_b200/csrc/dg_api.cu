@@ -14,7 +14,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/dg.h"
+#include "dg.h"
 #include "kernels.h"
 
 using namespace dg;
@@ -236,6 +236,14 @@ int grouped_tile(const dg_handle* H, int T) {
   return 64;
 }
 
+// Pipeline shape of a tensor-core GEMM launch: two 64-wide K blocks per
+// stage; narrow token tiles run two CTAs per SM (a single CTA cannot keep
+// enough L2 reads in flight), wide ones one CTA with a deeper pipeline.
+void tc_policy(TcGemm& g) {
+  g.ksub = 2;
+  g.ctas_per_sm = g.ntile <= 128 ? 2 : 1;
+}
+
 // ------------------------------------------------------------ GEMM helpers
 // out = x[T, K] * W^T (W [n_out, K]) for the dense projections.
 void dense_gemm(dg_handle* H, int cls, const void* x, const CUtensorMap* mx, const void* w, const CUtensorMap* mw,
@@ -256,6 +264,7 @@ void dense_gemm(dg_handle* H, int cls, const void* x, const CUtensorMap* mx, con
   g.out = out;
   g.ld_out = ld_out;
   g.err = H->d_err;
+  tc_policy(g);
   launch_gemm_tc(*mw, H->m_dummy, H->m_dummy, *mx, g, H->num_sms, H->stream);
 }
 
@@ -286,6 +295,7 @@ void qkv_gemm(dg_handle* H, int l, int T) {
   g.out = H->qkv;
   g.ld_out = ld;
   g.err = H->d_err;
+  tc_policy(g);
   const LayerMaps& M = H->lmaps[l];
   launch_gemm_tc(M.wq, M.wk, M.wv, H->m_xn, g, H->num_sms, H->stream);
 }
@@ -314,6 +324,8 @@ void moe_gemms(dg_handle* H, int l, int T) {
       g.out = H->hb;
       g.ld_out = c.d_ff;
       g.err = H->d_err;
+      tc_policy(g);
+  tc_policy(g);
       launch_gemm_tc(H->lmaps[l].gate, H->lmaps[l].up, H->m_dummy, H->m_xp, g, H->num_sms, H->stream);
     }
   }
@@ -337,6 +349,8 @@ void moe_gemms(dg_handle* H, int l, int T) {
       g.ld_out = c.d_model;
       g.row_map = H->perm;
       g.err = H->d_err;
+      tc_policy(g);
+  tc_policy(g);
       launch_gemm_tc(H->lmaps[l].down, H->m_dummy, H->m_dummy, H->m_hb, g, H->num_sms, H->stream);
     }
   }
@@ -968,6 +982,7 @@ int dg_selftest_gemm(dg_handle* H, const void* x, const void* w, int T, int M, i
   g.out = out;
   g.ld_out = M;
   g.err = H->d_err;
+  tc_policy(g);
   launch_gemm_tc(mw, mw, mw, mx, g, H->num_sms, H->stream);
   H->launches += 1;
   return check_launch(H, "selftest gemm");

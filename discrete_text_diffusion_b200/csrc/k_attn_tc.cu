@@ -10,12 +10,13 @@
 //   warp 1 lane 0: MMA issuer.  S_j = Q K_j^T (M 128, N 64, K 256) into one of
 //     two TMEM score buffers, one tile ahead of O += P_j V_j (M 128, N 256,
 //     K 64) with O resident in TMEM (256 columns).
-//   warps 2-5: softmax.  Thread = query row.  Scores are scaled to log2 units;
-//     the running max is only raised when a tile exceeds it by more than 8
-//     (then O and the running sum are rescaled through TMEM), so most tiles
-//     need no correction.  P (bf16) is written to one of two swizzled shared
-//     buffers for the PV MMA.  At the end O / l goes out as bf16, or O, max
-//     and sum go to the split workspace for the combine kernel.
+//   warps 2-9: softmax, two threads per query row (32 keys each).  Scores
+//     are scaled to log2 units; the running max is only raised when a tile
+//     exceeds it by more than 8 (then O and the running sum are rescaled
+//     through TMEM), so most tiles need no correction.  P (bf16) is written
+//     back into TMEM over its own scores and is the A operand of the PV MMA,
+//     so it never touches shared memory.  At the end O / l goes out as bf16,
+//     or O, max and sum go to the split workspace for the combine kernel.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -25,15 +26,15 @@
 
 namespace dg {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;   // producer, MMA issuer, 8 softmax warps
 constexpr int kQTile = 128;
 constexpr int kKTile = 64;
 constexpr int kHd = 256;
 constexpr int kQBytes = kQTile * kHd * 2;   // 64 KB
 constexpr int kKBytes = kKTile * kHd * 2;   // 32 KB
 constexpr int kVBytes = kHd * kKTile * 2;   // 32 KB
-constexpr int kPBytes = kQTile * kKTile * 2;  // 16 KB
-constexpr int kAttnSmem = 1024 + kQBytes + 2 * kKBytes + 2 * kVBytes + 2 * kPBytes + 256;
+constexpr int kRedBytes = 256 * 4;           // per-row exchange between the two halves
+constexpr int kAttnSmem = 1008 + kQBytes + 2 * kKBytes + 2 * kVBytes + kRedBytes + 128;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct AttnTcParams {
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (ntiles == 0) {
     // empty split (causal tail): contributes nothing to the combine
-    if (warp >= 2) {
+    if (warp >= 2 && warp < 6) {
       const int r = (warp & 3) * 32 + lane;
       const int qi = q0 + r;
       if (qi < a.nq && P.t.n_split > 1) {
@@ -84,13 +85,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sQ = base;
   uint8_t* sK = sQ + kQBytes;            // [2][kKBytes]
   uint8_t* sV = sK + 2 * kKBytes;        // [2][kVBytes]
-  uint8_t* sP = sV + 2 * kVBytes;        // [2][kPBytes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
+  float* red = reinterpret_cast<float*>(sV + 2 * kVBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * kVBytes + kRedBytes);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;     // [2]
   uint64_t* kv_empty = bars + 3;    // [2]
   uint64_t* s_full = bars + 5;      // [2]
-  uint64_t* s_empty = bars + 7;     // [2]
   uint64_t* p_full = bars + 9;      // [2]
   uint64_t* pv_done = bars + 11;    // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
@@ -102,8 +102,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 256);
       mbar_init(&pv_done[i], 1);
     }
     fence_mbar_init();
@@ -148,8 +147,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     auto issue_s = [&](int j) -> bool {
       const int s = j & 1;
       const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+      // S_j reuses the TMEM columns of P_{j-2}; PV_{j-2} was issued earlier,
+      // and tcgen05.mma of one thread run in issue order.
       if (!mbar_wait(&kv_full[s], ph, err, kErrTimeoutAttn)) return false;
-      if (!mbar_wait(&s_empty[s], ph ^ 1u, err, kErrTimeoutAttn)) return false;
       tc_fence_after();
       const uint32_t k_base = smem_u32(sK + s * kKBytes);
 #pragma unroll
@@ -167,18 +167,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int s = j & 1;
       if (!mbar_wait(&p_full[s], (uint32_t)(j >> 1) & 1u, err, kErrTimeoutAttn)) break;
       tc_fence_after();
-      const uint32_t p_base = smem_u32(sP + s * kPBytes);
+      // O += P_j V_j with P_j (bf16, 32 columns) read from TMEM where S_j was
       const uint32_t v_base = smem_u32(sV + s * kVBytes);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        umma_bf16(tO, sdesc_k_sw128(p_base + 32u * k), sdesc_k_sw128(v_base + 32u * k), idesc_o,
-                  (j > 0 || k > 0) ? 1u : 0u);
+        umma_bf16_ts(tO, tS + (uint32_t)(s * kKTile + 8 * k), sdesc_k_sw128(v_base + 32u * k), idesc_o,
+                     (j > 0 || k > 0) ? 1u : 0u);
       umma_commit(&pv_done[s]);
       umma_commit(&kv_empty[s]);
     }
   } else if (warp >= 2) {
     // ----------------------------------------------------------- softmax
+    // 8 warps: thread (quarter, lane) of half hf owns query row r and keys
+    // [32 hf, 32 hf + 32) of each 64-key tile, and O columns [128 hf, +128).
+    // The two halves of a row agree on the tile max through shared memory.
     const int quarter = warp & 3;
+    const int hf = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int qi = q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -190,24 +194,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t ph = (uint32_t)(j >> 1) & 1u;
       if (!mbar_wait(&s_full[s], ph, err, kErrTimeoutAttn)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld32(tS + lane_off + (uint32_t)(s * kKTile), *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(tS + lane_off + (uint32_t)(s * kKTile + 32), *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tc_fence_before();
-      mbar_arrive(&s_empty[s]);
-      const int key0 = (t_begin + j) * kKTile;
-      float x[64];
-      float tmax = -INFINITY;
+      uint32_t sv[32];
+      tmem_ld32(tS + lane_off + (uint32_t)(s * kKTile + hf * 32), sv);
+      const int kbase = (t_begin + j) * kKTile + hf * 32;
+      float x[32];
+      float hmax = -INFINITY;
+      if (kbase + 32 <= row_lim) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float v = (key0 + c < row_lim) ? __uint_as_float(sv[c]) * P.scale_log2 : -INFINITY;
-        x[c] = v;
-        tmax = fmaxf(tmax, v);
+        for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(sv[c]) * P.scale_log2; hmax = fmaxf(hmax, x[c]); }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          x[c] = (kbase + c < row_lim) ? __uint_as_float(sv[c]) * P.scale_log2 : -INFINITY;
+          hmax = fmaxf(hmax, x[c]);
+        }
       }
+      // tile max of the row: exchange with the other half.  The barrier also
+      // orders both halves' reads of S before any P write into these columns.
+      red[hf * 128 + r] = hmax;
+      named_barrier_sync(1, 256);
+      const float tmax = fmaxf(hmax, red[(hf ^ 1) * 128 + r]);
+      named_barrier_sync(1, 256);   // both halves have read before the buffer is reused
       // raise the running max only when this tile exceeds it by the threshold
       const bool raise = tmax > m_run + kRescaleThreshold;
       const float m_new = raise ? tmax : m_run;
-      const float alpha = (raise && m_run > -INFINITY) ? exp2f(m_run - m_new) : 1.f;
+      const float alpha = (raise && m_run > -INFINITY) ? fast_exp2(m_run - m_new) : 1.f;
       if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
         // O of rows in this warp must be rescaled: wait until PV_{j-1} landed
         if (!mbar_wait(&pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, err, kErrTimeoutAttn)) {
@@ -216,78 +227,83 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < kHd; c0 += 32) {
+        for (int c0 = 0; c0 < kHd / 2; c0 += 32) {
           uint32_t ov[32];
-          tmem_ld32(tO + lane_off + (uint32_t)c0, ov);
+          const uint32_t ta = tO + lane_off + (uint32_t)(hf * (kHd / 2) + c0);
+          tmem_ld32(ta, ov);
 #pragma unroll
           for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-          tmem_st32(tO + lane_off + (uint32_t)c0, ov);
+          tmem_st32(ta, ov);
         }
         tmem_st_wait();
       }
       l_run *= alpha;
       m_run = m_new;
-      // P_j -> shared buffer s, once PV_{j-2} has finished reading it
-      if (j >= 2 && !mbar_wait(&pv_done[s], (uint32_t)((j - 2) >> 1) & 1u, err, kErrTimeoutAttn)) {
-        ok = false;
-        break;
-      }
-      uint8_t* prow = sP + s * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
-      float lsum = 0.f;
+      // P_j (bf16) overwrites the first 32 columns of S_j's TMEM buffer:
+      // half hf's 32 keys are 16 packed columns at 16 hf.
+      uint32_t pk[16];
+      float ps[16];
+      const bool live = m_run > -INFINITY;
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = (m_run > -INFINITY) ? exp2f(x[c8 * 8 + 2 * e] - m_run) : 0.f;
-          const float p1 = (m_run > -INFINITY) ? exp2f(x[c8 * 8 + 2 * e + 1] - m_run) : 0.f;
-          const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
-          lsum += __low2float(pp) + __high2float(pp);   // sum what the MMA will see
-          pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
-        }
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int e = 0; e < 16; ++e) {
+        const float p0 = live ? fast_exp2(x[2 * e] - m_run) : 0.f;
+        const float p1 = live ? fast_exp2(x[2 * e + 1] - m_run) : 0.f;
+        const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+        pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+        ps[e] = __low2float(pp) + __high2float(pp);   // sum what the MMA will see
       }
-      l_run += lsum;
-      fence_proxy_async_smem();
+      tmem_st16_wait(tS + lane_off + (uint32_t)(s * kKTile + hf * 16), pk);
+#pragma unroll
+      for (int w2 = 8; w2 > 0; w2 >>= 1)
+#pragma unroll
+        for (int e = 0; e < w2; ++e) ps[e] += ps[e + w2];
+      l_run += ps[0];
       tc_fence_before();
       mbar_arrive(&p_full[s]);
+    }
+    // the row sum is the sum of both halves
+    if (ok) {
+      red[hf * 128 + r] = l_run;
+      named_barrier_sync(1, 256);
+      l_run += red[(hf ^ 1) * 128 + r];
     }
     if (ok) ok = mbar_wait(&pv_done[(ntiles - 1) & 1], (uint32_t)((ntiles - 1) >> 1) & 1u, err, kErrTimeoutAttn);
     if (ok) {
       tc_fence_after();
       const bool valid = qi < a.nq;
+      const int cbase = hf * (kHd / 2);
       if (P.t.n_split == 1) {
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        __nv_bfloat16* op = out + ((size_t)b * a.nq + qi) * ((size_t)a.hq * kHd) + (size_t)h * kHd;
+        __nv_bfloat16* op = out + ((size_t)b * a.nq + qi) * ((size_t)a.hq * kHd) + (size_t)h * kHd + cbase;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kHd; c0 += 32) {
+        for (int c0 = 0; c0 < kHd / 2; c0 += 32) {
           uint32_t ov[32];
-          tmem_ld32(tO + lane_off + (uint32_t)c0, ov);
+          tmem_ld32(tO + lane_off + (uint32_t)(cbase + c0), ov);
           if (valid) {
 #pragma unroll
             for (int c = 0; c < 32; c += 8) {
-              uint32_t pk[4];
+              uint32_t pq[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const __nv_bfloat162 pp = __floats2bfloat162_rn(__uint_as_float(ov[c + 2 * e]) * inv,
                                                                 __uint_as_float(ov[c + 2 * e + 1]) * inv);
-                pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+                pq[e] = *reinterpret_cast<const uint32_t*>(&pp);
               }
-              *reinterpret_cast<uint4*>(op + c0 + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              *reinterpret_cast<uint4*>(op + c0 + c) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
             }
           }
         }
       } else {
         const size_t pr = (size_t)split * a.B * a.hq * a.nq + row_id + qi;
-        if (valid) {
+        if (valid && hf == 0) {
           P.t.part_ml[2 * pr] = m_run;
           P.t.part_ml[2 * pr + 1] = l_run;
         }
-        float* po = P.t.part_o + pr * kHd;
+        float* po = P.t.part_o + pr * kHd + cbase;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kHd; c0 += 32) {
+        for (int c0 = 0; c0 < kHd / 2; c0 += 32) {
           uint32_t ov[32];
-          tmem_ld32(tO + lane_off + (uint32_t)c0, ov);
+          tmem_ld32(tO + lane_off + (uint32_t)(cbase + c0), ov);
           if (valid) {
 #pragma unroll
             for (int c = 0; c < 32; c += 4)

@@ -38,28 +38,54 @@ constexpr int kBoxN = 32;
 constexpr int kTcThreads = 192;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kMaxSmem = 232448;        // 227 KB opt-in limit per CTA
+#ifndef DG_GEMM_MAX_STAGES
+#define DG_GEMM_MAX_STAGES 8            // shared-memory pipeline depth cap
+#endif
+#ifndef DG_GEMM_KSUB
+#define DG_GEMM_KSUB 1                  // default 64-wide K blocks per stage
+#endif
+#ifndef DG_GEMM_CTAS_PER_SM
+#define DG_GEMM_CTAS_PER_SM 1           // default co-resident CTAs per SM
+#endif
+constexpr int kSmemPerSm = 233472;      // 228 KB of shared memory per SM
+#ifndef DG_GEMM_WARP_ISSUE
+#define DG_GEMM_WARP_ISSUE 1            // spread a stage's TMA boxes over the producer warp
+#endif
 
 struct TcLayout {
   int n_a;          // weight operands per stage (1 or 2)
+  int ksub;         // 64-wide K blocks per stage
   int stage_bytes;
   int stages;
   int acc_cols;     // TMEM columns of one accumulator buffer (all operands)
   int n_acc_buf;
   int tmem_cols;    // power of two >= 32
   int smem_bytes;
+  int per_sm;       // CTAs per SM the grid is sized for
 };
 
 static TcLayout tc_layout(const TcGemm& p) {
   TcLayout L;
   L.n_a = (p.mode == 1) ? 2 : 1;
-  L.stage_bytes = L.n_a * kABytes + p.ntile * kBK * 2;
-  const int overhead = 1024 /*align*/ + 1024 /*barriers*/;
-  L.stages = std::min(8, (kMaxSmem - overhead) / L.stage_bytes);
   L.acc_cols = L.n_a * p.ntile;
-  L.n_acc_buf = (2 * L.acc_cols <= 512) ? 2 : 1;
-  int need = L.n_acc_buf * L.acc_cols;
-  L.tmem_cols = 32;
-  while (L.tmem_cols < need) L.tmem_cols <<= 1;
+  L.per_sm = std::max(1, std::min(3, p.ctas_per_sm > 0 ? p.ctas_per_sm : DG_GEMM_CTAS_PER_SM));
+  L.ksub = std::max(1, std::min(4, p.ksub > 0 ? p.ksub : DG_GEMM_KSUB));
+  const int overhead = 1024 /*align*/ + 1024 /*barriers*/;
+  for (;;) {
+    // TMEM: every co-resident CTA holds its accumulators
+    L.n_acc_buf = (L.per_sm * 2 * L.acc_cols <= 512) ? 2 : 1;
+    const int need = L.n_acc_buf * L.acc_cols;
+    L.tmem_cols = 32;
+    while (L.tmem_cols < need) L.tmem_cols <<= 1;
+    const int budget = std::min(kMaxSmem, kSmemPerSm / L.per_sm - 1024);
+    L.stage_bytes = L.ksub * (L.n_a * kABytes + p.ntile * kBK * 2);
+    L.stages = std::min(DG_GEMM_MAX_STAGES, (budget - overhead) / L.stage_bytes);
+    if (L.per_sm * L.tmem_cols <= 512 && L.stages >= 2) break;
+    if (L.ksub > 1) { --L.ksub; continue; }
+    if (L.per_sm > 1) { --L.per_sm; continue; }
+    L.stages = std::max(L.stages, 1);
+    break;
+  }
   L.smem_bytes = overhead + L.stages * L.stage_bytes;
   return L;
 }
@@ -72,7 +98,7 @@ int gemm_tc_smem_bytes(const TcGemm& p, int* stages) {
 
 struct TcKParams {
   TcGemm g;
-  int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, n_ttiles;
+  int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, n_ttiles, ksub;
 };
 
 __device__ __forceinline__ void tc_item(const TcKParams& P, int item, int& m0, int& e, int& row0, int& rows) {
@@ -92,7 +118,7 @@ __device__ __forceinline__ void tc_item(const TcKParams& P, int item, int& m0, i
   }
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap ta1,
                    const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb,
                    const TcKParams P) {
@@ -131,38 +157,62 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles : (*g.n_work) * P.n_mtiles;
-  const int nk = g.K / kBK;
+  const int nk = g.K / kBK;                       // 64-wide K blocks
+  const int ksub = P.ksub;                        // K blocks per pipeline stage
+  const int nst = (nk + ksub - 1) / ksub;         // stages per output tile
   const int n_a = (g.mode == 1) ? 2 : 1;
+  const int b_sub = g.ntile * kBK * 2;            // bytes of one token sub-tile
+  // stage layout: [ksub x A0][ksub x A1 (mode 1)][ksub x B], each sub 1024-aligned
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Lane 0 waits for the slot and posts the byte count; then the stage's
+    // boxes (weights and token rows of every K block) are spread over the
+    // lanes of the warp, so they are issued to the TMA unit side by side.
     uint32_t kiter = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
       int m0, e, row0, rows;
       tc_item(P, item, m0, e, row0, rows);
       const int nb = (rows + kBoxN - 1) / kBoxN;
-      const uint32_t tx = (uint32_t)(n_a * kABytes + nb * kBoxN * kBK * 2);
       const CUtensorMap* am = &ta0;
       int am0 = m0;
       if (g.mode == 0) {
         if (m0 >= g.seg2) { am = &ta2; am0 = m0 - g.seg2; }
         else if (m0 >= g.seg1) { am = &ta1; am0 = m0 - g.seg1; }
       }
-      for (int kb = 0; kb < nk; ++kb, ++kiter) {
+      const int per_u = n_a + nb;  // boxes per K block
+      for (int j = 0; j < nst; ++j, ++kiter) {
         const int s = kiter % P.stages;
         const uint32_t ph = (kiter / P.stages) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) { ok = false; break; }
+        const int kb0 = j * ksub;
+        const int nsub = min(ksub, nk - kb0);
         uint8_t* st = stage0 + (size_t)s * P.stage_bytes;
-        mbar_expect_tx(&full[s], tx);
-        if (g.mode == 0) {
-          tma_load_2d(st, am, &full[s], kb * kBK, am0);
-        } else {
-          tma_load_3d(st, &ta0, &full[s], kb * kBK, m0, e);
-          if (g.mode == 1) tma_load_3d(st + kABytes, &ta1, &full[s], kb * kBK, m0, e);
+        if (lane == 0) mbar_expect_tx(&full[s], (uint32_t)(nsub * (n_a * kABytes + nb * kBoxN * kBK * 2)));
+        __syncwarp();
+#if DG_GEMM_WARP_ISSUE
+        for (int task = lane; task < nsub * per_u; task += 32) {
+#else
+        for (int task = 0; lane == 0 && task < nsub * per_u; ++task) {
+#endif
+          const int u = task / per_u, r = task - u * per_u;
+          const int kc = (kb0 + u) * kBK;
+          if (r == 0) {
+            if (g.mode == 0) tma_load_2d(st + u * kABytes, am, &full[s], kc, am0);
+            else tma_load_3d(st + u * kABytes, &ta0, &full[s], kc, m0, e);
+          } else if (r < n_a) {
+            tma_load_3d(st + (ksub + u) * kABytes, &ta1, &full[s], kc, m0, e);
+          } else {
+            const int i = r - n_a;
+            tma_load_2d(st + n_a * ksub * kABytes + u * b_sub + i * kBoxN * kBK * 2, &tb, &full[s], kc,
+                        row0 + i * kBoxN);
+          }
         }
-        uint8_t* sb = st + n_a * kABytes;
-        for (int i = 0; i < nb; ++i) tma_load_2d(sb + i * kBoxN * kBK * 2, &tb, &full[s], kb * kBK, row0 + i * kBoxN);
+        __syncwarp();
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -180,19 +230,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&acc_empty[ab], (use & 1u) ^ 1u, err, kErrTimeoutMma)) break;
       tc_fence_after();
       const uint32_t d0 = tmem_base + (uint32_t)(ab * P.acc_cols);
-      for (int kb = 0; kb < nk; ++kb, ++kiter) {
+      for (int j = 0; j < nst; ++j, ++kiter) {
         const int s = kiter % P.stages;
         const uint32_t ph = (kiter / P.stages) & 1u;
         if (!mbar_wait(&full[s], ph, err, kErrTimeoutMma)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sa = smem_u32(stage0 + (size_t)s * P.stage_bytes);
-        const uint32_t sb = sa + (uint32_t)(n_a * kABytes);
+        const int nsub = min(ksub, nk - j * ksub);
+        const uint32_t st = smem_u32(stage0 + (size_t)s * P.stage_bytes);
+        for (int u = 0; u < nsub; ++u) {
+          const uint32_t sa = st + (uint32_t)(u * kABytes);
+          const uint32_t sa1 = st + (uint32_t)((ksub + u) * kABytes);
+          const uint32_t sb = st + (uint32_t)(n_a * ksub * kABytes + u * b_sub);
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          const uint64_t bdesc = sdesc_k_sw128(sb + 32u * k);
-          const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-          umma_bf16(d0, sdesc_k_sw128(sa + 32u * k), bdesc, idesc, acc);
-          if (n_a == 2) umma_bf16(d0 + (uint32_t)g.ntile, sdesc_k_sw128(sa + kABytes + 32u * k), bdesc, idesc, acc);
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t bdesc = sdesc_k_sw128(sb + 32u * k);
+            const uint32_t acc = (j > 0 || u > 0 || k > 0) ? 1u : 0u;
+            umma_bf16(d0, sdesc_k_sw128(sa + 32u * k), bdesc, idesc, acc);
+            if (n_a == 2) umma_bf16(d0 + (uint32_t)g.ntile, sdesc_k_sw128(sa1 + 32u * k), bdesc, idesc, acc);
+          }
         }
         umma_commit(&empty[s]);
       }
@@ -275,6 +330,7 @@ void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensor
   TcKParams P;
   P.g = g;
   P.stages = L.stages;
+  P.ksub = L.ksub;
   P.stage_bytes = L.stage_bytes;
   P.acc_cols = L.acc_cols;
   P.n_acc_buf = L.n_acc_buf;
@@ -288,9 +344,7 @@ void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensor
     cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     attr_bytes = kMaxSmem;
   }
-  int per_sm = std::max(1, std::min(kMaxSmem / L.smem_bytes, 512 / L.tmem_cols));
-  per_sm = std::min(per_sm, 2);
-  const int grid = std::min(total, num_sms * per_sm);
+  const int grid = std::min(total, num_sms * L.per_sm);
   gemm_tc_kernel<<<grid, kTcThreads, L.smem_bytes, s>>>(a0, a1, a2, b, P);
 }
 

@@ -108,6 +108,8 @@ struct TcGemm {
   const float* bias;
   const int32_t* row_map;
   int* err;
+  int ksub;          // 64-wide K blocks per pipeline stage (0 = build default)
+  int ctas_per_sm;   // co-resident CTAs the grid is sized for (0 = build default)
 };
 void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
                     const TcGemm& p, int num_sms, cudaStream_t s);
