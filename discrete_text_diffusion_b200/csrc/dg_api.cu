@@ -53,6 +53,36 @@ bool tmap_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// A row-major [rows, cols] bf16 matrix seen as chunks of 64 columns:
+// dims (64, rows, cols/64), strides (row pitch, 128 B); box (64, box_rows, nz)
+// fetches nz consecutive 64-column chunks of box_rows rows with ONE TMA
+// instruction, landing as nz [box_rows x 128 B] 128-byte-swizzled tiles.
+// (TMA throughput per CTA grows with the bytes of each instruction.)
+bool tmap_chunks(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_pitch_elems,
+                 uint32_t box_rows, uint32_t nz) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {row_pitch_elems * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, nz};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// The same for n2 stacked matrices [n2][rows][cols]: dims (64, rows, cols/64, n2).
+bool tmap_chunks4(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t n2, uint32_t box_rows,
+                  uint32_t nz) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, rows, cols / 64, n2};
+  cuuint64_t strides[3] = {cols * 2, 128, cols * rows * 2};
+  cuuint32_t box[4] = {64, box_rows, nz, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 // 3D bf16 map over [n2, rows, cols], box (64, box_rows, 1).
 bool tmap_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t n2, uint32_t box_rows) {
   EncodeTiledFn fn = get_encode_fn();
@@ -76,8 +106,18 @@ const char* kProfNames[PC_COUNT] = {"embed",  "dense_gemm", "rope_scatter", "att
 
 }  // namespace
 
+// A weight matrix's TMA maps for 2- and 4-chunk (64-column) boxes of 128 rows.
+struct WMap {
+  CUtensorMap k2, k4;
+};
 struct LayerMaps {
-  CUtensorMap wq, wk, wv, wo, router, gate, up, down;
+  WMap wq, wk, wv, wo, router, gate, up, down;
+};
+struct BMapEntry {
+  const void* p;
+  uint64_t cols, rows;
+  int ntile, ksub;
+  CUtensorMap m;
 };
 
 struct dg_handle {
@@ -94,7 +134,9 @@ struct dg_handle {
   const float* final_norm = nullptr;
   std::vector<dg_layer_weights> lw;
   std::vector<LayerMaps> lmaps;
-  CUtensorMap m_embed{}, m_wsc{}, m_dummy{};
+  WMap m_embed{}, m_wsc{};
+  std::vector<BMapEntry> bmaps;   // token-operand maps, built on first use
+  bool bad_launch = false;        // a tensor map or GEMM tiling was rejected
   // KV cache (owned)
   void* kc = nullptr;
   void* vt = nullptr;
@@ -122,7 +164,6 @@ struct dg_handle {
   float* y = nullptr;
   float* logits = nullptr;
   float2* rope = nullptr;
-  CUtensorMap m_xn{}, m_eprev{}, m_attn{}, m_xp{}, m_hb{};
   // tensor-core attention (bf16, head dim 256)
   bool attn_tc = false;
   CUtensorMap m_q{};
@@ -230,24 +271,56 @@ int pick_ntile(int n_mtiles, int T, int num_sms) {
 
 int grouped_tile(const dg_handle* H, int T) {
   if (!H->bf16) return 64;
+  // at most 128 rows: the gate + up weights and a 256-row token tile would
+  // not fit a two-stage pipeline with two-chunk TMA boxes
   const double avg = (double)T * H->c.top_k / H->c.n_experts;
-  if (avg > 128) return 256;
-  if (avg > 48) return 128;
-  return 64;
+  return avg > 48 ? 128 : 64;
 }
 
-// Pipeline shape of a tensor-core GEMM launch: two 64-wide K blocks per
-// stage; narrow token tiles run two CTAs per SM (a single CTA cannot keep
-// enough L2 reads in flight), wide ones one CTA with a deeper pipeline.
-void tc_policy(TcGemm& g) {
-  g.ksub = 2;
-  g.ctas_per_sm = g.ntile <= 128 ? 2 : 1;
+// Pipeline shape of a tensor-core GEMM launch.  TMA throughput per CTA is
+// set by the bytes of each TMA instruction, so every stage loads each
+// operand with one instruction of ksub 64-column chunks: 4 chunks (64 KB of
+// weights) for narrow token tiles, 2 chunks when the token tile is wide or
+// two weight operands share the stage.
+#ifndef DG_NARROW_KSUB
+#define DG_NARROW_KSUB 2      // chunks per weight box when the token tile is <= 64 rows
+#endif
+#ifndef DG_NARROW_CTAS
+#define DG_NARROW_CTAS 2      // CTAs per SM when the token tile is <= 64 rows
+#endif
+int ksub_for(int mode, int ntile) { return (mode == 1 || ntile > 64) ? 2 : DG_NARROW_KSUB; }
+int ctas_for(int ntile) { return ntile <= 64 ? DG_NARROW_CTAS : 1; }
+
+const CUtensorMap& pick(const WMap& w, int ksub) { return ksub == 4 ? w.k4 : w.k2; }
+
+// Token-operand map of a (rows x cols) activation buffer for a tile of ntile
+// rows and ksub chunks, built on first use and kept for the handle's life.
+const CUtensorMap* bmap(dg_handle* H, const void* p, uint64_t cols, uint64_t rows, int ntile, int ksub) {
+  for (const auto& e : H->bmaps)
+    if (e.p == p && e.cols == cols && e.rows == rows && e.ntile == ntile && e.ksub == ksub) return &e.m;
+  BMapEntry e;
+  e.p = p;
+  e.cols = cols;
+  e.rows = rows;
+  e.ntile = ntile;
+  e.ksub = ksub;
+  if (!tmap_chunks(&e.m, p, cols, rows, cols, (uint32_t)ntile, (uint32_t)ksub)) {
+    H->bad_launch = true;
+    return nullptr;
+  }
+  H->bmaps.push_back(e);
+  return &H->bmaps.back().m;
+}
+
+void run_tc(dg_handle* H, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap* b,
+            TcGemm& g) {
+  if (!b || launch_gemm_tc(a0, a1, a2, *b, g, H->num_sms, H->stream) != 0) H->bad_launch = true;
 }
 
 // ------------------------------------------------------------ GEMM helpers
 // out = x[T, K] * W^T (W [n_out, K]) for the dense projections.
-void dense_gemm(dg_handle* H, int cls, const void* x, const CUtensorMap* mx, const void* w, const CUtensorMap* mw,
-                int T, int n_out, int K, Epi epi, void* out, int ld_out) {
+void dense_gemm(dg_handle* H, int cls, const void* x, const void* w, const WMap* mw, int T, int n_out, int K,
+                Epi epi, void* out, int ld_out) {
   ProfScope ps(H, cls);
   if (!H->bf16) {
     launch_gemm_simt<float>((const float*)x, (const float*)w, T, n_out, K, epi, out, ld_out, nullptr, H->stream);
@@ -264,8 +337,10 @@ void dense_gemm(dg_handle* H, int cls, const void* x, const CUtensorMap* mx, con
   g.out = out;
   g.ld_out = ld_out;
   g.err = H->d_err;
-  tc_policy(g);
-  launch_gemm_tc(*mw, H->m_dummy, H->m_dummy, *mx, g, H->num_sms, H->stream);
+  g.ksub = ksub_for(0, g.ntile);
+  g.ctas_per_sm = ctas_for(g.ntile);
+  const CUtensorMap& a = pick(*mw, g.ksub);
+  run_tc(H, a, a, a, bmap(H, x, K, H->T_max, g.ntile, g.ksub), g);
 }
 
 void qkv_gemm(dg_handle* H, int l, int T) {
@@ -295,9 +370,11 @@ void qkv_gemm(dg_handle* H, int l, int T) {
   g.out = H->qkv;
   g.ld_out = ld;
   g.err = H->d_err;
-  tc_policy(g);
+  g.ksub = ksub_for(0, g.ntile);
+  g.ctas_per_sm = ctas_for(g.ntile);
   const LayerMaps& M = H->lmaps[l];
-  launch_gemm_tc(M.wq, M.wk, M.wv, H->m_xn, g, H->num_sms, H->stream);
+  run_tc(H, pick(M.wq, g.ksub), pick(M.wk, g.ksub), pick(M.wv, g.ksub),
+         bmap(H, H->xn, c.d_model, H->T_max, g.ntile, g.ksub), g);
 }
 
 void moe_gemms(dg_handle* H, int l, int T) {
@@ -305,6 +382,7 @@ void moe_gemms(dg_handle* H, int l, int T) {
   const dg_layer_weights& L = H->lw[l];
   const int tile = grouped_tile(H, T);
   const int n_work_max = c.n_experts + (T * c.top_k + tile - 1) / tile;
+  const uint64_t rows = (uint64_t)H->T_max * c.top_k;
   {
     ProfScope ps(H, PC_MOE_UP);
     if (!H->bf16) {
@@ -324,9 +402,11 @@ void moe_gemms(dg_handle* H, int l, int T) {
       g.out = H->hb;
       g.ld_out = c.d_ff;
       g.err = H->d_err;
-      tc_policy(g);
-  tc_policy(g);
-      launch_gemm_tc(H->lmaps[l].gate, H->lmaps[l].up, H->m_dummy, H->m_xp, g, H->num_sms, H->stream);
+      g.ksub = ksub_for(1, tile);
+      g.ctas_per_sm = ctas_for(g.ntile);
+      const LayerMaps& M = H->lmaps[l];
+      run_tc(H, pick(M.gate, g.ksub), pick(M.up, g.ksub), pick(M.up, g.ksub),
+             bmap(H, H->xp, c.d_model, rows, tile, g.ksub), g);
     }
   }
   {
@@ -349,9 +429,10 @@ void moe_gemms(dg_handle* H, int l, int T) {
       g.ld_out = c.d_model;
       g.row_map = H->perm;
       g.err = H->d_err;
-      tc_policy(g);
-  tc_policy(g);
-      launch_gemm_tc(H->lmaps[l].down, H->m_dummy, H->m_dummy, H->m_hb, g, H->num_sms, H->stream);
+      g.ksub = ksub_for(2, tile);
+      g.ctas_per_sm = ctas_for(g.ntile);
+      const CUtensorMap& a = pick(H->lmaps[l].down, g.ksub);
+      run_tc(H, a, a, a, bmap(H, H->hb, c.d_ff, rows, tile, g.ksub), g);
     }
   }
 }
@@ -407,7 +488,7 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
     launch_embed<T>(tokens, prev, (const T*)H->embed, H->h, (T*)H->eprev, Tn, c.d_model, c.vocab, H->d_err,
                     H->stream);
   }
-  if (prev) dense_gemm(H, PC_DENSE, H->eprev, &H->m_eprev, H->w_sc, &H->m_wsc, Tn, c.d_model, c.d_model,
+  if (prev) dense_gemm(H, PC_DENSE, H->eprev, H->w_sc, &H->m_wsc, Tn, c.d_model, c.d_model,
                        EPI_ADD_F32, H->h, c.d_model);
   {
     ProfScope ps(H, PC_NORM);
@@ -425,13 +506,13 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
     }
     (void)ldqkv;
     attention(H, l, bi, nq, causal);
-    dense_gemm(H, PC_DENSE, H->attn, &H->m_attn, L.wo, &H->lmaps[l].wo, Tn, c.d_model, c.n_heads * c.head_dim,
+    dense_gemm(H, PC_DENSE, H->attn, L.wo, H->bf16 ? &H->lmaps[l].wo : nullptr, Tn, c.d_model, c.n_heads * c.head_dim,
                EPI_ADD_F32, H->h, c.d_model);
     {
       ProfScope ps(H, PC_NORM);
       launch_rmsnorm<T>(H->h, L.ffn_norm, xn, Tn, c.d_model, eps, H->stream);
     }
-    dense_gemm(H, PC_ROUTER, H->xn, &H->m_xn, L.router_w, &H->lmaps[l].router, Tn, c.n_experts, c.d_model,
+    dense_gemm(H, PC_ROUTER, H->xn, L.router_w, H->bf16 ? &H->lmaps[l].router : nullptr, Tn, c.n_experts, c.d_model,
                EPI_STORE_F32, H->glog, c.n_experts);
     {
       ProfScope ps(H, PC_ROUTER, 2);
@@ -458,7 +539,7 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
       launch_rmsnorm<T>(H->h, H->final_norm, xn, Tn, c.d_model, eps, H->stream);
     }
   }
-  if (head) dense_gemm(H, PC_LMHEAD, H->xn, &H->m_xn, H->embed, &H->m_embed, Tn, c.vocab, c.d_model, EPI_STORE_F32,
+  if (head) dense_gemm(H, PC_LMHEAD, H->xn, H->embed, &H->m_embed, Tn, c.vocab, c.d_model, EPI_STORE_F32,
                        logits, c.vocab);
 }
 
@@ -491,6 +572,10 @@ int upload_req(dg_handle* H, const BatchInfo& bi) {
 }
 
 int check_launch(dg_handle* H, const char* what) {
+  if (H->bad_launch) {
+    H->bad_launch = false;
+    return fail(H, DG_ECUDA, "%s: a tensor map or GEMM tiling was rejected (nothing was launched for it)", what);
+  }
   return cuda_check(H, cudaGetLastError(), what);
 }
 
@@ -698,32 +783,36 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
       for (int l = 0; l < c.n_layers; ++l) {
         const dg_layer_weights& L = H->lw[l];
         LayerMaps& M = H->lmaps[l];
-        tm &= tmap_2d(&M.wq, L.wq, d, qw, d, 128);
-        tm &= tmap_2d(&M.wk, L.wk, d, kw, d, 128);
-        tm &= tmap_2d(&M.wv, L.wv, d, kw, d, 128);
-        tm &= tmap_2d(&M.wo, L.wo, qw, d, qw, 128);
-        tm &= tmap_2d(&M.router, L.router_w, d, E, d, 128);
-        tm &= tmap_3d(&M.gate, L.w_gate, d, F, E, 128);
-        tm &= tmap_3d(&M.up, L.w_up, d, F, E, 128);
-        tm &= tmap_3d(&M.down, L.w_down, F, d, E, 128);
+        auto dense = [&](WMap& w, const void* p, uint64_t cols, uint64_t rows) {
+          tm &= tmap_chunks(&w.k2, p, cols, rows, cols, 128, 2);
+          tm &= tmap_chunks(&w.k4, p, cols, rows, cols, 128, 4);
+        };
+        auto experts = [&](WMap& w, const void* p, uint64_t cols, uint64_t rows) {
+          tm &= tmap_chunks4(&w.k2, p, cols, rows, E, 128, 2);
+          tm &= tmap_chunks4(&w.k4, p, cols, rows, E, 128, 4);
+        };
+        dense(M.wq, L.wq, d, qw);
+        dense(M.wk, L.wk, d, kw);
+        dense(M.wv, L.wv, d, kw);
+        dense(M.wo, L.wo, qw, d);
+        dense(M.router, L.router_w, d, E);
+        experts(M.gate, L.w_gate, d, F);
+        experts(M.up, L.w_up, d, F);
+        experts(M.down, L.w_down, F, d);
       }
-      tm &= tmap_2d(&H->m_embed, H->embed, d, c.vocab, d, 128);
-      tm &= tmap_2d(&H->m_wsc, H->w_sc, d, d, d, 128);
-      H->m_dummy = H->m_wsc;
-      tm &= tmap_2d(&H->m_xn, H->xn, d, T, d, 32);
-      tm &= tmap_2d(&H->m_eprev, H->eprev, d, T, d, 32);
-      tm &= tmap_2d(&H->m_attn, H->attn, qw, T, qw, 32);
-      tm &= tmap_2d(&H->m_xp, H->xp, d, (uint64_t)T * c.top_k, d, 32);
-      tm &= tmap_2d(&H->m_hb, H->hb, F, (uint64_t)T * c.top_k, F, 32);
+      tm &= tmap_chunks(&H->m_embed.k2, H->embed, d, c.vocab, d, 128, 2);
+      tm &= tmap_chunks(&H->m_embed.k4, H->embed, d, c.vocab, d, 128, 4);
+      tm &= tmap_chunks(&H->m_wsc.k2, H->w_sc, d, d, d, 128, 2);
+      tm &= tmap_chunks(&H->m_wsc.k4, H->w_sc, d, d, d, 128, 4);
       if (c.head_dim == 256) {
         H->attn_tc = true;
         const uint64_t hd = (uint64_t)c.head_dim;
-        tm &= tmap_2d(&H->m_q, H->q, hd, (uint64_t)T * c.n_heads, hd, 128);
+        tm &= tmap_chunks(&H->m_q, H->q, hd, (uint64_t)T * c.n_heads, hd, 128, 4);
         H->m_kc.resize(c.n_layers);
         H->m_vt.resize(c.n_layers);
         const uint64_t kv_rows = (uint64_t)c.max_batch * c.n_kv_heads;
         for (int l = 0; l < c.n_layers; ++l) {
-          tm &= tmap_2d(&H->m_kc[l], kc_layer(H, l), hd, kv_rows * c.max_ctx, hd, 64);
+          tm &= tmap_chunks(&H->m_kc[l], kc_layer(H, l), hd, kv_rows * c.max_ctx, hd, 64, 4);
           tm &= tmap_2d(&H->m_vt[l], vt_layer(H, l), (uint64_t)c.max_ctx, kv_rows * hd, (uint64_t)c.max_ctx, 256);
         }
       }
@@ -968,9 +1057,6 @@ int dg_selftest_philox(dg_handle* H, const uint32_t* ctr, const uint32_t* key, u
 int dg_selftest_gemm(dg_handle* H, const void* x, const void* w, int T, int M, int K, float* out) {
   if (!H || !x || !w || !out || T < 1 || M < 1 || K < 64 || K % 64) return H ? fail(H, DG_EINVAL, "bad gemm args") : DG_EINVAL;
   if (!aligned16(x) || !aligned16(w)) return fail(H, DG_EINVAL, "unaligned operands");
-  CUtensorMap mx, mw;
-  if (!tmap_2d(&mx, x, K, T, K, 32) || !tmap_2d(&mw, w, K, M, K, 128))
-    return fail(H, DG_ECUDA, "tensor map encode failed");
   TcGemm g{};
   g.mode = 0;
   g.M = M;
@@ -982,8 +1068,14 @@ int dg_selftest_gemm(dg_handle* H, const void* x, const void* w, int T, int M, i
   g.out = out;
   g.ld_out = M;
   g.err = H->d_err;
-  tc_policy(g);
-  launch_gemm_tc(mw, mw, mw, mx, g, H->num_sms, H->stream);
+  g.ksub = ksub_for(0, g.ntile);
+  g.ctas_per_sm = ctas_for(g.ntile);
+  CUtensorMap mx, mw;
+  if (!tmap_chunks(&mx, x, K, T, K, (uint32_t)g.ntile, (uint32_t)g.ksub) ||
+      !tmap_chunks(&mw, w, K, M, K, 128, (uint32_t)g.ksub))
+    return fail(H, DG_ECUDA, "tensor map encode failed");
+  if (launch_gemm_tc(mw, mw, mw, mx, g, H->num_sms, H->stream) != 0)
+    return fail(H, DG_EINVAL, "GEMM tiling rejected");
   H->launches += 1;
   return check_launch(H, "selftest gemm");
 }

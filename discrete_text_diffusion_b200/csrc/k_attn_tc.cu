@@ -26,7 +26,9 @@
 
 namespace dg {
 
-constexpr int kAttnThreads = 320;   // producer, MMA issuer, 8 softmax warps
+constexpr int kAttnThreads = 352;   // K producer, MMA issuer, 8 softmax warps, V producer
+constexpr int kKStages = 3;         // K tiles in flight (freed when their S MMA completes)
+constexpr int kVStages = 2;         // V tiles in flight (freed when their PV MMA completes)
 constexpr int kQTile = 128;
 constexpr int kKTile = 64;
 constexpr int kHd = 256;
@@ -34,7 +36,7 @@ constexpr int kQBytes = kQTile * kHd * 2;   // 64 KB
 constexpr int kKBytes = kKTile * kHd * 2;   // 32 KB
 constexpr int kVBytes = kHd * kKTile * 2;   // 32 KB
 constexpr int kRedBytes = 256 * 4;           // per-row exchange between the two halves
-constexpr int kAttnSmem = 1008 + kQBytes + 2 * kKBytes + 2 * kVBytes + kRedBytes + 128;
+constexpr int kAttnSmem = 1008 + kQBytes + kKStages * kKBytes + kVStages * kVBytes + kRedBytes + 160;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct AttnTcParams {
@@ -83,24 +85,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = base;
-  uint8_t* sK = sQ + kQBytes;            // [2][kKBytes]
-  uint8_t* sV = sK + 2 * kKBytes;        // [2][kVBytes]
-  float* red = reinterpret_cast<float*>(sV + 2 * kVBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * kVBytes + kRedBytes);
+  uint8_t* sK = sQ + kQBytes;                  // [kKStages][kKBytes]
+  uint8_t* sV = sK + kKStages * kKBytes;       // [kVStages][kVBytes]
+  float* red = reinterpret_cast<float*>(sV + kVStages * kVBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kVStages * kVBytes + kRedBytes);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;     // [2]
-  uint64_t* kv_empty = bars + 3;    // [2]
-  uint64_t* s_full = bars + 5;      // [2]
-  uint64_t* p_full = bars + 9;      // [2]
-  uint64_t* pv_done = bars + 11;    // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* k_full = bars + 1;      // [3]
+  uint64_t* k_empty = bars + 4;     // [3]
+  uint64_t* v_full = bars + 7;      // [2]
+  uint64_t* v_empty = bars + 9;     // [2]
+  uint64_t* s_full = bars + 11;     // [2]
+  uint64_t* p_full = bars + 13;     // [2]
+  uint64_t* pv_done = bars + 15;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   int* err = P.t.err;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 256);
       mbar_init(&pv_done[i], 1);
@@ -119,24 +127,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tO = tmem + 256;    // output accumulator: columns [256, 512)
 
   if (warp == 0 && lane == 0) {
-    // ----------------------------------------------------------- producer
+    // ----------------------------------------------------------- K producer
+    // One TMA instruction each for Q (4 chunks of 64 dims) and every K tile.
+    // K and V have separate rings: a K tile is free as soon as its S MMA is
+    // done, so the next K loads start a tile earlier than a shared ring allows.
     prefetch_tmap(&tq);
     prefetch_tmap(&tk);
-    prefetch_tmap(&tv);
     const int qrow = (int)row_id + q0;
     mbar_expect_tx(q_full, kQBytes);
-    for (int c = 0; c < kHd / 64; ++c) tma_load_2d(sQ + c * (kQTile * 128), &tq, q_full, c * 64, qrow);
+    tma_load_3d(sQ, &tq, q_full, 0, qrow, 0);
     const int krow = (slot * a.hkv + g) * a.max_ctx;
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % kKStages;
+      const uint32_t ph = (uint32_t)(j / kKStages) & 1u;
+      if (!mbar_wait(&k_empty[s], ph ^ 1u, err, kErrTimeoutAttn)) break;
+      mbar_expect_tx(&k_full[s], kKBytes);
+      tma_load_3d(sK + s * kKBytes, &tk, &k_full[s], 0, krow + (t_begin + j) * kKTile, 0);
+    }
+  } else if (warp == 10 && lane == 0) {
+    // ----------------------------------------------------------- V producer
+    prefetch_tmap(&tv);
     const int vrow = (slot * a.hkv + g) * kHd;
     for (int j = 0; j < ntiles; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-      if (!mbar_wait(&kv_empty[s], ph ^ 1u, err, kErrTimeoutAttn)) break;
-      const int key0 = (t_begin + j) * kKTile;
-      mbar_expect_tx(&kv_full[s], kKBytes + kVBytes);
-      uint8_t* k_dst = sK + s * kKBytes;
-      for (int c = 0; c < kHd / 64; ++c) tma_load_2d(k_dst + c * (kKTile * 128), &tk, &kv_full[s], c * 64, krow + key0);
-      tma_load_2d(sV + s * kVBytes, &tv, &kv_full[s], key0, vrow);
+      const int s = j % kVStages;
+      const uint32_t ph = (uint32_t)(j / kVStages) & 1u;
+      if (!mbar_wait(&v_empty[s], ph ^ 1u, err, kErrTimeoutAttn)) break;
+      mbar_expect_tx(&v_full[s], kVBytes);
+      tma_load_2d(sV + s * kVBytes, &tv, &v_full[s], (t_begin + j) * kKTile, vrow);
     }
   } else if (warp == 1 && lane == 0) {
     // ----------------------------------------------------------- MMA issuer
@@ -146,12 +163,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     bool ok = mbar_wait(q_full, 0, err, kErrTimeoutAttn);
     auto issue_s = [&](int j) -> bool {
       const int s = j & 1;
-      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+      const int ks = j % kKStages;
       // S_j reuses the TMEM columns of P_{j-2}; PV_{j-2} was issued earlier,
       // and tcgen05.mma of one thread run in issue order.
-      if (!mbar_wait(&kv_full[s], ph, err, kErrTimeoutAttn)) return false;
+      if (!mbar_wait(&k_full[ks], (uint32_t)(j / kKStages) & 1u, err, kErrTimeoutAttn)) return false;
       tc_fence_after();
-      const uint32_t k_base = smem_u32(sK + s * kKBytes);
+      const uint32_t k_base = smem_u32(sK + ks * kKBytes);
 #pragma unroll
       for (int c = 0; c < kHd / 64; ++c)
 #pragma unroll
@@ -159,6 +176,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           umma_bf16(tS + (uint32_t)(s * kKTile), sdesc_k_sw128(q_base + c * (kQTile * 128) + 32u * k),
                     sdesc_k_sw128(k_base + c * (kKTile * 128) + 32u * k), idesc_s, (c | k) ? 1u : 0u);
       umma_commit(&s_full[s]);
+      umma_commit(&k_empty[ks]);
       return true;
     };
     if (ok) ok = issue_s(0);
@@ -166,6 +184,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (j + 1 < ntiles && !issue_s(j + 1)) break;
       const int s = j & 1;
       if (!mbar_wait(&p_full[s], (uint32_t)(j >> 1) & 1u, err, kErrTimeoutAttn)) break;
+      if (!mbar_wait(&v_full[s], (uint32_t)(j >> 1) & 1u, err, kErrTimeoutAttn)) break;
       tc_fence_after();
       // O += P_j V_j with P_j (bf16, 32 columns) read from TMEM where S_j was
       const uint32_t v_base = smem_u32(sV + s * kVBytes);
@@ -174,9 +193,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         umma_bf16_ts(tO, tS + (uint32_t)(s * kKTile + 8 * k), sdesc_k_sw128(v_base + 32u * k), idesc_o,
                      (j > 0 || k > 0) ? 1u : 0u);
       umma_commit(&pv_done[s]);
-      umma_commit(&kv_empty[s]);
+      umma_commit(&v_empty[s]);
     }
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 10) {
     // ----------------------------------------------------------- softmax
     // 8 warps: thread (quarter, lane) of half hf owns query row r and keys
     // [32 hf, 32 hf + 32) of each 64-key tile, and O columns [128 hf, +128).

@@ -48,9 +48,6 @@ constexpr int kMaxSmem = 232448;        // 227 KB opt-in limit per CTA
 #define DG_GEMM_CTAS_PER_SM 1           // default co-resident CTAs per SM
 #endif
 constexpr int kSmemPerSm = 233472;      // 228 KB of shared memory per SM
-#ifndef DG_GEMM_WARP_ISSUE
-#define DG_GEMM_WARP_ISSUE 1            // spread a stage's TMA boxes over the producer warp
-#endif
 
 struct TcLayout {
   int n_a;          // weight operands per stage (1 or 2)
@@ -69,6 +66,7 @@ static TcLayout tc_layout(const TcGemm& p) {
   L.n_a = (p.mode == 1) ? 2 : 1;
   L.acc_cols = L.n_a * p.ntile;
   L.per_sm = std::max(1, std::min(3, p.ctas_per_sm > 0 ? p.ctas_per_sm : DG_GEMM_CTAS_PER_SM));
+  // the tensor maps are built for this chunk count: it is never changed here
   L.ksub = std::max(1, std::min(4, p.ksub > 0 ? p.ksub : DG_GEMM_KSUB));
   const int overhead = 1024 /*align*/ + 1024 /*barriers*/;
   for (;;) {
@@ -81,10 +79,8 @@ static TcLayout tc_layout(const TcGemm& p) {
     L.stage_bytes = L.ksub * (L.n_a * kABytes + p.ntile * kBK * 2);
     L.stages = std::min(DG_GEMM_MAX_STAGES, (budget - overhead) / L.stage_bytes);
     if (L.per_sm * L.tmem_cols <= 512 && L.stages >= 2) break;
-    if (L.ksub > 1) { --L.ksub; continue; }
     if (L.per_sm > 1) { --L.per_sm; continue; }
-    L.stages = std::max(L.stages, 1);
-    break;
+    break;   // stages < 2: rejected by the launcher
   }
   L.smem_bytes = overhead + L.stages * L.stage_bytes;
   return L;
@@ -164,56 +160,41 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   const int b_sub = g.ntile * kBK * 2;            // bytes of one token sub-tile
   // stage layout: [ksub x A0][ksub x A1 (mode 1)][ksub x B], each sub 1024-aligned
 
-  if (warp == 0) {
+  if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    // Lane 0 waits for the slot and posts the byte count; then the stage's
-    // boxes (weights and token rows of every K block) are spread over the
-    // lanes of the warp, so they are issued to the TMA unit side by side.
+    // One TMA instruction per operand and stage: the weight maps are
+    // (64, rows, K/64[, experts]) views with a box of ksub 64-column chunks,
+    // the token map a (64, rows, K/64) view with a box of ntile rows x ksub
+    // chunks.  A stage always receives whole boxes (chunks past K, rows past
+    // the matrix are zero-filled), so the byte count is fixed.
+    const uint32_t tx = (uint32_t)(ksub * (n_a * kABytes + b_sub));
     uint32_t kiter = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
       int m0, e, row0, rows;
       tc_item(P, item, m0, e, row0, rows);
-      const int nb = (rows + kBoxN - 1) / kBoxN;
       const CUtensorMap* am = &ta0;
       int am0 = m0;
       if (g.mode == 0) {
         if (m0 >= g.seg2) { am = &ta2; am0 = m0 - g.seg2; }
         else if (m0 >= g.seg1) { am = &ta1; am0 = m0 - g.seg1; }
       }
-      const int per_u = n_a + nb;  // boxes per K block
+      bool ok = true;
       for (int j = 0; j < nst; ++j, ++kiter) {
         const int s = kiter % P.stages;
         const uint32_t ph = (kiter / P.stages) & 1u;
-        int okw = 1;
-        if (lane == 0) okw = mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma) ? 1 : 0;
-        okw = __shfl_sync(0xffffffffu, okw, 0);
-        if (!okw) { ok = false; break; }
+        if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
         const int kb0 = j * ksub;
-        const int nsub = min(ksub, nk - kb0);
         uint8_t* st = stage0 + (size_t)s * P.stage_bytes;
-        if (lane == 0) mbar_expect_tx(&full[s], (uint32_t)(nsub * (n_a * kABytes + nb * kBoxN * kBK * 2)));
-        __syncwarp();
-#if DG_GEMM_WARP_ISSUE
-        for (int task = lane; task < nsub * per_u; task += 32) {
-#else
-        for (int task = 0; lane == 0 && task < nsub * per_u; ++task) {
-#endif
-          const int u = task / per_u, r = task - u * per_u;
-          const int kc = (kb0 + u) * kBK;
-          if (r == 0) {
-            if (g.mode == 0) tma_load_2d(st + u * kABytes, am, &full[s], kc, am0);
-            else tma_load_3d(st + u * kABytes, &ta0, &full[s], kc, m0, e);
-          } else if (r < n_a) {
-            tma_load_3d(st + (ksub + u) * kABytes, &ta1, &full[s], kc, m0, e);
-          } else {
-            const int i = r - n_a;
-            tma_load_2d(st + n_a * ksub * kABytes + u * b_sub + i * kBoxN * kBK * 2, &tb, &full[s], kc,
-                        row0 + i * kBoxN);
-          }
+        mbar_expect_tx(&full[s], tx);
+        if (g.mode == 0) {
+          tma_load_3d(st, am, &full[s], 0, am0, kb0);
+        } else {
+          tma_load_4d(st, &ta0, &full[s], 0, m0, kb0, e);
+          if (g.mode == 1) tma_load_4d(st + ksub * kABytes, &ta1, &full[s], 0, m0, kb0, e);
         }
-        __syncwarp();
+        tma_load_3d(st + n_a * ksub * kABytes, &tb, &full[s], 0, row0, kb0);
       }
+      if (!ok) break;
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -324,9 +305,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   }
 }
 
-void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
-                    const TcGemm& g, int num_sms, cudaStream_t s) {
+int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
+                   const TcGemm& g, int num_sms, cudaStream_t s) {
   const TcLayout L = tc_layout(g);
+  if (L.stages < 2) return -1;   // the tile does not fit a two-stage pipeline
   TcKParams P;
   P.g = g;
   P.stages = L.stages;
@@ -338,7 +320,7 @@ void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensor
   P.n_mtiles = (g.M + kBM - 1) / kBM;
   P.n_ttiles = (g.mode == 0) ? (g.T + g.ntile - 1) / g.ntile : 0;
   const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles : g.n_work_max * P.n_mtiles;
-  if (total <= 0) return;
+  if (total <= 0) return 0;
   static int attr_bytes = 0;
   if (attr_bytes < L.smem_bytes) {
     cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
@@ -346,6 +328,7 @@ void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensor
   }
   const int grid = std::min(total, num_sms * L.per_sm);
   gemm_tc_kernel<<<grid, kTcThreads, L.smem_bytes, s>>>(a0, a1, a2, b, P);
+  return 0;
 }
 
 }  // namespace dg

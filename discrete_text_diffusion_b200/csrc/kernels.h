@@ -111,8 +111,9 @@ struct TcGemm {
   int ksub;          // 64-wide K blocks per pipeline stage (0 = build default)
   int ctas_per_sm;   // co-resident CTAs the grid is sized for (0 = build default)
 };
-void launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
-                    const TcGemm& p, int num_sms, cudaStream_t s);
+// Returns 0, or -1 when the tile does not fit a two-stage pipeline (nothing launched).
+int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
+                   const TcGemm& p, int num_sms, cudaStream_t s);
 int gemm_tc_smem_bytes(const TcGemm& p, int* stages);
 
 // ---- attention
