@@ -289,6 +289,7 @@ int grouped_tile(const dg_handle* H, int T) {
 #define DG_NARROW_CTAS 2      // CTAs per SM when the token tile is <= 64 rows
 #endif
 int ksub_for(int mode, int ntile) { return (mode == 1 || ntile > 64) ? 2 : DG_NARROW_KSUB; }
+constexpr int kMaxKSplit = 16;   // K slices of a split-K projection (router logits)
 int ctas_for(int ntile) { return ntile <= 64 ? DG_NARROW_CTAS : 1; }
 
 const CUtensorMap& pick(const WMap& w, int ksub) { return ksub == 4 ? w.k4 : w.k2; }
@@ -318,13 +319,15 @@ void run_tc(dg_handle* H, const CUtensorMap& a0, const CUtensorMap& a1, const CU
 }
 
 // ------------------------------------------------------------ GEMM helpers
-// out = x[T, K] * W^T (W [n_out, K]) for the dense projections.
-void dense_gemm(dg_handle* H, int cls, const void* x, const void* w, const WMap* mw, int T, int n_out, int K,
-                Epi epi, void* out, int ld_out) {
+// out = x[T, K] * W^T (W [n_out, K]) for the dense projections.  With
+// max_split > 1 (EPI_STORE_F32 only) K may be split into slices that write
+// partial sums at out + s * T * ld_out; returns the number of slices used.
+int dense_gemm(dg_handle* H, int cls, const void* x, const void* w, const WMap* mw, int T, int n_out, int K,
+               Epi epi, void* out, int ld_out, int max_split = 1) {
   ProfScope ps(H, cls);
   if (!H->bf16) {
     launch_gemm_simt<float>((const float*)x, (const float*)w, T, n_out, K, epi, out, ld_out, nullptr, H->stream);
-    return;
+    return 1;
   }
   TcGemm g{};
   g.mode = 0;
@@ -339,8 +342,17 @@ void dense_gemm(dg_handle* H, int cls, const void* x, const void* w, const WMap*
   g.err = H->d_err;
   g.ksub = ksub_for(0, g.ntile);
   g.ctas_per_sm = ctas_for(g.ntile);
+  // split K (two stages per slice at least) while the grid is below two waves
+  const int nst = (K / 64 + g.ksub - 1) / g.ksub;
+  const int items = ((n_out + 127) / 128) * ((T + g.ntile - 1) / g.ntile);
+  int split = 1;
+  if (epi == EPI_STORE_F32 && max_split > 1)
+    while (split * 2 <= max_split && split * 2 * 2 <= nst && items * split < 2 * H->num_sms) split *= 2;
+  g.ksplit = split;
+  g.split_stride = (size_t)T * ld_out;
   const CUtensorMap& a = pick(*mw, g.ksub);
   run_tc(H, a, a, a, bmap(H, x, K, H->T_max, g.ntile, g.ksub), g);
+  return split;
 }
 
 void qkv_gemm(dg_handle* H, int l, int T) {
@@ -512,11 +524,12 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
       ProfScope ps(H, PC_NORM);
       launch_rmsnorm<T>(H->h, L.ffn_norm, xn, Tn, c.d_model, eps, H->stream);
     }
-    dense_gemm(H, PC_ROUTER, H->xn, L.router_w, H->bf16 ? &H->lmaps[l].router : nullptr, Tn, c.n_experts, c.d_model,
-               EPI_STORE_F32, H->glog, c.n_experts);
+    // the router projection has one 128-row weight tile: split K for parallelism
+    const int rsplit = dense_gemm(H, PC_ROUTER, H->xn, L.router_w, H->bf16 ? &H->lmaps[l].router : nullptr, Tn,
+                                  c.n_experts, c.d_model, EPI_STORE_F32, H->glog, c.n_experts, kMaxKSplit);
     {
       ProfScope ps(H, PC_ROUTER, 2);
-      launch_router_topk(H->glog, L.router_b, H->ids, H->wts, Tn, c.n_experts, c.top_k, H->stream);
+      launch_router_topk(H->glog, rsplit, L.router_b, H->ids, H->wts, Tn, c.n_experts, c.top_k, H->stream);
       launch_router_permute(H->ids, Tn * c.top_k, c.n_experts, grouped_tile(H, Tn), H->cnt, H->off, H->perm,
                             H->work, H->n_work, H->touched + l, H->stream);
     }
@@ -678,6 +691,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
       return fail(nullptr, DG_EINVAL, "bf16 needs d_model, d_ff, head_dim multiples of 64");
     if (!w || !w->embed || !w->w_sc || !w->final_norm || !w->layers)
       return fail(nullptr, DG_EINVAL, "null weight pointer");
+    if (!aligned16(w->final_norm)) return fail(nullptr, DG_EINVAL, "unaligned final_norm");
     for (int l = 0; l < c.n_layers; ++l) {
       const dg_layer_weights& L = w->layers[l];
       const void* ps[] = {L.attn_norm, L.wq, L.wk, L.wv, L.wo, L.ffn_norm, L.router_w, L.w_gate, L.w_up, L.w_down};
@@ -719,7 +733,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
     H->qkv = dalloc<float>((size_t)T * ldqkv, &ok);
     H->q = dalloc<char>((size_t)T * qw * H->esz, &ok);
     H->attn = dalloc<char>((size_t)T * qw * H->esz, &ok);
-    H->glog = dalloc<float>((size_t)T * c.n_experts, &ok);
+    H->glog = dalloc<float>((size_t)T * c.n_experts * kMaxKSplit, &ok);
     H->ids = dalloc<int32_t>((size_t)T * c.top_k, &ok);
     H->wts = dalloc<float>((size_t)T * c.top_k, &ok);
     H->cnt = dalloc<int32_t>(c.n_experts, &ok);
@@ -900,6 +914,7 @@ int dg_sample(dg_handle* H, const float* logits, int batch, const int* req, int 
   if (rc) return rc;
   if ((rc = check_sampler_params(H, sp))) return rc;
   if (!logits || !canvas) return fail(H, DG_EINVAL, "null logits or canvas");
+  if (!aligned16(logits)) return fail(H, DG_EINVAL, "logits must be 16-byte aligned");
   if ((rc = upload_req(H, bi))) return rc;
   const SamplerArgs a = sampler_args(*sp, step);
   run_sampler(H, logits, bi, a, canvas, (o && o->x_hat) ? o->x_hat : H->xh[0], (o && o->pmax) ? o->pmax : H->pmax,
@@ -917,6 +932,7 @@ int dg_denoise_step(dg_handle* H, const dg_step_args* a, const dg_step_out* o) {
   if (rc) return rc;
   if ((rc = check_sampler_params(H, &a->sp))) return rc;
   if (!a->canvas) return fail(H, DG_EINVAL, "null canvas");
+  if (a->logits_out && !aligned16(a->logits_out)) return fail(H, DG_EINVAL, "logits_out must be 16-byte aligned");
   if (a->step < 1) return fail(H, DG_EINVAL, "step must be >= 1");
   for (int b = 0; b < bi.B; ++b)
     if (bi.len[b] + c.canvas > c.max_ctx) return fail(H, DG_ECAPACITY, "cache + canvas exceeds max_ctx");

@@ -65,17 +65,48 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 }
 
 // ---------------------------------------------------------------- RMSNorm
+// Rows are processed as float4 when d % 4 == 0 (16-byte loads), else as floats.
+template <typename T>
+__device__ __forceinline__ void store4(T* o, int j4, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float* o, int j4, float4 v) {
+  reinterpret_cast<float4*>(o)[j4] = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* o, int j4, float4 v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<const uint32_t*>(&a);
+  u.y = *reinterpret_cast<const uint32_t*>(&b);
+  reinterpret_cast<uint2*>(o)[j4] = u;
+}
+
 template <typename T>
 __global__ void rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ w, T* __restrict__ xn,
                                int d, float eps) {
   __shared__ float red[32];
   const int t = blockIdx.x;
   const float* x = h + (size_t)t * d;
+  T* o = xn + (size_t)t * d;
   float ss = 0.f;
+  if ((d & 3) == 0) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    for (int j = threadIdx.x; j < d / 4; j += blockDim.x) {
+      const float4 v = x4[j];
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = block_sum(ss, red);
+    const float r = rsqrtf(ss / (float)d + eps);
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+    for (int j = threadIdx.x; j < d / 4; j += blockDim.x) {
+      const float4 v = x4[j], g = w4[j];
+      store4<T>(o, j, make_float4(v.x * r * g.x, v.y * r * g.y, v.z * r * g.z, v.w * r * g.w));
+    }
+    return;
+  }
   for (int j = threadIdx.x; j < d; j += blockDim.x) ss += x[j] * x[j];
   ss = block_sum(ss, red);
   const float r = rsqrtf(ss / (float)d + eps);
-  T* o = xn + (size_t)t * d;
   for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f32<T>(x[j] * r * w[j]);
 }
 
@@ -88,7 +119,8 @@ void launch_rmsnorm(const float* h, const float* w, T* xn, int n_tok, int d, flo
 // ---------------------------------------------------------------- combine
 // h[t] += sum over the k slots, in slot order, of w[t,s] * y[t*k+s]; then the
 // optional RMSNorm of the new residual into xn.  Each element is owned by one
-// thread: no atomics, bitwise reproducible.
+// thread and summed in slot order: no atomics, bitwise reproducible.  The
+// float4 path issues the k slot loads of a column group together.
 template <typename T>
 __global__ void combine_kernel(float* __restrict__ h, const float* __restrict__ y, const float* __restrict__ wts,
                                int k, const float* __restrict__ norm_w, T* __restrict__ xn, int d, float eps) {
@@ -100,6 +132,40 @@ __global__ void combine_kernel(float* __restrict__ h, const float* __restrict__ 
   float* hr = h + (size_t)t * d;
   const float* yr = y + (size_t)t * k * d;
   float ss = 0.f;
+  if ((d & 3) == 0) {
+    const int d4 = d / 4;
+    float4* h4 = reinterpret_cast<float4*>(hr);
+    const float4* y4 = reinterpret_cast<const float4*>(yr);
+    for (int j = threadIdx.x; j < d4; j += blockDim.x) {
+      float4 yv[16];
+#pragma unroll
+      for (int s = 0; s < 16; ++s)
+        if (s < k) yv[s] = y4[(size_t)s * d4 + j];
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s = 0; s < 16; ++s)
+        if (s < k) {
+          acc.x += ws[s] * yv[s].x;
+          acc.y += ws[s] * yv[s].y;
+          acc.z += ws[s] * yv[s].z;
+          acc.w += ws[s] * yv[s].w;
+        }
+      float4 v = h4[j];
+      v.x += acc.x; v.y += acc.y; v.z += acc.z; v.w += acc.w;
+      h4[j] = v;
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    if (norm_w == nullptr) return;
+    ss = block_sum(ss, red);
+    const float r = rsqrtf(ss / (float)d + eps);
+    const float4* w4 = reinterpret_cast<const float4*>(norm_w);
+    T* o = xn + (size_t)t * d;
+    for (int j = threadIdx.x; j < d4; j += blockDim.x) {
+      const float4 v = h4[j], g = w4[j];
+      store4<T>(o, j, make_float4(v.x * r * g.x, v.y * r * g.y, v.z * r * g.z, v.w * r * g.w));
+    }
+    return;
+  }
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
     float acc = 0.f;
     for (int s = 0; s < k; ++s) acc += ws[s] * yr[(size_t)s * d + j];

@@ -97,14 +97,25 @@ struct TcKParams {
   int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, n_ttiles, ksub;
 };
 
-__device__ __forceinline__ void tc_item(const TcKParams& P, int item, int& m0, int& e, int& row0, int& rows) {
+// Work item -> weight tile, token rows and (dense split-K) the range of K
+// stages [j0, j1) with its split index ks.
+__device__ __forceinline__ void tc_item(const TcKParams& P, int item, int nst, int& m0, int& e, int& row0,
+                                        int& rows, int& j0, int& j1, int& ks) {
   const TcGemm& g = P.g;
+  j0 = 0;
+  j1 = nst;
+  ks = 0;
   if (g.mode == 0) {
-    const int tt = item % P.n_ttiles, mt = item / P.n_ttiles;
+    const int nsplit = g.ksplit > 1 ? g.ksplit : 1;
+    ks = item % nsplit;
+    const int rest = item / nsplit;
+    const int tt = rest % P.n_ttiles, mt = rest / P.n_ttiles;
     m0 = mt * kBM;
     e = 0;
     row0 = tt * g.ntile;
     rows = min(g.ntile, g.T - row0);
+    j0 = ks * nst / nsplit;
+    j1 = (ks + 1) * nst / nsplit;
   } else {
     const int mt = item % P.n_mtiles, w = item / P.n_mtiles;
     m0 = mt * kBM;
@@ -152,7 +163,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles : (*g.n_work) * P.n_mtiles;
+  const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles * (g.ksplit > 1 ? g.ksplit : 1)
+                                  : (*g.n_work) * P.n_mtiles;
   const int nk = g.K / kBK;                       // 64-wide K blocks
   const int ksub = P.ksub;                        // K blocks per pipeline stage
   const int nst = (nk + ksub - 1) / ksub;         // stages per output tile
@@ -170,8 +182,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const uint32_t tx = (uint32_t)(ksub * (n_a * kABytes + b_sub));
     uint32_t kiter = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
-      int m0, e, row0, rows;
-      tc_item(P, item, m0, e, row0, rows);
+      int m0, e, row0, rows, j0, j1, ks;
+      tc_item(P, item, nst, m0, e, row0, rows, j0, j1, ks);
       const CUtensorMap* am = &ta0;
       int am0 = m0;
       if (g.mode == 0) {
@@ -179,7 +191,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         else if (m0 >= g.seg1) { am = &ta1; am0 = m0 - g.seg1; }
       }
       bool ok = true;
-      for (int j = 0; j < nst; ++j, ++kiter) {
+      for (int j = j0; j < j1; ++j, ++kiter) {
         const int s = kiter % P.stages;
         const uint32_t ph = (kiter / P.stages) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
@@ -202,8 +214,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++it) {
-      int m0, e, row0, rows;
-      tc_item(P, item, m0, e, row0, rows);
+      int m0, e, row0, rows, j0, j1, ks;
+      tc_item(P, item, nst, m0, e, row0, rows, j0, j1, ks);
       const int n_mma = (rows + 15) & ~15;
       const uint32_t idesc = idesc_bf16(kBM, n_mma);
       const int ab = it % P.n_acc_buf;
@@ -211,7 +223,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       if (!mbar_wait(&acc_empty[ab], (use & 1u) ^ 1u, err, kErrTimeoutMma)) break;
       tc_fence_after();
       const uint32_t d0 = tmem_base + (uint32_t)(ab * P.acc_cols);
-      for (int j = 0; j < nst; ++j, ++kiter) {
+      for (int j = j0; j < j1; ++j, ++kiter) {
         const int s = kiter % P.stages;
         const uint32_t ph = (kiter / P.stages) & 1u;
         if (!mbar_wait(&full[s], ph, err, kErrTimeoutMma)) { ok = false; break; }
@@ -225,7 +237,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t bdesc = sdesc_k_sw128(sb + 32u * k);
-            const uint32_t acc = (j > 0 || u > 0 || k > 0) ? 1u : 0u;
+            const uint32_t acc = (j > j0 || u > 0 || k > 0) ? 1u : 0u;
             umma_bf16(d0, sdesc_k_sw128(sa + 32u * k), bdesc, idesc, acc);
             if (n_a == 2) umma_bf16(d0 + (uint32_t)g.ntile, sdesc_k_sw128(sa1 + 32u * k), bdesc, idesc, acc);
           }
@@ -241,8 +253,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int r = q * 32 + lane;
     int it = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
-      int m0, e, row0, rows;
-      tc_item(P, item, m0, e, row0, rows);
+      int m0, e, row0, rows, j0, j1, ks;
+      tc_item(P, item, nst, m0, e, row0, rows, j0, j1, ks);
       const int ab = it % P.n_acc_buf;
       const uint32_t use = (uint32_t)(it / P.n_acc_buf);
       if (!mbar_wait(&acc_full[ab], use & 1u, err, kErrTimeoutEpi)) break;
@@ -280,7 +292,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                   const int orow = g.row_map[row0 + c0 + j];
                   reinterpret_cast<float*>(g.out)[(size_t)orow * g.ld_out + m] = acc;
                 } else if (g.epi == EPI_STORE_F32) {
-                  reinterpret_cast<float*>(g.out)[(size_t)(row0 + c0 + j) * g.ld_out + m] = acc;
+                  reinterpret_cast<float*>(g.out)[(size_t)ks * g.split_stride + (size_t)(row0 + c0 + j) * g.ld_out + m] =
+                      acc;
                 } else if (g.epi == EPI_ADD_F32) {
                   reinterpret_cast<float*>(g.out)[(size_t)(row0 + c0 + j) * g.ld_out + m] += acc;
                 } else {
@@ -319,7 +332,8 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   P.tmem_cols = L.tmem_cols;
   P.n_mtiles = (g.M + kBM - 1) / kBM;
   P.n_ttiles = (g.mode == 0) ? (g.T + g.ntile - 1) / g.ntile : 0;
-  const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles : g.n_work_max * P.n_mtiles;
+  const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles * (g.ksplit > 1 ? g.ksplit : 1)
+                                  : g.n_work_max * P.n_mtiles;
   if (total <= 0) return 0;
   static int attr_bytes = 0;
   if (attr_bytes < L.smem_bytes) {

@@ -10,7 +10,7 @@ namespace dg {
 
 // One warp per token.  Lane l holds experts l, l+32, ...; k rounds of a warp
 // arg-max with (value desc, id asc) ordering pick the top-k.
-__global__ void router_topk_kernel(const float* __restrict__ glog, const float* __restrict__ bias,
+__global__ void router_topk_kernel(const float* __restrict__ glog, int nsplit, const float* __restrict__ bias,
                                    int32_t* __restrict__ ids, float* __restrict__ wts, int n_tok, int e, int k) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -20,7 +20,13 @@ __global__ void router_topk_kernel(const float* __restrict__ glog, const float* 
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
     const int ex = lane + 32 * j;
-    v[j] = (ex < e) ? glog[(size_t)warp * e + ex] + (bias ? bias[ex] : 0.f) : -INFINITY;
+    float g = -INFINITY;
+    if (ex < e) {
+      g = glog[(size_t)warp * e + ex];
+      for (int sp = 1; sp < nsplit; ++sp) g += glog[(size_t)sp * n_tok * e + (size_t)warp * e + ex];
+      g += bias ? bias[ex] : 0.f;
+    }
+    v[j] = g;
   }
   float sel_v[16];
   int sel_i[16];
@@ -57,12 +63,12 @@ __global__ void router_topk_kernel(const float* __restrict__ glog, const float* 
   }
 }
 
-void launch_router_topk(const float* glog, const float* bias, int32_t* ids, float* wts, int n_tok, int e, int k,
-                        cudaStream_t s) {
+void launch_router_topk(const float* glog, int nsplit, const float* bias, int32_t* ids, float* wts, int n_tok,
+                        int e, int k, cudaStream_t s) {
   if (n_tok <= 0) return;
   const int threads = 256;
   const int blocks = (n_tok * 32 + threads - 1) / threads;
-  router_topk_kernel<<<blocks, threads, 0, s>>>(glog, bias, ids, wts, n_tok, e, k);
+  router_topk_kernel<<<blocks, threads, 0, s>>>(glog, nsplit, bias, ids, wts, n_tok, e, k);
 }
 
 // Single-CTA counting sort.  Items i = t*k + s in order; inside an expert the

@@ -48,8 +48,10 @@ void launch_set_kv(const T* k, const T* v, T* kc, T* vt, int hkv, int n, int hd,
 
 // ---- router (k_router.cu)
 // Per token: g = glog + bias; top-k (ties -> lower id); softmax over the k.
-void launch_router_topk(const float* glog, const float* bias, int32_t* ids, float* wts, int n_tok, int e,
-                        int k, cudaStream_t s);
+// glog holds nsplit partial-sum slices of [n_tok, e] at a stride of n_tok*e
+// floats; they are added in slice order.
+void launch_router_topk(const float* glog, int nsplit, const float* bias, int32_t* ids, float* wts, int n_tok,
+                        int e, int k, cudaStream_t s);
 // Deterministic counting sort of the n_tok*k (token, slot) items by expert
 // (tokens ascending inside an expert).  perm[pos] = t*k+s; cnt[E]; off[E+1];
 // work list of (expert, first row, rows) tiles of at most `tile` rows;
@@ -110,6 +112,9 @@ struct TcGemm {
   int* err;
   int ksub;          // 64-wide K blocks per pipeline stage (0 = build default)
   int ctas_per_sm;   // co-resident CTAs the grid is sized for (0 = build default)
+  int ksplit;        // dense EPI_STORE_F32 only: K split into ksplit slices, slice s
+                     // writes its partial sums at out + s * split_stride (floats)
+  size_t split_stride;
 };
 // Returns 0, or -1 when the tile does not fit a two-stage pipeline (nothing launched).
 int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,

@@ -132,7 +132,7 @@ typedef struct dg_step_args {
   const int32_t* prev_pred;    /* [B, N] previous x_hat for self-conditioning, or NULL */
   int step;                    /* t >= 1, Philox counter word 1 */
   dg_sampler_params sp;
-  float* logits_out;           /* [B, N, V] fp32 to receive the logits, or NULL */
+  float* logits_out;           /* [B, N, V] fp32 to receive the logits (16-byte aligned), or NULL */
   float* hidden_out;           /* [B*N, d] fp32 residual stream before the final
                                   norm, or NULL */
 } dg_step_args;
@@ -207,6 +207,7 @@ int dg_denoise_step(dg_handle* h, const dg_step_args* a, const dg_step_out* o);
  * keep = top keep_k positions by pmax (ties to the lower index);
  * canvas[b,i] = keep ? x_hat : (w1 * V) >> 32 (uniform re-noise from word 1);
  * mean entropy and stop = mean < stop_threshold.
+ * logits must be 16-byte aligned (DG_EINVAL otherwise).
  */
 int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int step,
               const dg_sampler_params* sp, int32_t* canvas, const dg_step_out* o);

@@ -122,3 +122,19 @@ def test_sampler_large_batch_sampled_canvases(dg, B, k):
     del logits
     torch.cuda.empty_cache()
     h.close()
+
+
+@pytest.mark.gpu
+def test_sampler_rejects_unaligned_logits(dg):
+    """Pass 1 reads the logits with 16-byte loads: an unaligned pointer is refused on the host."""
+    n, V = 32, 1024
+    h = _handle(dg, 1, vocab=V, n=n)
+    buf = torch.zeros(n * V + 4, device="cuda")
+    canvas = torch.zeros((1, n), dtype=torch.int32, device="cuda")
+    sp = dg.sampler_params(temperature=1.0, keep_k=4)
+    with pytest.raises(dg.DgError) as ei:
+        dg.dg_sample(h, buf[1:], [0], 1, sp, canvas, dg.step_out())
+    assert ei.value.code == 1 and "aligned" in str(ei.value)
+    dg.dg_sample(h, buf[4:], [0], 1, sp, canvas, dg.step_out())   # 16-byte offset is fine
+    dg.dg_synchronize(h)
+    h.close()
