@@ -217,8 +217,9 @@ def run_ours(args):
 
     stream = torch.cuda.current_stream(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # inside the timed region only the roofline kernel's launches carry events
     m.dg_profile_reset(h)
-    m.dg_profile_enable(h, True)
+    m.dg_profile_enable(h, True, classes=["moe_up"])
     launches0 = m.dg_launch_count(h)
     steps_seen.clear()
     with ClockSampler(local) as clk:
@@ -249,6 +250,13 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = (time.perf_counter() - e0) * 1e3
     e2e_max, _ = aggregate(dist, e2e_ms, units, device=dev)
+
+    # per-class kernel time from one extra, untimed step with every class profiled
+    m.dg_profile_reset(h)
+    m.dg_profile_enable(h, True)
+    one_step()
+    breakdown = m.dg_profile_read(h)
+    m.dg_profile_enable(h, False)
 
     peaks, peak_kind = load_peaks()
     roof = None
@@ -287,7 +295,7 @@ def run_ours(args):
         "roofline": roof,
         "clocks": clocks,
         "prefill_s": round(prefill_s, 2),
-        "kernel_ms": {k: round(v[1], 3) for k, v in prof.items()},
+        "kernel_ms_one_step": {k: round(v[1], 3) for k, v in breakdown.items()},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(W, line["denoise_steps_per_block"])

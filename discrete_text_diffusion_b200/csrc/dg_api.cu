@@ -103,6 +103,13 @@ enum ProfClass {
 const char* kProfNames[PC_COUNT] = {"embed",  "dense_gemm", "rope_scatter", "attention", "rmsnorm",
                                     "router", "gather",     "moe_up",       "moe_down",  "combine",
                                     "lm_head", "sampler_rows", "sampler_finish"};
+static_assert(PC_EMBED == DG_PROF_EMBED && PC_DENSE == DG_PROF_DENSE_GEMM && PC_ROPE == DG_PROF_ROPE_SCATTER &&
+                  PC_ATTN == DG_PROF_ATTENTION && PC_NORM == DG_PROF_RMSNORM && PC_ROUTER == DG_PROF_ROUTER &&
+                  PC_GATHER == DG_PROF_GATHER && PC_MOE_UP == DG_PROF_MOE_UP && PC_MOE_DOWN == DG_PROF_MOE_DOWN &&
+                  PC_COMBINE == DG_PROF_COMBINE && PC_LMHEAD == DG_PROF_LM_HEAD &&
+                  PC_SAMPLER == DG_PROF_SAMPLER_ROWS && PC_FINISH == DG_PROF_SAMPLER_FINISH &&
+                  PC_COUNT == DG_PROF_COUNT,
+              "profiler classes must follow include/dg.h");
 
 }  // namespace
 
@@ -188,6 +195,7 @@ struct dg_handle {
   int32_t* h_done = nullptr;  // pinned
   // profiling
   bool prof = false;
+  uint32_t prof_mask = 0;
   struct Rec { int cls; cudaEvent_t a, b; };
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
@@ -227,8 +235,10 @@ struct ProfScope {
   int cls;
   cudaEvent_t b = nullptr;
   int n;
-  ProfScope(dg_handle* h, int c, int n_launch = 1) : H(h), cls(c), n(n_launch) {
-    if (H->prof) {
+  bool on;
+  ProfScope(dg_handle* h, int c, int n_launch = 1)
+      : H(h), cls(c), n(n_launch), on(h->prof && ((h->prof_mask >> c) & 1u)) {
+    if (on) {
       cudaEvent_t a = pool_event(H);
       b = pool_event(H);
       cudaEventRecord(a, H->stream);
@@ -236,7 +246,7 @@ struct ProfScope {
     }
   }
   ~ProfScope() {
-    if (H->prof) cudaEventRecord(b, H->stream);
+    if (on) cudaEventRecord(b, H->stream);
     H->launches += (uint64_t)n;
   }
 };
@@ -1022,9 +1032,10 @@ int dg_synchronize(dg_handle* H) {
 
 uint64_t dg_launch_count(const dg_handle* H) { return H ? H->launches : 0; }
 
-int dg_profile_enable(dg_handle* H, int on) {
+int dg_profile_enable(dg_handle* H, int mask) {
   if (!H) return DG_EINVAL;
-  H->prof = on != 0;
+  H->prof = mask != 0;
+  H->prof_mask = (uint32_t)mask;
   return DG_OK;
 }
 

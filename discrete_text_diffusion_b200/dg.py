@@ -253,8 +253,17 @@ def dg_launch_count(h: Handle) -> int:
     return int(lib().dg_launch_count(h.ptr))
 
 
-def dg_profile_enable(h: Handle, on: bool):
-    return h.check(lib().dg_profile_enable(h.ptr, 1 if on else 0))
+# profiler kernel classes in the header's order (bit k of the mask = class k)
+PROFILE_CLASSES = ("embed", "dense_gemm", "rope_scatter", "attention", "rmsnorm", "router", "gather", "moe_up",
+                   "moe_down", "combine", "lm_head", "sampler_rows", "sampler_finish")
+
+
+def dg_profile_enable(h: Handle, on: bool, classes=None):
+    """on=False: off; on=True: every class, or only the named ``classes``."""
+    mask = 0
+    if on:
+        mask = -1 if classes is None else sum(1 << PROFILE_CLASSES.index(c) for c in classes)
+    return h.check(lib().dg_profile_enable(h.ptr, mask))
 
 
 def dg_profile_reset(h: Handle):

@@ -233,8 +233,33 @@ int dg_synchronize(dg_handle* h);
 /* Kernel launches issued by this handle since creation. */
 uint64_t dg_launch_count(const dg_handle* h);
 
-/* Per-kernel-class CUDA-event timing: enable/disable, read (synchronises), reset. */
-int dg_profile_enable(dg_handle* h, int on);
+/* Kernel classes of the profiler; bit k of dg_profile_enable's mask selects class k. */
+enum {
+  DG_PROF_EMBED = 0,
+  DG_PROF_DENSE_GEMM = 1,     /* self-conditioning, QKV and O projections */
+  DG_PROF_ROPE_SCATTER = 2,
+  DG_PROF_ATTENTION = 3,      /* attention + split-KV combine */
+  DG_PROF_RMSNORM = 4,
+  DG_PROF_ROUTER = 5,         /* router logits, top-k, permutation */
+  DG_PROF_GATHER = 6,
+  DG_PROF_MOE_UP = 7,         /* grouped gate/up + SwiGLU */
+  DG_PROF_MOE_DOWN = 8,
+  DG_PROF_COMBINE = 9,
+  DG_PROF_LM_HEAD = 10,
+  DG_PROF_SAMPLER_ROWS = 11,
+  DG_PROF_SAMPLER_FINISH = 12,
+  DG_PROF_COUNT = 13
+};
+#define DG_PROFILE_ALL (-1)
+
+/*
+ * Per-kernel-class CUDA-event timing on the handle's stream.  mask = 0 turns
+ * it off; otherwise bit k times class k (DG_PROFILE_ALL: every class).  Each
+ * timed launch group costs two event records, so time only the classes you
+ * read when the surrounding run is itself being timed.  dg_profile_read
+ * synchronises; dg_profile_reset drops the records.
+ */
+int dg_profile_enable(dg_handle* h, int mask);
 int dg_profile_read(dg_handle* h, dg_profile_entry* out, int max_entries, int* n_entries);
 int dg_profile_reset(dg_handle* h);
 

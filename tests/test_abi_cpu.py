@@ -115,3 +115,12 @@ def test_null_handle_calls_fail_cleanly(lib):
     assert lib.dg_set_length(None, 0, 0) == B.DG_EINVAL
     assert lib.dg_launch_count(None) == 0
     lib.dg_destroy(None)
+
+
+def test_profile_classes_follow_header():
+    import re
+    hdr = open(os.path.join(os.path.dirname(B.LIB_PATH), "..", "include", "dg.h")).read()
+    vals = {m.group(1).lower(): int(m.group(2)) for m in re.finditer(r"DG_PROF_(\w+) = (\d+)", hdr)}
+    count = vals.pop("count")
+    assert count == len(B.PROFILE_CLASSES)
+    assert [c for c, _ in sorted(vals.items(), key=lambda x: x[1])] == list(B.PROFILE_CLASSES)
