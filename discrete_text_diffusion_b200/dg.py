@@ -22,7 +22,7 @@ EXPORTS = (
     "dg_create", "dg_destroy", "dg_last_error", "dg_prefill_prompt", "dg_set_kv", "dg_set_length",
     "dg_get_length", "dg_denoise_step", "dg_sample", "dg_generate_block", "dg_generate_block_host",
     "dg_synchronize", "dg_launch_count", "dg_profile_enable", "dg_profile_read", "dg_profile_reset",
-    "dg_selftest_philox", "dg_selftest_gemm",
+    "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc",
 )
 
 
@@ -102,6 +102,9 @@ def lib():
         L.dg_profile_reset.argtypes = [P]
         L.dg_selftest_philox.argtypes = [P, P, P, P, P, C.c_int]
         L.dg_selftest_gemm.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, P]
+        L.dg_sample_noalloc.argtypes = [P, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_int), C.c_int,
+                                        C.POINTER(DgSamplerParams), P, C.POINTER(DgStepOut), P, C.c_char_p,
+                                        C.c_size_t]
         _lib = L
     return _lib
 
@@ -225,6 +228,19 @@ def dg_denoise_step(h: Handle, req, canvas, prev_pred, step, sp: DgSamplerParams
 def dg_sample(h: Handle, logits, req, step, sp: DgSamplerParams, canvas, out: DgStepOut):
     return h.check(lib().dg_sample(h.ptr, _ptr(logits), len(req), _ints(req), step, C.byref(sp), _ptr(canvas),
                                    C.byref(out)))
+
+
+def dg_sample_noalloc(logits, req, step, sp: DgSamplerParams, canvas, out: DgStepOut = None, stream=None):
+    """dg_sample without a handle: logits [B, N, V] fp32 on the stream's device.
+    stream: a torch.cuda.Stream (or None for the legacy default stream)."""
+    B, n, V = logits.shape
+    err = C.create_string_buffer(512)
+    sptr = None if stream is None else C.c_void_p(stream.cuda_stream)
+    rc = lib().dg_sample_noalloc(_ptr(logits), B, n, V, _ints(req), step, C.byref(sp), _ptr(canvas),
+                                 None if out is None else C.byref(out), sptr, err, len(err))
+    if rc != 0:
+        raise DgError(rc, err.value.decode())
+    return rc
 
 
 def block_args(req, max_steps, schedule_steps, temperature=1.0, logit_scale_growth=1.0, stop_threshold=-1.0,

@@ -213,6 +213,51 @@ int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int 
               const dg_sampler_params* sp, int32_t* canvas, const dg_step_out* o);
 
 /*
+ * dg_sample without a handle and without allocating.  The pages have no
+ * counterpart: this is a library convenience, not a step of the method.
+ *
+ * It computes exactly what dg_sample computes (same kernels, same Philox
+ * counters) for logits [batch, n, vocab] fp32 (16-byte aligned).  It is meant
+ * for callers that must not allocate device memory: a serving runtime that
+ * reserved the GPU's memory up front, or code sampling from logits it already
+ * owns.  Those callers cannot pay for dg_create, which allocates a KV cache and
+ * workspaces.  This call never calls cudaMalloc, cudaFree or any allocating
+ * library.  Its scratch is one fixed 8 MiB device array per device that the
+ * CUDA runtime sets aside when this library's module loads.
+ *
+ * Arguments:
+ *   req: HOST [batch] request ids (Philox counter word 3), each >= 0;
+ *        1 <= batch <= 64.
+ *   n: canvas length, 1..1024.
+ *   step, sp: as for dg_sample; sp->keep_k <= n.
+ *   canvas: device [batch, n]; in: unused, out: the re-noised canvas.
+ *   o: as for dg_sample, or NULL.  x_hat / pmax / entropy that o does not
+ *      request are kept in the scratch; experts_touched is ignored.
+ *   stream: a cudaStream_t of the current device (NULL = legacy default).
+ *   err: buffer of err_len bytes for a message (may be NULL).
+ *
+ * Limits and behaviour:
+ *   - The request must fit the scratch:
+ *     ceil(vocab / 4096) * 24 bytes per row of logits, plus ~12 bytes per row
+ *     and 1 KB.  At vocab = 262144 that is about 5400 rows (21 canvases of 256).
+ *     A larger request returns DG_ECAPACITY before anything is launched.
+ *   - The first call on a device does the setup (looks up the scratch's
+ *     address, loading the module if needed); make it before any stream capture.
+ *   - Nothing in the scratch has to start at zero: a call reads only what it
+ *     wrote itself.
+ *   - Every call on a device shares the one scratch.  Calls on a device must
+ *     therefore be ordered: the same stream, or streams ordered by events.
+ *     Overlapping calls race on the scratch and give wrong results.
+ *   - The request ids are copied from pageable host memory, so the call may
+ *     wait for earlier work on the stream.
+ *   - Returns DG_OK, DG_EINVAL (bad argument), DG_ECAPACITY (too large) or
+ *     DG_ECUDA (a launch or runtime call failed).
+ */
+int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const int* req, int step,
+                      const dg_sampler_params* sp, int32_t* canvas, const dg_step_out* o, void* stream,
+                      char* err, size_t err_len);
+
+/*
  * One block per request: canvas from Philox word 1 of counter (i, 0, block,
  * req); steps t = 1..max_steps with keep_k = ceil(N t / schedule_steps) and
  * logit scale growth^(t-1), self-conditioning on the previous x_hat; a request
