@@ -178,6 +178,8 @@ struct dg_handle {
   float* part_o = nullptr;
   float* part_ml = nullptr;
   size_t part_rows_cap = 0;   // split-rows capacity of part_o / part_ml
+  float* kpart = nullptr;      // K-slice partial sums of the split-K dense projections
+  size_t kpart_floats = 0;
   // sampler workspace
   void* sws = nullptr;
   int32_t* xh[2] = {nullptr, nullptr};
@@ -300,6 +302,8 @@ int grouped_tile(const dg_handle* H, int T) {
 #endif
 int ksub_for(int mode, int ntile) { return (mode == 1 || ntile > 64) ? 2 : DG_NARROW_KSUB; }
 constexpr int kMaxKSplit = 16;   // K slices of a split-K projection (router logits)
+constexpr int kMaxDenseSplit = 8;      // K slices of the split-K dense projections
+constexpr int kDenseSplitRows = 256;   // token rows up to which they take the split-K form
 int ctas_for(int ntile) { return ntile <= 64 ? DG_NARROW_CTAS : 1; }
 
 const CUtensorMap& pick(const WMap& w, int ksub) { return ksub == 4 ? w.k4 : w.k2; }
@@ -365,11 +369,81 @@ int dense_gemm(dg_handle* H, int cls, const void* x, const void* w, const WMap* 
   return split;
 }
 
-void qkv_gemm(dg_handle* H, int l, int T) {
+// Split-K form of a dense projection for up to kDenseSplitRows tokens: the
+// token tile holds every row (up to DG_DENSE_MAXN), so each weight tile is
+// streamed once, and K is split into slices until the grid fills the SMs.
+// Slice s writes its fp32 partial sums to part + s * T * n_out ([T, n_out]
+// row-major); the consumer adds the slices in order.  (Adding the slices
+// inside a thread-block cluster through distributed shared memory measured
+// slower on this part: the partials round-trip through L2 instead.)
+#ifndef DG_DENSE_MAXN
+#define DG_DENSE_MAXN 256     // token-tile cap (rows of the N operand)
+#endif
+struct SplitPlan {
+  int ntile = 0, ksub = 2, split = 0;
+};
+
+SplitPlan split_plan(int num_sms, int T, int n_out, int K, size_t cap_floats) {
+  SplitPlan p;
+  if (T < 1 || T > kDenseSplitRows || (size_t)T * n_out > cap_floats) return p;
+  p.ntile = 32;
+  while (p.ntile < T && p.ntile < DG_DENSE_MAXN) p.ntile <<= 1;
+  const int nst = (K / 64 + p.ksub - 1) / p.ksub;
+  const int tiles = ((n_out + 127) / 128) * ((T + p.ntile - 1) / p.ntile);
+  p.split = 1;
+  while (p.split < kMaxDenseSplit && tiles * (p.split + 1) <= num_sms && (p.split + 1) * 2 <= nst &&
+         (size_t)(p.split + 1) * T * n_out <= cap_floats)
+    ++p.split;
+  return p;
+}
+
+void run_split(dg_handle* H, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
+               const CUtensorMap* b, int seg1, int seg2, int T, int n_out, int K, const SplitPlan& p, float* part) {
+  TcGemm g{};
+  g.mode = 0;
+  g.M = n_out;
+  g.K = K;
+  g.T = T;
+  g.ntile = p.ntile;
+  g.seg1 = seg1;
+  g.seg2 = seg2;
+  g.epi = EPI_STORE_F32;
+  g.out = part;
+  g.ld_out = n_out;
+  g.err = H->d_err;
+  g.ksub = p.ksub;
+  g.ctas_per_sm = 1;
+  g.ksplit = p.split;
+  g.split_stride = (size_t)T * n_out;
+  run_tc(H, a0, a1, a2, b, g);
+}
+
+// The layers' use of the split-K form: up to three weight maps stacked along
+// M (boundaries seg1, seg2), partials in H->kpart.  Returns the number of
+// slices, or 0 when the call does not take this form (nothing launched).
+int dense_gemm_part(dg_handle* H, int cls, const void* x, const WMap& a0, const WMap& a1, const WMap& a2, int seg1,
+                    int seg2, int T, int n_out, int K) {
+  if (!H->bf16 || !H->kpart) return 0;
+  const SplitPlan p = split_plan(H->num_sms, T, n_out, K, H->kpart_floats);
+  if (p.split < 1) return 0;
+  ProfScope ps(H, cls);
+  run_split(H, pick(a0, p.ksub), pick(a1, p.ksub), pick(a2, p.ksub), bmap(H, x, K, H->T_max, p.ntile, p.ksub), seg1,
+            seg2, T, n_out, K, p, H->kpart);
+  return p.split;
+}
+
+// q|k|v rows of the layer (fp32 [T, (Hq + 2 Hkv) hd]): returns the number of
+// K slices written to H->kpart by the split-K form, or 0 when they are in H->qkv.
+int qkv_gemm(dg_handle* H, int l, int T) {
   const dg_config& c = H->c;
   const dg_layer_weights& L = H->lw[l];
   const int nq = c.n_heads * c.head_dim, nk = c.n_kv_heads * c.head_dim;
   const int ld = nq + 2 * nk;
+  if (H->bf16) {
+    const LayerMaps& M = H->lmaps[l];
+    const int ns = dense_gemm_part(H, PC_DENSE, H->xn, M.wq, M.wk, M.wv, nq, nq + nk, T, ld, c.d_model);
+    if (ns > 0) return ns;
+  }
   ProfScope ps(H, PC_DENSE, H->bf16 ? 1 : 3);
   if (!H->bf16) {
     const float* x = (const float*)H->xn;
@@ -378,7 +452,7 @@ void qkv_gemm(dg_handle* H, int l, int T) {
                             H->stream);
     launch_gemm_simt<float>(x, (const float*)L.wv, T, nk, c.d_model, EPI_STORE_F32, H->qkv + nq + nk, ld, nullptr,
                             H->stream);
-    return;
+    return 0;
   }
   TcGemm g{};
   g.mode = 0;
@@ -397,6 +471,7 @@ void qkv_gemm(dg_handle* H, int l, int T) {
   const LayerMaps& M = H->lmaps[l];
   run_tc(H, pick(M.wq, g.ksub), pick(M.wk, g.ksub), pick(M.wv, g.ksub),
          bmap(H, H->xn, c.d_model, H->T_max, g.ntile, g.ksub), g);
+  return 0;
 }
 
 void moe_gemms(dg_handle* H, int l, int T) {
@@ -510,29 +585,42 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
     launch_embed<T>(tokens, prev, (const T*)H->embed, H->h, (T*)H->eprev, Tn, c.d_model, c.vocab, H->d_err,
                     H->stream);
   }
-  if (prev) dense_gemm(H, PC_DENSE, H->eprev, H->w_sc, &H->m_wsc, Tn, c.d_model, c.d_model,
-                       EPI_ADD_F32, H->h, c.d_model);
+  int scs = 0;  // K slices of the self-conditioning term in H->kpart
+  if (prev) {
+    scs = dense_gemm_part(H, PC_DENSE, H->eprev, H->m_wsc, H->m_wsc, H->m_wsc, INT_MAX, INT_MAX, Tn, c.d_model,
+                          c.d_model);
+    if (!scs) dense_gemm(H, PC_DENSE, H->eprev, H->w_sc, &H->m_wsc, Tn, c.d_model, c.d_model, EPI_ADD_F32, H->h,
+                         c.d_model);
+  }
   {
     ProfScope ps(H, PC_NORM);
     const float* w0 = c.n_layers > 0 ? H->lw[0].attn_norm : H->final_norm;
-    launch_rmsnorm<T>(H->h, w0, xn, Tn, c.d_model, eps, H->stream);
+    if (scs) launch_add_rmsnorm<T>(H->h, H->kpart, scs, (size_t)Tn * c.d_model, w0, xn, Tn, c.d_model, eps,
+                                   H->stream);
+    else launch_rmsnorm<T>(H->h, w0, xn, Tn, c.d_model, eps, H->stream);
   }
   const int ldqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& L = H->lw[l];
-    qkv_gemm(H, l, Tn);
+    const int qs = qkv_gemm(H, l, Tn);
     {
       ProfScope ps(H, PC_ROPE);
-      launch_rope_scatter<T>(H->qkv, (T*)H->q, (T*)kc_layer(H, l), (T*)vt_layer(H, l), (const float*)H->rope, bi,
-                             nq, c.n_heads, c.n_kv_heads, c.head_dim, c.max_ctx, H->stream);
+      launch_rope_scatter<T>(qs ? H->kpart : H->qkv, qs ? qs : 1, (size_t)Tn * ldqkv, (T*)H->q, (T*)kc_layer(H, l),
+                             (T*)vt_layer(H, l), (const float*)H->rope, bi, nq, c.n_heads, c.n_kv_heads, c.head_dim,
+                             c.max_ctx, H->stream);
     }
-    (void)ldqkv;
     attention(H, l, bi, nq, causal);
-    dense_gemm(H, PC_DENSE, H->attn, L.wo, H->bf16 ? &H->lmaps[l].wo : nullptr, Tn, c.d_model, c.n_heads * c.head_dim,
-               EPI_ADD_F32, H->h, c.d_model);
+    const int nqc = c.n_heads * c.head_dim;
+    const int os = H->bf16 ? dense_gemm_part(H, PC_DENSE, H->attn, H->lmaps[l].wo, H->lmaps[l].wo, H->lmaps[l].wo,
+                                             INT_MAX, INT_MAX, Tn, c.d_model, nqc)
+                           : 0;
+    if (!os) dense_gemm(H, PC_DENSE, H->attn, L.wo, H->bf16 ? &H->lmaps[l].wo : nullptr, Tn, c.d_model, nqc,
+                        EPI_ADD_F32, H->h, c.d_model);
     {
       ProfScope ps(H, PC_NORM);
-      launch_rmsnorm<T>(H->h, L.ffn_norm, xn, Tn, c.d_model, eps, H->stream);
+      if (os) launch_add_rmsnorm<T>(H->h, H->kpart, os, (size_t)Tn * c.d_model, L.ffn_norm, xn, Tn, c.d_model, eps,
+                                    H->stream);
+      else launch_rmsnorm<T>(H->h, L.ffn_norm, xn, Tn, c.d_model, eps, H->stream);
     }
     // the router projection has one 128-row weight tile: split K for parallelism
     const int rsplit = dense_gemm(H, PC_ROUTER, H->xn, L.router_w, H->bf16 ? &H->lmaps[l].router : nullptr, Tn,
@@ -759,6 +847,10 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
     H->logits = dalloc<float>((size_t)nrow * c.vocab, &ok);
     H->rope = dalloc<float2>((size_t)c.max_ctx * (c.head_dim / 2), &ok);
     H->tok_ws = dalloc<int32_t>((size_t)T, &ok);
+    if (c.dtype == DG_BF16) {
+      H->kpart_floats = (size_t)kMaxDenseSplit * std::min(T, kDenseSplitRows) * std::max(ldqkv, c.d_model);
+      H->kpart = dalloc<float>(H->kpart_floats, &ok);
+    }
     if (c.dtype == DG_BF16 && c.head_dim == 256) {
       H->part_rows_cap = (size_t)16 * c.canvas * c.n_heads;
       H->part_o = dalloc<float>(H->part_rows_cap * c.head_dim, &ok);
@@ -861,7 +953,7 @@ void dg_destroy(dg_handle* H) {
   void* ps[] = {H->kc, H->vt, H->h, H->xn, H->eprev, H->qkv, H->q, H->attn, H->glog, H->ids, H->wts, H->cnt,
                 H->off, H->perm, H->work, H->n_work, H->touched, H->xp, H->hb, H->y, H->logits, H->rope, H->sws,
                 H->xh[0], H->xh[1], H->pmax, H->ent, H->keep, H->meanh, H->stop, H->done, H->canvas, H->out_tok,
-                H->req_dev, H->tok_ws, H->d_err, H->part_o, H->part_ml};
+                H->req_dev, H->tok_ws, H->d_err, H->part_o, H->part_ml, H->kpart};
   for (void* p : ps)
     if (p) cudaFree(p);
   if (H->h_done) cudaFreeHost(H->h_done);
@@ -1105,6 +1197,24 @@ int dg_selftest_gemm(dg_handle* H, const void* x, const void* w, int T, int M, i
     return fail(H, DG_EINVAL, "GEMM tiling rejected");
   H->launches += 1;
   return check_launch(H, "selftest gemm");
+}
+
+int dg_selftest_gemm_split(dg_handle* H, const void* x, const void* w, int T, int M, int K, float* part,
+                           int max_split, int* nsplit) {
+  if (!H || !x || !w || !part || !nsplit || T < 1 || M < 1 || K < 64 || K % 64 || max_split < 1)
+    return H ? fail(H, DG_EINVAL, "bad gemm args") : DG_EINVAL;
+  if (!H->bf16) return fail(H, DG_ESTATE, "needs a bf16 handle");
+  if (!aligned16(x) || !aligned16(w)) return fail(H, DG_EINVAL, "unaligned operands");
+  const SplitPlan p = split_plan(H->num_sms, T, M, K, (size_t)max_split * T * M);
+  if (p.split < 1) return fail(H, DG_EINVAL, "T = %d is above the split-K form's %d rows", T, kDenseSplitRows);
+  CUtensorMap mx, mw;
+  if (!tmap_chunks(&mx, x, K, T, K, (uint32_t)p.ntile, (uint32_t)p.ksub) ||
+      !tmap_chunks(&mw, w, K, M, K, 128, (uint32_t)p.ksub))
+    return fail(H, DG_ECUDA, "tensor map encode failed");
+  run_split(H, mw, mw, mw, &mx, INT_MAX, INT_MAX, T, M, K, p, part);
+  H->launches += 1;
+  *nsplit = p.split;
+  return check_launch(H, "selftest split gemm");
 }
 
 }  // extern "C"

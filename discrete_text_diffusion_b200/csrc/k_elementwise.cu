@@ -110,10 +110,145 @@ __global__ void rmsnorm_kernel(const float* __restrict__ h, const float* __restr
   for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f32<T>(x[j] * r * w[j]);
 }
 
+// Register-resident rows: thread x owns float4 columns x, x + blockDim, ...
+// (VPT of them), so a row is read from memory once and normalised from
+// registers.  One CTA per row, blockDim = ceil(d / 4 / VPT) rounded to a warp.
+constexpr int kRowThreadsMax = 1024;
+
+__host__ __device__ constexpr int row_threads(int d4, int vpt) { return ((d4 + vpt - 1) / vpt + 31) / 32 * 32; }
+
+inline int row_vpt(int d) {
+  if (d % 4 != 0) return 0;
+  const int d4 = d / 4;
+  for (int v = 1; v <= 8; v *= 2)
+    if (row_threads(d4, v) <= kRowThreadsMax) return v;
+  return 0;
+}
+
+template <typename T, int VPT>
+__global__ void __launch_bounds__(kRowThreadsMax) rmsnorm_reg_kernel(const float* __restrict__ h,
+                                                                     const float* __restrict__ w,
+                                                                     T* __restrict__ xn, int d, float eps) {
+  __shared__ float red[32];
+  const int t = blockIdx.x, d4 = d >> 2;
+  const float4* x4 = reinterpret_cast<const float4*>(h + (size_t)t * d);
+  float4 v[VPT];
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int j = threadIdx.x + u * blockDim.x;
+    v[u] = j < d4 ? x4[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += v[u].x * v[u].x + v[u].y * v[u].y + v[u].z * v[u].z + v[u].w * v[u].w;
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / (float)d + eps);
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+  T* o = xn + (size_t)t * d;
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int j = threadIdx.x + u * blockDim.x;
+    if (j < d4) {
+      const float4 g = w4[j];
+      store4<T>(o, j, make_float4(v[u].x * r * g.x, v[u].y * r * g.y, v[u].z * r * g.z, v[u].w * r * g.w));
+    }
+  }
+}
+
 template <typename T>
 void launch_rmsnorm(const float* h, const float* w, T* xn, int n_tok, int d, float eps, cudaStream_t s) {
   if (n_tok <= 0) return;
-  rmsnorm_kernel<T><<<n_tok, 256, 0, s>>>(h, w, xn, d, eps);
+  const int vpt = row_vpt(d);
+  const int thr = vpt ? row_threads(d / 4, vpt) : 256;
+  switch (vpt) {
+    case 1: rmsnorm_reg_kernel<T, 1><<<n_tok, thr, 0, s>>>(h, w, xn, d, eps); break;
+    case 2: rmsnorm_reg_kernel<T, 2><<<n_tok, thr, 0, s>>>(h, w, xn, d, eps); break;
+    case 4: rmsnorm_reg_kernel<T, 4><<<n_tok, thr, 0, s>>>(h, w, xn, d, eps); break;
+    case 8: rmsnorm_reg_kernel<T, 8><<<n_tok, thr, 0, s>>>(h, w, xn, d, eps); break;
+    default: rmsnorm_kernel<T><<<n_tok, 256, 0, s>>>(h, w, xn, d, eps);
+  }
+}
+
+// Residual add of split-K partial sums, then RMSNorm.  Each thread owns VPT
+// float4 columns; the slices are added in slice order.  VPT 0 is the generic
+// form: any d, columns strided over the block, the row re-read for the norm.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(kRowThreadsMax) add_rmsnorm_kernel(float* __restrict__ h,
+                                                                     const float* __restrict__ part, int nsplit,
+                                                                     size_t split_stride,
+                                                                     const float* __restrict__ w,
+                                                                     T* __restrict__ xn, int d, float eps) {
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  float* hr = h + (size_t)t * d;
+  const float* pr = part + (size_t)t * d;
+  T* o = xn + (size_t)t * d;
+  float ss = 0.f;
+  if constexpr (VPT == 0) {
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+      float a = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) a += pr[(size_t)sp * split_stride + j];
+      const float x = hr[j] + a;
+      hr[j] = x;
+      ss += x * x;
+    }
+    ss = block_sum(ss, red);
+    const float r = rsqrtf(ss / (float)d + eps);
+    for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f32<T>(hr[j] * r * w[j]);
+  } else {
+    const int d4 = d >> 2;
+    float4* h4 = reinterpret_cast<float4*>(hr);
+    const float4* p4 = reinterpret_cast<const float4*>(pr);
+    const size_t s4 = split_stride / 4;
+    float4 v[VPT];
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      const int j = threadIdx.x + u * blockDim.x;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < d4) {
+        float4 a = p4[j];
+        for (int sp0 = 1; sp0 < nsplit; sp0 += 4) {
+          float4 b[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (sp0 + q < nsplit) b[q] = p4[(size_t)(sp0 + q) * s4 + j];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (sp0 + q < nsplit) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
+        }
+        float4 x = h4[j];
+        x.x += a.x; x.y += a.y; x.z += a.z; x.w += a.w;
+        h4[j] = x;
+        v[u] = x;
+        ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+      }
+    }
+    ss = block_sum(ss, red);
+    const float r = rsqrtf(ss / (float)d + eps);
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      const int j = threadIdx.x + u * blockDim.x;
+      if (j < d4) {
+        const float4 g = w4[j];
+        store4<T>(o, j, make_float4(v[u].x * r * g.x, v[u].y * r * g.y, v[u].z * r * g.z, v[u].w * r * g.w));
+      }
+    }
+  }
+}
+
+template <typename T>
+void launch_add_rmsnorm(float* h, const float* part, int nsplit, size_t split_stride, const float* w, T* xn,
+                        int n_tok, int d, float eps, cudaStream_t s) {
+  if (n_tok <= 0) return;
+  const int vpt = (split_stride % 4 == 0) ? row_vpt(d) : 0;
+  const int thr = vpt ? row_threads(d / 4, vpt) : 256;
+  switch (vpt) {
+    case 1: add_rmsnorm_kernel<T, 1><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps); break;
+    case 2: add_rmsnorm_kernel<T, 2><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps); break;
+    case 4: add_rmsnorm_kernel<T, 4><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps); break;
+    case 8: add_rmsnorm_kernel<T, 8><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps); break;
+    default: add_rmsnorm_kernel<T, 0><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps);
+  }
 }
 
 // ---------------------------------------------------------------- combine
@@ -180,11 +315,80 @@ __global__ void combine_kernel(float* __restrict__ h, const float* __restrict__ 
   for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = from_f32<T>(hr[j] * r * norm_w[j]);
 }
 
+// Register-resident combine: as combine_kernel, each thread owning VPT float4
+// columns; the slot loads of a column are issued four at a time and summed
+// in slot order.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(kRowThreadsMax) combine_reg_kernel(float* __restrict__ h,
+                                                                     const float* __restrict__ y,
+                                                                     const float* __restrict__ wts, int k,
+                                                                     const float* __restrict__ norm_w,
+                                                                     T* __restrict__ xn, int d, float eps) {
+  __shared__ float red[32];
+  __shared__ float ws[16];
+  const int t = blockIdx.x, d4 = d >> 2;
+  if (threadIdx.x < k) ws[threadIdx.x] = wts[(size_t)t * k + threadIdx.x];
+  __syncthreads();
+  float4* h4 = reinterpret_cast<float4*>(h + (size_t)t * d);
+  const float4* y4 = reinterpret_cast<const float4*>(y + (size_t)t * k * d);
+  float4 v[VPT];
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int j = threadIdx.x + u * blockDim.x;
+    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < d4) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < k; s0 += 4) {
+        float4 yv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (s0 + q < k) yv[q] = y4[(size_t)(s0 + q) * d4 + j];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (s0 + q < k) {
+            const float c = ws[s0 + q];
+            acc.x += c * yv[q].x;
+            acc.y += c * yv[q].y;
+            acc.z += c * yv[q].z;
+            acc.w += c * yv[q].w;
+          }
+      }
+      float4 x = h4[j];
+      x.x += acc.x; x.y += acc.y; x.z += acc.z; x.w += acc.w;
+      h4[j] = x;
+      v[u] = x;
+      ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+    }
+  }
+  if (norm_w == nullptr) return;
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / (float)d + eps);
+  const float4* w4 = reinterpret_cast<const float4*>(norm_w);
+  T* o = xn + (size_t)t * d;
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int j = threadIdx.x + u * blockDim.x;
+    if (j < d4) {
+      const float4 g = w4[j];
+      store4<T>(o, j, make_float4(v[u].x * r * g.x, v[u].y * r * g.y, v[u].z * r * g.z, v[u].w * r * g.w));
+    }
+  }
+}
+
 template <typename T>
 void launch_combine(float* h, const float* y, const float* wts, int k, const float* norm_w, T* xn, int n_tok,
                     int d, float eps, cudaStream_t s) {
   if (n_tok <= 0) return;
-  combine_kernel<T><<<n_tok, 256, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps);
+  const int vpt = k <= 16 ? row_vpt(d) : 0;
+  const int thr = vpt ? row_threads(d / 4, vpt) : 256;
+  switch (vpt) {
+    case 1: combine_reg_kernel<T, 1><<<n_tok, thr, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps); break;
+    case 2: combine_reg_kernel<T, 2><<<n_tok, thr, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps); break;
+    case 4: combine_reg_kernel<T, 4><<<n_tok, thr, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps); break;
+    case 8: combine_reg_kernel<T, 8><<<n_tok, thr, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps); break;
+    default: combine_kernel<T><<<n_tok, 256, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps);
+  }
 }
 
 // ------------------------------------------------------------ RoPE scatter
@@ -192,7 +396,8 @@ void launch_combine(float* h, const float* y, const float* wts, int k, const flo
 // continues the prompt's positions).  rope_cs[pos][j] = (cos, sin) of
 // pos * base^(-2j/hd), tabulated on the host in double precision.
 template <typename T>
-__global__ void rope_scatter_kernel(const float* __restrict__ qkv, T* __restrict__ q, T* __restrict__ kc,
+__global__ void rope_scatter_kernel(const float* __restrict__ qkv, int nsplit, size_t split_stride,
+                                    T* __restrict__ q, T* __restrict__ kc,
                                     T* __restrict__ vt, const float2* __restrict__ rope_cs, BatchInfo bi, int nq,
                                     int hq, int hkv, int hd, int max_ctx) {
   const int t = blockIdx.x;            // token row b*nq + i
@@ -204,7 +409,11 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, T* __restrict
   const int ncol = (hq + 2 * hkv) * hd;
   const float* src = qkv + (size_t)t * ncol + (size_t)head * hd;
   for (int j = threadIdx.x; j < half; j += blockDim.x) {
-    const float x1 = src[j], x2 = src[j + half];
+    float x1 = src[j], x2 = src[j + half];
+    for (int sp = 1; sp < nsplit; ++sp) {
+      x1 += src[(size_t)sp * split_stride + j];
+      x2 += src[(size_t)sp * split_stride + j + half];
+    }
     if (head < hq + hkv) {
       const float2 cs = rope_cs[(size_t)pos * half + j];
       const float r1 = x1 * cs.x - x2 * cs.y;
@@ -227,14 +436,102 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, T* __restrict
   }
 }
 
+// Tiled form: one CTA per (32 token rows, head).  Q and K rows are rotated
+// four pairs per thread with 16-byte loads.  V rows are staged in shared
+// memory and written transposed, one head dimension per warp instruction with
+// lane = token, so consecutive lanes store consecutive cache positions.
+constexpr int kRopeTok = 32;
+
 template <typename T>
-void launch_rope_scatter(const float* qkv, T* q, T* kc, T* vt, const float* rope_cs, const BatchInfo& bi,
-                         int nq, int hq, int hkv, int hd, int max_ctx, cudaStream_t s) {
+__global__ void __launch_bounds__(256) rope_scatter_tiled_kernel(const float* __restrict__ qkv, int nsplit,
+                                                                 size_t split_stride, T* __restrict__ q,
+                                                                 T* __restrict__ kc, T* __restrict__ vt,
+                                                                 const float2* __restrict__ rope_cs, BatchInfo bi,
+                                                                 int nq, int n_tok, int hq, int hkv, int hd,
+                                                                 int max_ctx) {
+  extern __shared__ __align__(16) unsigned char rope_smem[];
+  const int t0 = blockIdx.x * kRopeTok;
+  const int head = blockIdx.y;
+  const int half = hd >> 1, g4 = half >> 2;
+  const size_t ncol = (size_t)(hq + 2 * hkv) * hd;
+  const int ntk = min(kRopeTok, n_tok - t0);
+  if (head < hq + hkv) {
+    for (int idx = threadIdx.x; idx < ntk * g4; idx += blockDim.x) {
+      const int tt = idx / g4, jg = idx - tt * g4, j = jg * 4;
+      const int t = t0 + tt;
+      const int b = t / nq, i = t - b * nq;
+      const int pos = bi.len[b] + i;
+      const float* src = qkv + (size_t)t * ncol + (size_t)head * hd;
+      float4 x1 = *reinterpret_cast<const float4*>(src + j);
+      float4 x2 = *reinterpret_cast<const float4*>(src + half + j);
+      for (int sp = 1; sp < nsplit; ++sp) {
+        const float4 a = *reinterpret_cast<const float4*>(src + (size_t)sp * split_stride + j);
+        const float4 c = *reinterpret_cast<const float4*>(src + (size_t)sp * split_stride + half + j);
+        x1.x += a.x; x1.y += a.y; x1.z += a.z; x1.w += a.w;
+        x2.x += c.x; x2.y += c.y; x2.z += c.z; x2.w += c.w;
+      }
+      const float4* cs4 = reinterpret_cast<const float4*>(rope_cs + (size_t)pos * half + j);
+      const float4 ca = cs4[0], cb = cs4[1];  // (cos, sin) of pairs j, j+1 | j+2, j+3
+      const float4 r1 = make_float4(x1.x * ca.x - x2.x * ca.y, x1.y * ca.z - x2.y * ca.w, x1.z * cb.x - x2.z * cb.y,
+                                    x1.w * cb.z - x2.w * cb.w);
+      const float4 r2 = make_float4(x2.x * ca.x + x1.x * ca.y, x2.y * ca.z + x1.y * ca.w, x2.z * cb.x + x1.z * cb.y,
+                                    x2.w * cb.z + x1.w * cb.w);
+      T* dst;
+      if (head < hq) {
+        dst = q + (((size_t)b * hq + head) * nq + i) * hd;
+      } else {
+        dst = kc + (((size_t)bi.slot[b] * hkv + (head - hq)) * max_ctx + pos) * hd;
+      }
+      store4<T>(dst, jg, r1);
+      store4<T>(dst + half, jg, r2);
+    }
+    return;
+  }
+  T* tile = reinterpret_cast<T*>(rope_smem);
+  const int ld = hd + 2;  // odd word stride for 2-byte T: conflict-free column reads
+  const int d4n = hd >> 2;
+  for (int idx = threadIdx.x; idx < ntk * d4n; idx += blockDim.x) {
+    const int tt = idx / d4n, jj = (idx - tt * d4n) * 4;
+    const float* src = qkv + (size_t)(t0 + tt) * ncol + (size_t)head * hd + jj;
+    float4 x = *reinterpret_cast<const float4*>(src);
+    for (int sp = 1; sp < nsplit; ++sp) {
+      const float4 a = *reinterpret_cast<const float4*>(src + (size_t)sp * split_stride);
+      x.x += a.x; x.y += a.y; x.z += a.z; x.w += a.w;
+    }
+    T* r = tile + tt * ld + jj;
+    r[0] = from_f32<T>(x.x);
+    r[1] = from_f32<T>(x.y);
+    r[2] = from_f32<T>(x.z);
+    r[3] = from_f32<T>(x.w);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (lane < ntk) {
+    const int t = t0 + lane;
+    const int b = t / nq, i = t - b * nq;
+    const int pos = bi.len[b] + i;
+    T* col = vt + ((size_t)bi.slot[b] * hkv + (head - hq - hkv)) * hd * (size_t)max_ctx + pos;
+    for (int dd = w; dd < hd; dd += nw) col[(size_t)dd * max_ctx] = tile[lane * ld + dd];
+  }
+}
+
+template <typename T>
+void launch_rope_scatter(const float* qkv, int nsplit, size_t split_stride, T* q, T* kc, T* vt,
+                         const float* rope_cs, const BatchInfo& bi, int nq, int hq, int hkv, int hd, int max_ctx,
+                         cudaStream_t s) {
   const int n_tok = bi.B * nq;
   if (n_tok <= 0) return;
+  if (hd % 8 == 0) {
+    dim3 grid((n_tok + kRopeTok - 1) / kRopeTok, hq + 2 * hkv);
+    const size_t smem = (size_t)kRopeTok * (hd + 2) * sizeof(T);
+    rope_scatter_tiled_kernel<T><<<grid, 256, smem, s>>>(qkv, nsplit, split_stride, q, kc, vt,
+                                                         reinterpret_cast<const float2*>(rope_cs), bi, nq, n_tok,
+                                                         hq, hkv, hd, max_ctx);
+    return;
+  }
   dim3 grid(n_tok, hq + 2 * hkv);
-  rope_scatter_kernel<T><<<grid, 128, 0, s>>>(qkv, q, kc, vt, reinterpret_cast<const float2*>(rope_cs), bi,
-                                              nq, hq, hkv, hd, max_ctx);
+  rope_scatter_kernel<T><<<grid, 128, 0, s>>>(qkv, nsplit, split_stride, q, kc, vt,
+                                              reinterpret_cast<const float2*>(rope_cs), bi, nq, hq, hkv, hd, max_ctx);
 }
 
 // ------------------------------------------------------------ gather rows
@@ -304,8 +601,10 @@ void launch_set_kv(const T* k, const T* v, T* kc, T* vt, int hkv, int n, int hd,
   template void launch_rmsnorm<T>(const float*, const float*, T*, int, int, float, cudaStream_t);            \
   template void launch_combine<T>(float*, const float*, const float*, int, const float*, T*, int, int, float, \
                                   cudaStream_t);                                                             \
-  template void launch_rope_scatter<T>(const float*, T*, T*, T*, const float*, const BatchInfo&, int, int, int, \
-                                       int, int, cudaStream_t);                                              \
+  template void launch_rope_scatter<T>(const float*, int, size_t, T*, T*, T*, const float*, const BatchInfo&,  \
+                                       int, int, int, int, int, cudaStream_t);                               \
+  template void launch_add_rmsnorm<T>(float*, const float*, int, size_t, const float*, T*, int, int, float,   \
+                                      cudaStream_t);                                                         \
   template void launch_gather_rows<T>(const T*, const int32_t*, T*, int, int, int, cudaStream_t);            \
   template void launch_set_kv<T>(const T*, const T*, T*, T*, int, int, int, int, cudaStream_t);
 DG_INST(float)

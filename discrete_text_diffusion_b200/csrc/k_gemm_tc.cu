@@ -48,6 +48,12 @@ constexpr int kMaxSmem = 232448;        // 227 KB opt-in limit per CTA
 #define DG_GEMM_CTAS_PER_SM 1           // default co-resident CTAs per SM
 #endif
 constexpr int kSmemPerSm = 233472;      // 228 KB of shared memory per SM
+#ifndef DG_EPI_STAGE_MODES
+#define DG_EPI_STAGE_MODES 1            // bit m: mode m writes its output through the staging tile (dense only:
+                                        // the grouped kernels measured no gain or a loss)
+#endif
+constexpr int kEpiRows = 32;            // token rows per epilogue chunk
+constexpr int kEpiBytes = kEpiRows * kBM * 4;  // staging tile of one chunk (fp32) = 16 KB
 
 struct TcLayout {
   int n_a;          // weight operands per stage (1 or 2)
@@ -68,7 +74,7 @@ static TcLayout tc_layout(const TcGemm& p) {
   L.per_sm = std::max(1, std::min(3, p.ctas_per_sm > 0 ? p.ctas_per_sm : DG_GEMM_CTAS_PER_SM));
   // the tensor maps are built for this chunk count: it is never changed here
   L.ksub = std::max(1, std::min(4, p.ksub > 0 ? p.ksub : DG_GEMM_KSUB));
-  const int overhead = 1024 /*align*/ + 1024 /*barriers*/;
+  const int overhead = 1024 /*align*/ + 1024 /*barriers*/ + (((DG_EPI_STAGE_MODES >> p.mode) & 1) ? kEpiBytes : 0);
   for (;;) {
     // TMEM: every co-resident CTA holds its accumulators
     L.n_acc_buf = (L.per_sm * 2 * L.acc_cols <= 512) ? 2 : 1;
@@ -95,6 +101,7 @@ int gemm_tc_smem_bytes(const TcGemm& p, int* stages) {
 struct TcKParams {
   TcGemm g;
   int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, n_ttiles, ksub;
+  int vec;   // output rows may be written as aligned 16-byte vectors
 };
 
 // Work item -> weight tile, token rows and (dense split-K) the range of K
@@ -249,8 +256,21 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
+    // Per chunk of 32 token rows: each warp reads its 32-lane quarter of the
+    // accumulator (row m = m0 + q*32 + lane, one column per token) and writes
+    // it transposed into a [token][128] staging tile in shared memory; then
+    // the 128 epilogue threads write whole output rows with 16-byte stores
+    // (512 bytes of fp32, or 256 of bf16, per token row).  Writing the
+    // accumulator column by column instead (one 128-byte store per warp
+    // instruction) leaves the epilogue store-issue bound.
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
+    const int te = threadIdx.x - 64;  // 0..127 over the epilogue warps
+    float* stg = reinterpret_cast<float*>(base + P.stages * P.stage_bytes + 1024);
+    __nv_bfloat16* stg_b = reinterpret_cast<__nv_bfloat16*>(stg);
+    const bool f32out = g.mode == 2 || g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32;
+    float* out_f = reinterpret_cast<float*>(g.out);
+    __nv_bfloat16* out_b = reinterpret_cast<__nv_bfloat16*>(g.out);
     int it = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
       int m0, e, row0, rows, j0, j1, ks;
@@ -260,50 +280,108 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       if (!mbar_wait(&acc_full[ab], use & 1u, err, kErrTimeoutEpi)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * P.acc_cols);
-      const int m = m0 + r;
-      const bool mvalid = m < g.M;
-      for (int c0 = 0; c0 < rows; c0 += 32) {
+      const float bv = (g.bias && m0 + r < g.M) ? g.bias[m0 + r] : 0.f;
+      const bool staged = (DG_EPI_STAGE_MODES >> g.mode) & 1;
+      for (int c0 = 0; c0 < rows; c0 += kEpiRows) {
         uint32_t v[32];
         tmem_ld32(tbase + (uint32_t)c0, v);
-        if (g.mode == 1) {
-          uint32_t u[32];
-          tmem_ld32(tbase + (uint32_t)(g.ntile + c0), u);
-          tmem_ld_wait();
-          if (mvalid) {
-            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out);
+        if (!staged) {
+          // direct form: each thread writes its row m, one token column at a time
+          const int m = m0 + r;
+          if (g.mode == 1) {
+            uint32_t u[32];
+            tmem_ld32(tbase + (uint32_t)(g.ntile + c0), u);
+            tmem_ld_wait();
+            if (m < g.M) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (c0 + j < rows) {
-                const float gt = __uint_as_float(v[j]), up = __uint_as_float(u[j]);
-                const float hv = gt / (1.f + expf(-gt)) * up;
-                o[(size_t)(row0 + c0 + j) * g.ld_out + m] = __float2bfloat16_rn(hv);
+              for (int j = 0; j < 32; ++j) {
+                if (c0 + j < rows) {
+                  const float gt = __uint_as_float(v[j]), up = __uint_as_float(u[j]);
+                  out_b[(size_t)(row0 + c0 + j) * g.ld_out + m] = __float2bfloat16_rn(gt / (1.f + expf(-gt)) * up);
+                }
               }
             }
-          }
-        } else {
-          tmem_ld_wait();
-          if (mvalid) {
-            const float bv = g.bias ? g.bias[m] : 0.f;
+          } else {
+            tmem_ld_wait();
+            if (m < g.M) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (c0 + j < rows) {
-                const float acc = __uint_as_float(v[j]) + bv;
-                if (g.mode == 2) {
-                  const int orow = g.row_map[row0 + c0 + j];
-                  reinterpret_cast<float*>(g.out)[(size_t)orow * g.ld_out + m] = acc;
-                } else if (g.epi == EPI_STORE_F32) {
-                  reinterpret_cast<float*>(g.out)[(size_t)ks * g.split_stride + (size_t)(row0 + c0 + j) * g.ld_out + m] =
-                      acc;
-                } else if (g.epi == EPI_ADD_F32) {
-                  reinterpret_cast<float*>(g.out)[(size_t)(row0 + c0 + j) * g.ld_out + m] += acc;
-                } else {
-                  reinterpret_cast<__nv_bfloat16*>(g.out)[(size_t)(row0 + c0 + j) * g.ld_out + m] =
-                      __float2bfloat16_rn(acc);
+              for (int j = 0; j < 32; ++j) {
+                if (c0 + j < rows) {
+                  const float acc = __uint_as_float(v[j]) + bv;
+                  const int tok = row0 + c0 + j;
+                  if (g.mode == 2) out_f[(size_t)g.row_map[tok] * g.ld_out + m] = acc;
+                  else if (g.epi == EPI_STORE_F32) out_f[(size_t)ks * g.split_stride + (size_t)tok * g.ld_out + m] = acc;
+                  else if (g.epi == EPI_ADD_F32) out_f[(size_t)tok * g.ld_out + m] += acc;
+                  else out_b[(size_t)tok * g.ld_out + m] = __float2bfloat16_rn(acc);
                 }
               }
             }
           }
+          continue;
         }
+        if (g.mode == 1) {
+          uint32_t u[32];
+          tmem_ld32(tbase + (uint32_t)(g.ntile + c0), u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float gt = __uint_as_float(v[j]), up = __uint_as_float(u[j]);
+            stg_b[j * kBM + r] = __float2bfloat16_rn(gt / (1.f + expf(-gt)) * up);
+          }
+        } else if (f32out) {
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[j * kBM + r] = __uint_as_float(v[j]) + bv;
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg_b[j * kBM + r] = __float2bfloat16_rn(__uint_as_float(v[j]) + bv);
+        }
+        named_barrier_sync(1, 128);
+        const int nrow = min(kEpiRows, rows - c0);
+        if (f32out) {
+#pragma unroll 4
+          for (int it2 = 0; it2 < kEpiRows * 32 / 128; ++it2) {
+            const int idx = it2 * 128 + te, row = idx >> 5, c4 = idx & 31;
+            const int mm = m0 + c4 * 4;
+            if (row < nrow && mm < g.M) {
+              const int tok = row0 + c0 + row;
+              float* dst = (g.mode == 2) ? out_f + (size_t)g.row_map[tok] * g.ld_out + mm
+                                         : out_f + (size_t)ks * g.split_stride + (size_t)tok * g.ld_out + mm;
+              const float4 val = *reinterpret_cast<const float4*>(stg + row * kBM + c4 * 4);
+              const bool add = g.mode == 0 && g.epi == EPI_ADD_F32;
+              if (P.vec && mm + 3 < g.M) {
+                float4* d4 = reinterpret_cast<float4*>(dst);
+                if (add) {
+                  float4 o = *d4;
+                  o.x += val.x; o.y += val.y; o.z += val.z; o.w += val.w;
+                  *d4 = o;
+                } else {
+                  *d4 = val;
+                }
+              } else {
+                const float vv[4] = {val.x, val.y, val.z, val.w};
+                for (int c = 0; c < 4 && mm + c < g.M; ++c) dst[c] = add ? dst[c] + vv[c] : vv[c];
+              }
+            }
+          }
+        } else {
+#pragma unroll 4
+          for (int it2 = 0; it2 < kEpiRows * 16 / 128; ++it2) {
+            const int idx = it2 * 128 + te, row = idx >> 4, c8 = idx & 15;
+            const int mm = m0 + c8 * 8;
+            if (row < nrow && mm < g.M) {
+              __nv_bfloat16* dst = out_b + (size_t)(row0 + c0 + row) * g.ld_out + mm;
+              const __nv_bfloat16* src = stg_b + row * kBM + c8 * 8;
+              if (P.vec && mm + 7 < g.M) {
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+              } else {
+                for (int c = 0; c < 8 && mm + c < g.M; ++c) dst[c] = src[c];
+              }
+            }
+          }
+        }
+        named_barrier_sync(1, 128);  // the staging tile is reused by the next chunk
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);
@@ -315,6 +393,14 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, (uint32_t)P.tmem_cols);
+  }
+}
+
+static void set_smem_attr() {
+  static bool done = false;
+  if (!done) {
+    cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    done = true;
   }
 }
 
@@ -332,14 +418,17 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   P.tmem_cols = L.tmem_cols;
   P.n_mtiles = (g.M + kBM - 1) / kBM;
   P.n_ttiles = (g.mode == 0) ? (g.T + g.ntile - 1) / g.ntile : 0;
+  {
+    // 16-byte output vectors need aligned rows (and slices) in elements of the output type
+    const bool f32out = g.mode == 2 || g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32;
+    const int per_vec = f32out ? 4 : 8;
+    P.vec = ((uintptr_t)g.out % 16 == 0) && g.ld_out % per_vec == 0 &&
+            (g.ksplit <= 1 || g.split_stride % (size_t)per_vec == 0);
+  }
   const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles * (g.ksplit > 1 ? g.ksplit : 1)
                                   : g.n_work_max * P.n_mtiles;
   if (total <= 0) return 0;
-  static int attr_bytes = 0;
-  if (attr_bytes < L.smem_bytes) {
-    cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-    attr_bytes = kMaxSmem;
-  }
+  set_smem_attr();
   const int grid = std::min(total, num_sms * L.per_sm);
   gemm_tc_kernel<<<grid, kTcThreads, L.smem_bytes, s>>>(a0, a1, a2, b, P);
   return 0;

@@ -63,12 +63,93 @@ __global__ void router_topk_kernel(const float* __restrict__ glog, int nsplit, c
   }
 }
 
+// Vector form for E = 32 * EPL (EPL a multiple of 4): lane l owns experts
+// l*EPL .. l*EPL+EPL-1, read as float4.  The K slices are loaded a group at a
+// time (all loads of a group in flight together) and added in slice order,
+// so the sums equal the scalar kernel's.
+template <int EPL>
+__global__ void router_topk_vec_kernel(const float* __restrict__ glog, int nsplit, const float* __restrict__ bias,
+                                       int32_t* __restrict__ ids, float* __restrict__ wts, int n_tok, int k) {
+  constexpr int E = 32 * EPL, NV = EPL / 4, G = NV == 1 ? 8 : 4;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_tok) return;
+  const float4* g4 = reinterpret_cast<const float4*>(glog + (size_t)warp * E + lane * EPL);
+  const size_t slice4 = (size_t)n_tok * E / 4;
+  float v[EPL];
+#pragma unroll
+  for (int q = 0; q < NV; ++q) {
+    const float4 a = g4[q];
+    v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+  }
+  for (int sp0 = 1; sp0 < nsplit; sp0 += G) {
+    float4 a[G][NV];
+#pragma unroll
+    for (int u = 0; u < G; ++u)
+#pragma unroll
+      for (int q = 0; q < NV; ++q)
+        if (sp0 + u < nsplit) a[u][q] = g4[(size_t)(sp0 + u) * slice4 + q];
+#pragma unroll
+    for (int u = 0; u < G; ++u)
+#pragma unroll
+      for (int q = 0; q < NV; ++q)
+        if (sp0 + u < nsplit) {
+          v[4 * q] += a[u][q].x; v[4 * q + 1] += a[u][q].y; v[4 * q + 2] += a[u][q].z; v[4 * q + 3] += a[u][q].w;
+        }
+  }
+  if (bias) {
+    const float4* b4 = reinterpret_cast<const float4*>(bias + lane * EPL);
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      const float4 b = b4[q];
+      v[4 * q] += b.x; v[4 * q + 1] += b.y; v[4 * q + 2] += b.z; v[4 * q + 3] += b.w;
+    }
+  }
+  float sel_v[16];
+  int sel_i[16];
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (v[j] > bv) { bv = v[j]; bi = lane * EPL + j; }   // ascending ids: the first of equals wins
+    if (bi == 0x7fffffff) bi = lane * EPL;                  // all -inf: lowest own id
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    sel_v[r] = bv;
+    sel_i[r] = bi;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (lane * EPL + j == bi) v[j] = -INFINITY;
+  }
+  if (lane == 0) {
+    const float m = sel_v[0];
+    float s = 0.f;
+    for (int r = 0; r < k; ++r) s += expf(sel_v[r] - m);
+    for (int r = 0; r < k; ++r) {
+      ids[(size_t)warp * k + r] = sel_i[r];
+      wts[(size_t)warp * k + r] = expf(sel_v[r] - m) / s;
+    }
+  }
+}
+
 void launch_router_topk(const float* glog, int nsplit, const float* bias, int32_t* ids, float* wts, int n_tok,
                         int e, int k, cudaStream_t s) {
   if (n_tok <= 0) return;
   const int threads = 256;
   const int blocks = (n_tok * 32 + threads - 1) / threads;
-  router_topk_kernel<<<blocks, threads, 0, s>>>(glog, nsplit, bias, ids, wts, n_tok, e, k);
+  const bool vec = ((uintptr_t)glog & 15u) == 0 && (bias == nullptr || ((uintptr_t)bias & 15u) == 0);
+  if (vec && e == 128) {
+    router_topk_vec_kernel<4><<<blocks, threads, 0, s>>>(glog, nsplit, bias, ids, wts, n_tok, k);
+  } else if (vec && e == 256) {
+    router_topk_vec_kernel<8><<<blocks, threads, 0, s>>>(glog, nsplit, bias, ids, wts, n_tok, k);
+  } else {
+    router_topk_kernel<<<blocks, threads, 0, s>>>(glog, nsplit, bias, ids, wts, n_tok, e, k);
+  }
 }
 
 // Single-CTA counting sort.  Items i = t*k + s in order; inside an expert the

@@ -31,10 +31,17 @@ void launch_rmsnorm(const float* h, const float* w, T* xn, int n_tok, int d, flo
 template <typename T>
 void launch_combine(float* h, const float* y, const float* wts, int k, const float* norm_w, T* xn,
                     int n_tok, int d, float eps, cudaStream_t s);
-// Split fp32 q|k|v rows into rotated Q [B,Hq,nq,hd], K cache rows and transposed V cache rows.
+// h[t,:] += sum over s < nsplit (in order) of part[s*split_stride + t*d + :]; then
+// xn = rmsnorm(h, w).  Sums the K slices of a split-K projection into the residual.
 template <typename T>
-void launch_rope_scatter(const float* qkv, T* q, T* kc, T* vt, const float* rope_cs, const BatchInfo& bi,
-                         int nq, int hq, int hkv, int hd, int max_ctx, cudaStream_t s);
+void launch_add_rmsnorm(float* h, const float* part, int nsplit, size_t split_stride, const float* w, T* xn,
+                        int n_tok, int d, float eps, cudaStream_t s);
+// Split fp32 q|k|v rows into rotated Q [B,Hq,nq,hd], K cache rows and transposed V cache rows.
+// The rows are the sum of nsplit K slices qkv + s*split_stride (nsplit 1: qkv itself).
+template <typename T>
+void launch_rope_scatter(const float* qkv, int nsplit, size_t split_stride, T* q, T* kc, T* vt,
+                         const float* rope_cs, const BatchInfo& bi, int nq, int hq, int hkv, int hd, int max_ctx,
+                         cudaStream_t s);
 // xp[p,:] = xn[perm[p]/k,:] for p < n_rows
 template <typename T>
 void launch_gather_rows(const T* xn, const int32_t* perm, T* xp, int n_rows, int k, int d, cudaStream_t s);

@@ -13,7 +13,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdg.so")
+# DG_LIB selects another build of the library (default: the in-tree libdg.so)
+LIB_PATH = os.environ.get("DG_LIB") or os.path.join(_HERE, "libdg.so")
 
 DG_OK, DG_EINVAL, DG_ENOMEM, DG_ECUDA, DG_ECAPACITY, DG_ESTATE, DG_ETIMEOUT = range(7)
 DG_FP32, DG_BF16 = 0, 1
@@ -22,7 +23,7 @@ EXPORTS = (
     "dg_create", "dg_destroy", "dg_last_error", "dg_prefill_prompt", "dg_set_kv", "dg_set_length",
     "dg_get_length", "dg_denoise_step", "dg_sample", "dg_generate_block", "dg_generate_block_host",
     "dg_synchronize", "dg_launch_count", "dg_profile_enable", "dg_profile_read", "dg_profile_reset",
-    "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc",
+    "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc", "dg_selftest_gemm_split",
 )
 
 
@@ -102,6 +103,7 @@ def lib():
         L.dg_profile_reset.argtypes = [P]
         L.dg_selftest_philox.argtypes = [P, P, P, P, P, C.c_int]
         L.dg_selftest_gemm.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, P]
+        L.dg_selftest_gemm_split.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, P, C.c_int, C.POINTER(C.c_int)]
         L.dg_sample_noalloc.argtypes = [P, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_int), C.c_int,
                                         C.POINTER(DgSamplerParams), P, C.POINTER(DgStepOut), P, C.c_char_p,
                                         C.c_size_t]
@@ -301,3 +303,11 @@ def dg_selftest_philox(h: Handle, ctr, key, out, out_curand=None):
 def dg_selftest_gemm(h: Handle, x, w, out):
     """out[T, M] fp32 = x[T, K] @ w[M, K]^T through the tensor-core GEMM."""
     return h.check(lib().dg_selftest_gemm(h.ptr, _ptr(x), _ptr(w), x.shape[0], w.shape[0], x.shape[1], _ptr(out)))
+
+
+def dg_selftest_gemm_split(h: Handle, x, w, part):
+    """Split-K partial slices of x @ w.T into part [max_split, T, M]; returns the slice count."""
+    n = C.c_int()
+    h.check(lib().dg_selftest_gemm_split(h.ptr, _ptr(x), _ptr(w), x.shape[0], w.shape[0], x.shape[1], _ptr(part),
+                                         part.shape[0], C.byref(n)))
+    return n.value

@@ -324,6 +324,16 @@ int dg_selftest_philox(dg_handle* h, const uint32_t* ctr, const uint32_t* key, u
  */
 int dg_selftest_gemm(dg_handle* h, const void* x, const void* w, int T, int M, int K, float* out);
 
+/*
+ * Test hook: the split-K form the layers use for up to 256 tokens (QKV, O and
+ * self-conditioning projections).  Writes *nsplit (<= max_split) fp32 partial
+ * slices part[s][T][M], whose sum over s is x[T, K] * w[M, K]^T.  part holds
+ * max_split * T * M floats.  Same operand rules as dg_selftest_gemm;
+ * DG_EINVAL if T > 256.
+ */
+int dg_selftest_gemm_split(dg_handle* h, const void* x, const void* w, int T, int M, int K, float* part,
+                           int max_split, int* nsplit);
+
 #ifdef __cplusplus
 }
 #endif

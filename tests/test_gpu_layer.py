@@ -36,6 +36,30 @@ def test_tc_gemm_matches_float64_matmul(dg, T, Mr, K):
     h.close()
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,Mr,K", [(256, 8192, 2816), (256, 2816, 4096), (256, 2816, 2816), (37, 384, 192),
+                                    (130, 200, 2816), (1, 128, 64)])
+def test_split_k_gemm_slices_sum_to_float64_matmul(dg, T, Mr, K):
+    """The split-K form of the QKV / O / self-conditioning projections: its
+    slices, added in order, equal the product (several tiles, ragged M and T)."""
+    g = torch.Generator(device="cuda").manual_seed(T * 5 + Mr)
+    x = torch.randn((T, K), generator=g, device="cuda").to(torch.bfloat16)
+    w = (torch.randn((Mr, K), generator=g, device="cuda") * 0.05).to(torch.bfloat16)
+    part = torch.full((8, T, Mr), float("nan"), device="cuda")
+    h = dg.dg_create(dict(vocab=8, canvas=4), None, dtype="bf16", max_batch=1, max_ctx=64)
+    ns = dg.dg_selftest_gemm_split(h, x, w, part)
+    dg.dg_synchronize(h)
+    assert 1 <= ns <= 8
+    if (T, Mr, K) == (256, 2816, 4096):
+        assert ns > 1      # the O-projection shape splits K
+    assert not torch.isnan(part[:ns]).any()
+    got = part[:ns].double().sum(0)
+    ref = x.double().cpu() @ w.double().cpu().T
+    err = max_abs_rel(to_np(got), ref.numpy())
+    assert err < 1e-3, err
+    h.close()
+
+
 def _layer_setup(dg):
     w = synth.make_weights(M, seed=W["seed"], dtype="bf16", router_bias=True, device="cuda")
     k, v = synth.normal_kv(M["n_kv_heads"], W["cache_len"], M["head_dim"], seed=W["seed"] + 50, dtype="bf16",
