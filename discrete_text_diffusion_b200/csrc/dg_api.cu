@@ -113,9 +113,9 @@ static_assert(PC_EMBED == DG_PROF_EMBED && PC_DENSE == DG_PROF_DENSE_GEMM && PC_
 
 }  // namespace
 
-// A weight matrix's TMA maps for 2- and 4-chunk (64-column) boxes of 128 rows.
+// A weight matrix's TMA maps for 1-, 2- and 4-chunk (64-column) boxes of 128 rows.
 struct WMap {
-  CUtensorMap k2, k4;
+  CUtensorMap k1, k2, k4;
 };
 struct LayerMaps {
   WMap wq, wk, wv, wo, router, gate, up, down;
@@ -281,12 +281,19 @@ int pick_ntile(int n_mtiles, int T, int num_sms) {
   return nt;
 }
 
+#ifndef DG_MOE_DOWN_KSUB
+#define DG_MOE_DOWN_KSUB 2    // 64-column chunks per stage of the expert down projection
+#endif
+#ifndef DG_GROUPED_TILE
+#define DG_GROUPED_TILE 128   // rows of a tensor-core expert work item (64, 128 or 256)
+#endif
+// Rows of an expert's work item.  Each item loads a token box sized to its
+// rows (32 .. DG_GROUPED_TILE), so a small item does not pay for a large box.
+// Larger items stream an expert's weights fewer times but leave fewer items
+// to spread over the SMs when the routing concentrates on a few experts.
 int grouped_tile(const dg_handle* H, int T) {
-  if (!H->bf16) return 64;
-  // at most 128 rows: the gate + up weights and a 256-row token tile would
-  // not fit a two-stage pipeline with two-chunk TMA boxes
-  const double avg = (double)T * H->c.top_k / H->c.n_experts;
-  return avg > 48 ? 128 : 64;
+  (void)T;
+  return H->bf16 ? DG_GROUPED_TILE : 64;
 }
 
 // Pipeline shape of a tensor-core GEMM launch.  TMA throughput per CTA is
@@ -306,7 +313,7 @@ constexpr int kMaxDenseSplit = 8;      // K slices of the split-K dense projecti
 constexpr int kDenseSplitRows = 256;   // token rows up to which they take the split-K form
 int ctas_for(int ntile) { return ntile <= 64 ? DG_NARROW_CTAS : 1; }
 
-const CUtensorMap& pick(const WMap& w, int ksub) { return ksub == 4 ? w.k4 : w.k2; }
+const CUtensorMap& pick(const WMap& w, int ksub) { return ksub == 4 ? w.k4 : ksub == 1 ? w.k1 : w.k2; }
 
 // Token-operand map of a (rows x cols) activation buffer for a tile of ntile
 // rows and ksub chunks, built on first use and kept for the handle's life.
@@ -328,8 +335,20 @@ const CUtensorMap* bmap(dg_handle* H, const void* p, uint64_t cols, uint64_t row
 }
 
 void run_tc(dg_handle* H, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap* b,
-            TcGemm& g) {
-  if (!b || launch_gemm_tc(a0, a1, a2, *b, g, H->num_sms, H->stream) != 0) H->bad_launch = true;
+            TcGemm& g, const CUtensorMap* bsub = nullptr) {
+  if (!b || launch_gemm_tc(a0, a1, a2, *b, bsub, g, H->num_sms, H->stream) != 0) H->bad_launch = true;
+}
+
+// Token maps of a grouped GEMM's activation rows: boxes of 32, 64 and 128
+// rows (bsub) besides the ntile-row map, for work items with fewer rows.
+// Returns false when a map could not be built.
+bool grouped_bsub(dg_handle* H, const void* x, uint64_t cols, uint64_t rows, int ksub, CUtensorMap bsub[3]) {
+  for (int k = 0; k < 3; ++k) {
+    const CUtensorMap* m = bmap(H, x, cols, rows, 32 << k, ksub);
+    if (!m) return false;
+    bsub[k] = *m;
+  }
+  return true;
 }
 
 // ------------------------------------------------------------ GEMM helpers
@@ -499,11 +518,15 @@ void moe_gemms(dg_handle* H, int l, int T) {
       g.out = H->hb;
       g.ld_out = c.d_ff;
       g.err = H->d_err;
-      g.ksub = ksub_for(1, tile);
+      g.ksub = tile > 128 ? 1 : 2;   // stage = ksub x (gate + up + token box) must leave two stages
       g.ctas_per_sm = ctas_for(g.ntile);
       const LayerMaps& M = H->lmaps[l];
-      run_tc(H, pick(M.gate, g.ksub), pick(M.up, g.ksub), pick(M.up, g.ksub),
-             bmap(H, H->xp, c.d_model, rows, tile, g.ksub), g);
+      CUtensorMap bsub[3];
+      if (grouped_bsub(H, H->xp, c.d_model, rows, g.ksub, bsub))
+        run_tc(H, pick(M.gate, g.ksub), pick(M.up, g.ksub), pick(M.up, g.ksub),
+               bmap(H, H->xp, c.d_model, rows, tile, g.ksub), g, bsub);
+      else
+        H->bad_launch = true;
     }
   }
   {
@@ -526,10 +549,14 @@ void moe_gemms(dg_handle* H, int l, int T) {
       g.ld_out = c.d_model;
       g.row_map = H->perm;
       g.err = H->d_err;
-      g.ksub = ksub_for(2, tile);
+      g.ksub = DG_MOE_DOWN_KSUB;
       g.ctas_per_sm = ctas_for(g.ntile);
       const CUtensorMap& a = pick(H->lmaps[l].down, g.ksub);
-      run_tc(H, a, a, a, bmap(H, H->hb, c.d_ff, rows, tile, g.ksub), g);
+      CUtensorMap bsub[3];
+      if (grouped_bsub(H, H->hb, c.d_ff, rows, g.ksub, bsub))
+        run_tc(H, a, a, a, bmap(H, H->hb, c.d_ff, rows, tile, g.ksub), g, bsub);
+      else
+        H->bad_launch = true;
     }
   }
 }
@@ -546,12 +573,20 @@ void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
   a.causal = causal ? 1 : 0;
   a.bi = bi;
   if (H->attn_tc) {
-    // split the keys so that the grid covers the SMs about twice
+    // Split the keys: one CTA per SM, so the time is about waves x (key tiles
+    // per CTA + a fixed cost of ~2 tiles); each split adds partial-output
+    // traffic and combine work (charged half a tile).
     int max_len = 0;
     for (int b = 0; b < bi.B; ++b) max_len = std::max(max_len, bi.len[b] + nq);
     const int base = bi.B * c.n_heads * ((nq + 127) / 128);
     const int tiles = (max_len + 63) / 64;
-    int n_split = std::max(1, std::min({(2 * H->num_sms + base - 1) / base, 16, std::max(1, tiles / 4)}));
+    int n_split = 1;
+    double best = 1e30;
+    for (int n = 1; n <= std::min(16, std::max(1, tiles / 4)); ++n) {
+      const int waves = (base * n + H->num_sms - 1) / H->num_sms;
+      const double cost = waves * ((tiles + n - 1) / n + 2.0) + 0.5 * n;
+      if (cost < best - 1e-9) { best = cost; n_split = n; }
+    }
     if ((size_t)n_split * bi.B * c.n_heads * nq > H->part_rows_cap) n_split = 1;
     AttnTcArgs t{};
     t.a = a;
@@ -900,10 +935,12 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
         const dg_layer_weights& L = H->lw[l];
         LayerMaps& M = H->lmaps[l];
         auto dense = [&](WMap& w, const void* p, uint64_t cols, uint64_t rows) {
+          tm &= tmap_chunks(&w.k1, p, cols, rows, cols, 128, 1);
           tm &= tmap_chunks(&w.k2, p, cols, rows, cols, 128, 2);
           tm &= tmap_chunks(&w.k4, p, cols, rows, cols, 128, 4);
         };
         auto experts = [&](WMap& w, const void* p, uint64_t cols, uint64_t rows) {
+          tm &= tmap_chunks4(&w.k1, p, cols, rows, E, 128, 1);
           tm &= tmap_chunks4(&w.k2, p, cols, rows, E, 128, 2);
           tm &= tmap_chunks4(&w.k4, p, cols, rows, E, 128, 4);
         };
@@ -916,8 +953,10 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
         experts(M.up, L.w_up, d, F);
         experts(M.down, L.w_down, F, d);
       }
+      tm &= tmap_chunks(&H->m_embed.k1, H->embed, d, c.vocab, d, 128, 1);
       tm &= tmap_chunks(&H->m_embed.k2, H->embed, d, c.vocab, d, 128, 2);
       tm &= tmap_chunks(&H->m_embed.k4, H->embed, d, c.vocab, d, 128, 4);
+      tm &= tmap_chunks(&H->m_wsc.k1, H->w_sc, d, d, d, 128, 1);
       tm &= tmap_chunks(&H->m_wsc.k2, H->w_sc, d, d, d, 128, 2);
       tm &= tmap_chunks(&H->m_wsc.k4, H->w_sc, d, d, d, 128, 4);
       if (c.head_dim == 256) {
@@ -1193,7 +1232,7 @@ int dg_selftest_gemm(dg_handle* H, const void* x, const void* w, int T, int M, i
   if (!tmap_chunks(&mx, x, K, T, K, (uint32_t)g.ntile, (uint32_t)g.ksub) ||
       !tmap_chunks(&mw, w, K, M, K, 128, (uint32_t)g.ksub))
     return fail(H, DG_ECUDA, "tensor map encode failed");
-  if (launch_gemm_tc(mw, mw, mw, mx, g, H->num_sms, H->stream) != 0)
+  if (launch_gemm_tc(mw, mw, mw, mx, nullptr, g, H->num_sms, H->stream) != 0)
     return fail(H, DG_EINVAL, "GEMM tiling rejected");
   H->launches += 1;
   return check_launch(H, "selftest gemm");

@@ -343,7 +343,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-// Merge the split partials of one (b, h, query) row: one warp per row.
+// Merge the split partials of one (b, h, query) row: one warp per row, lane
+// l owning columns [8l, 8l + 8) (two 16-byte loads per split, one 16-byte
+// store).  The loads of all splits are independent and issued together.  A
+// split that saw no key (max -inf) contributes nothing, whatever its O holds.
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                     __nv_bfloat16* __restrict__ out, int n_split, int B, int hq, int nq) {
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -354,26 +357,35 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   float M = -INFINITY;
   for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[2 * (s * stride + row)]);
   float L = 0.f;
-  float acc[8];
-#pragma unroll
-  for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+  float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll 4
   for (int s = 0; s < n_split; ++s) {
     const float ms = part_ml[2 * (s * stride + row)];
-    if (ms == -INFINITY) continue;
-    const float w = exp2f(ms - M);
-    L += part_ml[2 * (s * stride + row) + 1] * w;
-    const float* po = part_o + (s * stride + row) * kHd;
-#pragma unroll
-    for (int x = 0; x < 8; ++x) acc[x] += w * po[lane + 32 * x];
+    const float ls = part_ml[2 * (s * stride + row) + 1];
+    const float4* po = reinterpret_cast<const float4*>(part_o + (s * stride + row) * kHd) + 2 * lane;
+    const float4 v0 = po[0], v1 = po[1];
+    const bool live = ms != -INFINITY;
+    const float w = live ? exp2f(ms - M) : 0.f;
+    if (live) {
+      L += ls * w;
+      a0.x += w * v0.x; a0.y += w * v0.y; a0.z += w * v0.z; a0.w += w * v0.w;
+      a1.x += w * v1.x; a1.y += w * v1.y; a1.z += w * v1.z; a1.w += w * v1.w;
+    }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   // row = (b*hq + h)*nq + q  ->  out[(b*nq + q), h*hd + d]
   const int q = row % nq;
   const int bh = row / nq;
   const int h = bh % hq, b = bh / hq;
-  __nv_bfloat16* op = out + ((size_t)b * nq + q) * ((size_t)hq * kHd) + (size_t)h * kHd;
-#pragma unroll
-  for (int x = 0; x < 8; ++x) op[lane + 32 * x] = __float2bfloat16_rn(acc[x] * inv);
+  __nv_bfloat16* op = out + ((size_t)b * nq + q) * ((size_t)hq * kHd) + (size_t)h * kHd + 8 * lane;
+  const __nv_bfloat162 p0 = __floats2bfloat162_rn(a0.x * inv, a0.y * inv), p1 = __floats2bfloat162_rn(a0.z * inv, a0.w * inv);
+  const __nv_bfloat162 p2 = __floats2bfloat162_rn(a1.x * inv, a1.y * inv), p3 = __floats2bfloat162_rn(a1.z * inv, a1.w * inv);
+  uint4 u;
+  u.x = *reinterpret_cast<const uint32_t*>(&p0);
+  u.y = *reinterpret_cast<const uint32_t*>(&p1);
+  u.z = *reinterpret_cast<const uint32_t*>(&p2);
+  u.w = *reinterpret_cast<const uint32_t*>(&p3);
+  *reinterpret_cast<uint4*>(op) = u;
 }
 
 size_t attn_tc_partial_floats(int n_split, int B, int hq, int nq_pad, int hd) {

@@ -49,8 +49,8 @@ constexpr int kMaxSmem = 232448;        // 227 KB opt-in limit per CTA
 #endif
 constexpr int kSmemPerSm = 233472;      // 228 KB of shared memory per SM
 #ifndef DG_EPI_STAGE_MODES
-#define DG_EPI_STAGE_MODES 1            // bit m: mode m writes its output through the staging tile (dense only:
-                                        // the grouped kernels measured no gain or a loss)
+#define DG_EPI_STAGE_MODES 5            // bit m: mode m writes its output through the staging tile (dense and
+                                        // expert down; the bf16 gate/up output measured a loss)
 #endif
 constexpr int kEpiRows = 32;            // token rows per epilogue chunk
 constexpr int kEpiBytes = kEpiRows * kBM * 4;  // staging tile of one chunk (fp32) = 16 KB
@@ -101,8 +101,19 @@ int gemm_tc_smem_bytes(const TcGemm& p, int* stages) {
 struct TcKParams {
   TcGemm g;
   int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, n_ttiles, ksub;
-  int vec;   // output rows may be written as aligned 16-byte vectors
+  int vec;         // output rows may be written as aligned 16-byte vectors
+  int box_levels;  // grouped modes: token maps tbs[k] with boxes of 32 << k rows (< ntile) exist for k < box_levels
 };
+
+// Token box of a work item: grouped modes load only as many rows as the item
+// has (a box of 32, 64, 128, ... rows, at most ntile); dense mode always ntile.
+__device__ __forceinline__ int item_box(const TcKParams& P, int rows, int* level) {
+  int k = 0;
+  if (P.g.mode != 0)
+    while (k < P.box_levels && (32 << k) < rows) ++k;
+  *level = k;
+  return k < P.box_levels ? (32 << k) : P.g.ntile;
+}
 
 // Work item -> weight tile, token rows and (dense split-K) the range of K
 // stages [j0, j1) with its split index ks.
@@ -135,7 +146,8 @@ __device__ __forceinline__ void tc_item(const TcKParams& P, int item, int nst, i
 __global__ void __launch_bounds__(kTcThreads, 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap ta1,
                    const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb,
-                   const TcKParams P) {
+                   const __grid_constant__ CUtensorMap tbs0, const __grid_constant__ CUtensorMap tbs1,
+                   const __grid_constant__ CUtensorMap tbs2, const TcKParams P) {
   extern __shared__ uint8_t smem_raw[];
   const TcGemm& g = P.g;
   const uint32_t raw = smem_u32(smem_raw);
@@ -176,7 +188,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   const int ksub = P.ksub;                        // K blocks per pipeline stage
   const int nst = (nk + ksub - 1) / ksub;         // stages per output tile
   const int n_a = (g.mode == 1) ? 2 : 1;
-  const int b_sub = g.ntile * kBK * 2;            // bytes of one token sub-tile
   // stage layout: [ksub x A0][ksub x A1 (mode 1)][ksub x B], each sub 1024-aligned
 
   if (warp == 0 && lane == 0) {
@@ -186,11 +197,14 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     // the token map a (64, rows, K/64) view with a box of ntile rows x ksub
     // chunks.  A stage always receives whole boxes (chunks past K, rows past
     // the matrix are zero-filled), so the byte count is fixed.
-    const uint32_t tx = (uint32_t)(ksub * (n_a * kABytes + b_sub));
     uint32_t kiter = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
       int m0, e, row0, rows, j0, j1, ks;
       tc_item(P, item, nst, m0, e, row0, rows, j0, j1, ks);
+      int lvl;
+      const int box = item_box(P, rows, &lvl);
+      const CUtensorMap* bm = box == g.ntile ? &tb : (lvl == 0 ? &tbs0 : lvl == 1 ? &tbs1 : &tbs2);
+      const uint32_t tx = (uint32_t)(ksub * (n_a * kABytes + box * kBK * 2));
       const CUtensorMap* am = &ta0;
       int am0 = m0;
       if (g.mode == 0) {
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           tma_load_4d(st, &ta0, &full[s], 0, m0, kb0, e);
           if (g.mode == 1) tma_load_4d(st + ksub * kABytes, &ta1, &full[s], 0, m0, kb0, e);
         }
-        tma_load_3d(st + n_a * ksub * kABytes, &tb, &full[s], 0, row0, kb0);
+        tma_load_3d(st + n_a * ksub * kABytes, bm, &full[s], 0, row0, kb0);
       }
       if (!ok) break;
     }
@@ -225,6 +239,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       tc_item(P, item, nst, m0, e, row0, rows, j0, j1, ks);
       const int n_mma = (rows + 15) & ~15;
       const uint32_t idesc = idesc_bf16(kBM, n_mma);
+      int lvl;
+      const int bsub = item_box(P, rows, &lvl) * kBK * 2;  // bytes of one token chunk in this item's box
       const int ab = it % P.n_acc_buf;
       const uint32_t use = (uint32_t)(it / P.n_acc_buf);
       if (!mbar_wait(&acc_empty[ab], (use & 1u) ^ 1u, err, kErrTimeoutMma)) break;
@@ -240,7 +256,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         for (int u = 0; u < nsub; ++u) {
           const uint32_t sa = st + (uint32_t)(u * kABytes);
           const uint32_t sa1 = st + (uint32_t)((ksub + u) * kABytes);
-          const uint32_t sb = st + (uint32_t)(n_a * ksub * kABytes + u * b_sub);
+          const uint32_t sb = st + (uint32_t)(n_a * ksub * kABytes + u * bsub);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t bdesc = sdesc_k_sw128(sb + 32u * k);
@@ -405,7 +421,7 @@ static void set_smem_attr() {
 }
 
 int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
-                   const TcGemm& g, int num_sms, cudaStream_t s) {
+                   const CUtensorMap* bsub, const TcGemm& g, int num_sms, cudaStream_t s) {
   const TcLayout L = tc_layout(g);
   if (L.stages < 2) return -1;   // the tile does not fit a two-stage pipeline
   TcKParams P;
@@ -418,6 +434,9 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   P.tmem_cols = L.tmem_cols;
   P.n_mtiles = (g.M + kBM - 1) / kBM;
   P.n_ttiles = (g.mode == 0) ? (g.T + g.ntile - 1) / g.ntile : 0;
+  P.box_levels = 0;
+  if (g.mode != 0 && bsub)
+    while (P.box_levels < 3 && (32 << P.box_levels) < g.ntile) ++P.box_levels;
   {
     // 16-byte output vectors need aligned rows (and slices) in elements of the output type
     const bool f32out = g.mode == 2 || g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32;
@@ -430,7 +449,10 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   if (total <= 0) return 0;
   set_smem_attr();
   const int grid = std::min(total, num_sms * L.per_sm);
-  gemm_tc_kernel<<<grid, kTcThreads, L.smem_bytes, s>>>(a0, a1, a2, b, P);
+  const CUtensorMap& s0 = P.box_levels > 0 ? bsub[0] : b;
+  const CUtensorMap& s1 = P.box_levels > 1 ? bsub[1] : b;
+  const CUtensorMap& s2 = P.box_levels > 2 ? bsub[2] : b;
+  gemm_tc_kernel<<<grid, kTcThreads, L.smem_bytes, s>>>(a0, a1, a2, b, s0, s1, s2, P);
   return 0;
 }
 

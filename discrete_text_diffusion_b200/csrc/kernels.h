@@ -124,8 +124,11 @@ struct TcGemm {
   size_t split_stride;
 };
 // Returns 0, or -1 when the tile does not fit a two-stage pipeline (nothing launched).
+// b: token map with boxes of ntile rows.  bsub (grouped modes, or NULL): maps of the
+// same tokens with boxes of 32, 64, 128 rows (those below ntile), used for work
+// items with fewer rows.
 int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
-                   const TcGemm& p, int num_sms, cudaStream_t s);
+                   const CUtensorMap* bsub, const TcGemm& p, int num_sms, cudaStream_t s);
 int gemm_tc_smem_bytes(const TcGemm& p, int* stages);
 
 // ---- attention

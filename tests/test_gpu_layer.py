@@ -60,8 +60,12 @@ def test_split_k_gemm_slices_sum_to_float64_matmul(dg, T, Mr, K):
     h.close()
 
 
-def _layer_setup(dg):
+def _layer_setup(dg, hot_experts=0):
     w = synth.make_weights(M, seed=W["seed"], dtype="bf16", router_bias=True, device="cuda")
+    if hot_experts:
+        # a large bias on a few experts routes every token to them: expert work
+        # items of 256 rows next to items of a few rows
+        w["layers"][0]["router_b"][:hot_experts] += 8.0
     k, v = synth.normal_kv(M["n_kv_heads"], W["cache_len"], M["head_dim"], seed=W["seed"] + 50, dtype="bf16",
                            device="cuda")
     h = dg.dg_create(M, w, dtype="bf16", max_batch=1, max_ctx=W["cache_len"] + M["canvas"])
@@ -73,8 +77,9 @@ def _layer_setup(dg):
 
 
 @pytest.mark.gpu
-def test_full_width_layer_step(dg):
-    w, h, om = _layer_setup(dg)
+@pytest.mark.parametrize("hot_experts", [0, 4])
+def test_full_width_layer_step(dg, hot_experts):
+    w, h, om = _layer_setup(dg, hot_experts)
     n, vocab, d = M["canvas"], M["vocab"], M["d_model"]
     canvas = synth.uniform_tokens(n, vocab, seed=W["seed"] + 1)
     prev = synth.uniform_tokens(n, vocab, seed=W["seed"] + 2)
@@ -106,4 +111,6 @@ def test_full_width_layer_step(dg):
         err_l = max_abs_rel(to_np(logits)[0][r], ref_l)
         assert err_l < TOL_BF16, f"logits max-abs-rel {err_l}"
         assert 1 <= int(touched.item()) <= M["n_experts"]
+        if hot_experts:
+            assert (tr["router_ids"] < hot_experts).sum(1).min() == hot_experts
     h.close()
