@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (ntiles == 0) {
     // empty split (causal tail): contributes nothing to the combine
+    pdl_wait();
+    pdl_trigger();
     if (warp >= 2 && warp < 6) {
       const int r = (warp & 3) * 32 + lane;
       const int qi = q0 + r;
@@ -123,6 +125,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the set-up above touches no global memory: it overlaps the previous kernel
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tS = tmem;          // two score buffers: columns [0, 64), [64, 128)
   const uint32_t tO = tmem + 256;    // output accumulator: columns [256, 512)
 
@@ -349,6 +354,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // split that saw no key (max -inf) contributes nothing, whatever its O holds.
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                     __nv_bfloat16* __restrict__ out, int n_split, int B, int hq, int nq) {
+  pdl_wait();
+  pdl_trigger();
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int rows = B * hq * nq;
@@ -406,10 +413,10 @@ void launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
   P.n_qtiles = (a.nq + kQTile - 1) / kQTile;
   P.scale_log2 = 1.4426950408889634f / sqrtf((float)a.hd);
   dim3 grid(P.n_qtiles * t.n_split, a.hq, a.B);
-  attn_tc_kernel<<<grid, kAttnThreads, kAttnSmem, s>>>(tq, tk, tv, out, P);
+  launch_k(attn_tc_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmem, s, tq, tk, tv, out, P);
   if (t.n_split > 1) {
     const int rows = a.B * a.hq * a.nq;
-    attn_combine_kernel<<<(rows * 32 + 255) / 256, 256, 0, s>>>(t.part_o, t.part_ml, out, t.n_split, a.B, a.hq,
+    launch_k(attn_combine_kernel, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, t.part_o, t.part_ml, out, t.n_split, a.B, a.hq,
                                                                  a.nq);
   }
 }

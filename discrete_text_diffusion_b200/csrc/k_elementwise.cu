@@ -26,6 +26,8 @@ template <typename T>
 __global__ void embed_kernel(const int32_t* __restrict__ tok, const int32_t* __restrict__ prev,
                              const T* __restrict__ embed, float* __restrict__ h, T* __restrict__ eprev, int d,
                              int vocab, int* err) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const T* e = embed + (size_t)checked_token(tok[t], vocab, err) * d;
   float* ho = h + (size_t)t * d;
@@ -41,7 +43,7 @@ template <typename T>
 void launch_embed(const int32_t* tok, const int32_t* prev, const T* embed, float* h, T* eprev, int n_tok, int d,
                   int vocab, int* err, cudaStream_t s) {
   if (n_tok <= 0) return;
-  embed_kernel<T><<<n_tok, 256, 0, s>>>(tok, prev, embed, h, eprev, d, vocab, err);
+  launch_k(embed_kernel<T>, dim3(n_tok), dim3(256), 0, s, tok, prev, embed, h, eprev, d, vocab, err);
 }
 
 // ------------------------------------------------------------ block reduce
@@ -84,6 +86,8 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* o, int j4, 
 template <typename T>
 __global__ void rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ w, T* __restrict__ xn,
                                int d, float eps) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   const int t = blockIdx.x;
   const float* x = h + (size_t)t * d;
@@ -129,6 +133,8 @@ template <typename T, int VPT>
 __global__ void __launch_bounds__(kRowThreadsMax) rmsnorm_reg_kernel(const float* __restrict__ h,
                                                                      const float* __restrict__ w,
                                                                      T* __restrict__ xn, int d, float eps) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   const int t = blockIdx.x, d4 = d >> 2;
   const float4* x4 = reinterpret_cast<const float4*>(h + (size_t)t * d);
@@ -160,11 +166,11 @@ void launch_rmsnorm(const float* h, const float* w, T* xn, int n_tok, int d, flo
   const int vpt = row_vpt(d);
   const int thr = vpt ? row_threads(d / 4, vpt) : 256;
   switch (vpt) {
-    case 1: rmsnorm_reg_kernel<T, 1><<<n_tok, thr, 0, s>>>(h, w, xn, d, eps); break;
-    case 2: rmsnorm_reg_kernel<T, 2><<<n_tok, thr, 0, s>>>(h, w, xn, d, eps); break;
-    case 4: rmsnorm_reg_kernel<T, 4><<<n_tok, thr, 0, s>>>(h, w, xn, d, eps); break;
-    case 8: rmsnorm_reg_kernel<T, 8><<<n_tok, thr, 0, s>>>(h, w, xn, d, eps); break;
-    default: rmsnorm_kernel<T><<<n_tok, 256, 0, s>>>(h, w, xn, d, eps);
+    case 1: launch_k(rmsnorm_reg_kernel<T, 1>, dim3(n_tok), dim3(thr), 0, s, h, w, xn, d, eps); break;
+    case 2: launch_k(rmsnorm_reg_kernel<T, 2>, dim3(n_tok), dim3(thr), 0, s, h, w, xn, d, eps); break;
+    case 4: launch_k(rmsnorm_reg_kernel<T, 4>, dim3(n_tok), dim3(thr), 0, s, h, w, xn, d, eps); break;
+    case 8: launch_k(rmsnorm_reg_kernel<T, 8>, dim3(n_tok), dim3(thr), 0, s, h, w, xn, d, eps); break;
+    default: launch_k(rmsnorm_kernel<T>, dim3(n_tok), dim3(256), 0, s, h, w, xn, d, eps);
   }
 }
 
@@ -177,6 +183,8 @@ __global__ void __launch_bounds__(kRowThreadsMax) add_rmsnorm_kernel(float* __re
                                                                      size_t split_stride,
                                                                      const float* __restrict__ w,
                                                                      T* __restrict__ xn, int d, float eps) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   const int t = blockIdx.x;
   float* hr = h + (size_t)t * d;
@@ -243,11 +251,11 @@ void launch_add_rmsnorm(float* h, const float* part, int nsplit, size_t split_st
   const int vpt = (split_stride % 4 == 0) ? row_vpt(d) : 0;
   const int thr = vpt ? row_threads(d / 4, vpt) : 256;
   switch (vpt) {
-    case 1: add_rmsnorm_kernel<T, 1><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps); break;
-    case 2: add_rmsnorm_kernel<T, 2><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps); break;
-    case 4: add_rmsnorm_kernel<T, 4><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps); break;
-    case 8: add_rmsnorm_kernel<T, 8><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps); break;
-    default: add_rmsnorm_kernel<T, 0><<<n_tok, thr, 0, s>>>(h, part, nsplit, split_stride, w, xn, d, eps);
+    case 1: launch_k(add_rmsnorm_kernel<T, 1>, dim3(n_tok), dim3(thr), 0, s, h, part, nsplit, split_stride, w, xn, d, eps); break;
+    case 2: launch_k(add_rmsnorm_kernel<T, 2>, dim3(n_tok), dim3(thr), 0, s, h, part, nsplit, split_stride, w, xn, d, eps); break;
+    case 4: launch_k(add_rmsnorm_kernel<T, 4>, dim3(n_tok), dim3(thr), 0, s, h, part, nsplit, split_stride, w, xn, d, eps); break;
+    case 8: launch_k(add_rmsnorm_kernel<T, 8>, dim3(n_tok), dim3(thr), 0, s, h, part, nsplit, split_stride, w, xn, d, eps); break;
+    default: launch_k(add_rmsnorm_kernel<T, 0>, dim3(n_tok), dim3(thr), 0, s, h, part, nsplit, split_stride, w, xn, d, eps);
   }
 }
 
@@ -259,6 +267,8 @@ void launch_add_rmsnorm(float* h, const float* part, int nsplit, size_t split_st
 template <typename T>
 __global__ void combine_kernel(float* __restrict__ h, const float* __restrict__ y, const float* __restrict__ wts,
                                int k, const float* __restrict__ norm_w, T* __restrict__ xn, int d, float eps) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   __shared__ float ws[16];
   const int t = blockIdx.x;
@@ -324,6 +334,8 @@ __global__ void __launch_bounds__(kRowThreadsMax) combine_reg_kernel(float* __re
                                                                      const float* __restrict__ wts, int k,
                                                                      const float* __restrict__ norm_w,
                                                                      T* __restrict__ xn, int d, float eps) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[32];
   __shared__ float ws[16];
   const int t = blockIdx.x, d4 = d >> 2;
@@ -383,11 +395,11 @@ void launch_combine(float* h, const float* y, const float* wts, int k, const flo
   const int vpt = k <= 16 ? row_vpt(d) : 0;
   const int thr = vpt ? row_threads(d / 4, vpt) : 256;
   switch (vpt) {
-    case 1: combine_reg_kernel<T, 1><<<n_tok, thr, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps); break;
-    case 2: combine_reg_kernel<T, 2><<<n_tok, thr, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps); break;
-    case 4: combine_reg_kernel<T, 4><<<n_tok, thr, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps); break;
-    case 8: combine_reg_kernel<T, 8><<<n_tok, thr, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps); break;
-    default: combine_kernel<T><<<n_tok, 256, 0, s>>>(h, y, wts, k, norm_w, xn, d, eps);
+    case 1: launch_k(combine_reg_kernel<T, 1>, dim3(n_tok), dim3(thr), 0, s, h, y, wts, k, norm_w, xn, d, eps); break;
+    case 2: launch_k(combine_reg_kernel<T, 2>, dim3(n_tok), dim3(thr), 0, s, h, y, wts, k, norm_w, xn, d, eps); break;
+    case 4: launch_k(combine_reg_kernel<T, 4>, dim3(n_tok), dim3(thr), 0, s, h, y, wts, k, norm_w, xn, d, eps); break;
+    case 8: launch_k(combine_reg_kernel<T, 8>, dim3(n_tok), dim3(thr), 0, s, h, y, wts, k, norm_w, xn, d, eps); break;
+    default: launch_k(combine_kernel<T>, dim3(n_tok), dim3(256), 0, s, h, y, wts, k, norm_w, xn, d, eps);
   }
 }
 
@@ -400,6 +412,8 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int nsplit, s
                                     T* __restrict__ q, T* __restrict__ kc,
                                     T* __restrict__ vt, const float2* __restrict__ rope_cs, BatchInfo bi, int nq,
                                     int hq, int hkv, int hd, int max_ctx) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;            // token row b*nq + i
   const int head = blockIdx.y;         // 0..hq+2hkv-1
   const int b = t / nq, i = t - b * nq;
@@ -449,6 +463,8 @@ __global__ void __launch_bounds__(256) rope_scatter_tiled_kernel(const float* __
                                                                  const float2* __restrict__ rope_cs, BatchInfo bi,
                                                                  int nq, int n_tok, int hq, int hkv, int hd,
                                                                  int max_ctx) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char rope_smem[];
   const int t0 = blockIdx.x * kRopeTok;
   const int head = blockIdx.y;
@@ -524,13 +540,13 @@ void launch_rope_scatter(const float* qkv, int nsplit, size_t split_stride, T* q
   if (hd % 8 == 0) {
     dim3 grid((n_tok + kRopeTok - 1) / kRopeTok, hq + 2 * hkv);
     const size_t smem = (size_t)kRopeTok * (hd + 2) * sizeof(T);
-    rope_scatter_tiled_kernel<T><<<grid, 256, smem, s>>>(qkv, nsplit, split_stride, q, kc, vt,
+    launch_k(rope_scatter_tiled_kernel<T>, dim3(grid), dim3(256), smem, s, qkv, nsplit, split_stride, q, kc, vt,
                                                          reinterpret_cast<const float2*>(rope_cs), bi, nq, n_tok,
                                                          hq, hkv, hd, max_ctx);
     return;
   }
   dim3 grid(n_tok, hq + 2 * hkv);
-  rope_scatter_kernel<T><<<grid, 128, 0, s>>>(qkv, nsplit, split_stride, q, kc, vt,
+  launch_k(rope_scatter_kernel<T>, dim3(grid), dim3(128), 0, s, qkv, nsplit, split_stride, q, kc, vt,
                                               reinterpret_cast<const float2*>(rope_cs), bi, nq, hq, hkv, hd, max_ctx);
 }
 
@@ -538,6 +554,8 @@ void launch_rope_scatter(const float* qkv, int nsplit, size_t split_stride, T* q
 template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ xn, const int32_t* __restrict__ perm, T* __restrict__ xp,
                                    int k, int d) {
+  pdl_wait();
+  pdl_trigger();
   const int p = blockIdx.x;
   const int src = perm[p] / k;
   // 16-byte vectors when the row is 16-byte aligned (d * sizeof(T) % 16 == 0)
@@ -554,13 +572,15 @@ __global__ void gather_rows_kernel(const T* __restrict__ xn, const int32_t* __re
 template <typename T>
 void launch_gather_rows(const T* xn, const int32_t* perm, T* xp, int n_rows, int k, int d, cudaStream_t s) {
   if (n_rows <= 0) return;
-  gather_rows_kernel<T><<<n_rows, 128, 0, s>>>(xn, perm, xp, k, d);
+  launch_k(gather_rows_kernel<T>, dim3(n_rows), dim3(128), 0, s, xn, perm, xp, k, d);
 }
 
 // ------------------------------------------------------------ init canvas
 // [P1 一], [P2 运作机制]: the canvas starts as uniform-random vocabulary tokens.
 __global__ void init_canvas_kernel(int32_t* canvas, BatchInfo bi, const int* req_ids, int n, int vocab,
                                    uint64_t seed, uint32_t block) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const int req = bi.slot[b];
   (void)req_ids;
@@ -573,13 +593,15 @@ __global__ void init_canvas_kernel(int32_t* canvas, BatchInfo bi, const int* req
 void launch_init_canvas(int32_t* canvas, const BatchInfo& bi, const int* req_ids, int n, int vocab, uint64_t seed,
                         uint32_t block, cudaStream_t s) {
   if (bi.B <= 0) return;
-  init_canvas_kernel<<<bi.B, 256, 0, s>>>(canvas, bi, req_ids, n, vocab, seed, block);
+  launch_k(init_canvas_kernel, dim3(bi.B), dim3(256), 0, s, canvas, bi, req_ids, n, vocab, seed, block);
 }
 
 // ----------------------------------------------------------------- set_kv
 template <typename T>
 __global__ void set_kv_kernel(const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ kc,
                               T* __restrict__ vt, int n, int hd, int max_ctx) {
+  pdl_wait();
+  pdl_trigger();
   const int g = blockIdx.y;
   const int p = blockIdx.x;
   for (int j = threadIdx.x; j < hd; j += blockDim.x) {
@@ -591,7 +613,7 @@ __global__ void set_kv_kernel(const T* __restrict__ k, const T* __restrict__ v, 
 template <typename T>
 void launch_set_kv(const T* k, const T* v, T* kc, T* vt, int hkv, int n, int hd, int max_ctx, cudaStream_t s) {
   if (n <= 0) return;
-  set_kv_kernel<T><<<dim3(n, hkv), 128, 0, s>>>(k, v, kc, vt, n, hd, max_ctx);
+  launch_k(set_kv_kernel<T>, dim3(dim3(n, hkv)), dim3(128), 0, s, k, v, kc, vt, n, hd, max_ctx);
 }
 
 // ------------------------------------------------------------ instantiation

@@ -181,6 +181,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the set-up above touches no global memory: it overlaps the previous kernel
+  pdl_wait();
+  pdl_trigger();
 
   const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles * (g.ksplit > 1 ? g.ksplit : 1)
                                   : (*g.n_work) * P.n_mtiles;
@@ -452,7 +455,7 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   const CUtensorMap& s0 = P.box_levels > 0 ? bsub[0] : b;
   const CUtensorMap& s1 = P.box_levels > 1 ? bsub[1] : b;
   const CUtensorMap& s2 = P.box_levels > 2 ? bsub[2] : b;
-  gemm_tc_kernel<<<grid, kTcThreads, L.smem_bytes, s>>>(a0, a1, a2, b, s0, s1, s2, P);
+  launch_k(gemm_tc_kernel, dim3(grid), dim3(kTcThreads), L.smem_bytes, s, a0, a1, a2, b, s0, s1, s2, P);
   return 0;
 }
 

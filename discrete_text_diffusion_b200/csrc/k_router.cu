@@ -12,6 +12,8 @@ namespace dg {
 // arg-max with (value desc, id asc) ordering pick the top-k.
 __global__ void router_topk_kernel(const float* __restrict__ glog, int nsplit, const float* __restrict__ bias,
                                    int32_t* __restrict__ ids, float* __restrict__ wts, int n_tok, int e, int k) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_tok) return;
@@ -70,6 +72,8 @@ __global__ void router_topk_kernel(const float* __restrict__ glog, int nsplit, c
 template <int EPL>
 __global__ void router_topk_vec_kernel(const float* __restrict__ glog, int nsplit, const float* __restrict__ bias,
                                        int32_t* __restrict__ ids, float* __restrict__ wts, int n_tok, int k) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int E = 32 * EPL, NV = EPL / 4, G = NV == 1 ? 8 : 4;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -144,11 +148,11 @@ void launch_router_topk(const float* glog, int nsplit, const float* bias, int32_
   const int blocks = (n_tok * 32 + threads - 1) / threads;
   const bool vec = ((uintptr_t)glog & 15u) == 0 && (bias == nullptr || ((uintptr_t)bias & 15u) == 0);
   if (vec && e == 128) {
-    router_topk_vec_kernel<4><<<blocks, threads, 0, s>>>(glog, nsplit, bias, ids, wts, n_tok, k);
+    launch_k(router_topk_vec_kernel<4>, dim3(blocks), dim3(threads), 0, s, glog, nsplit, bias, ids, wts, n_tok, k);
   } else if (vec && e == 256) {
-    router_topk_vec_kernel<8><<<blocks, threads, 0, s>>>(glog, nsplit, bias, ids, wts, n_tok, k);
+    launch_k(router_topk_vec_kernel<8>, dim3(blocks), dim3(threads), 0, s, glog, nsplit, bias, ids, wts, n_tok, k);
   } else {
-    router_topk_kernel<<<blocks, threads, 0, s>>>(glog, nsplit, bias, ids, wts, n_tok, e, k);
+    launch_k(router_topk_kernel, dim3(blocks), dim3(threads), 0, s, glog, nsplit, bias, ids, wts, n_tok, e, k);
   }
 }
 
@@ -161,6 +165,8 @@ __global__ void __launch_bounds__(1024) router_permute_kernel(const int32_t* __r
                                                              int32_t* __restrict__ perm, int32_t* __restrict__ work,
                                                              int32_t* __restrict__ n_work,
                                                              int32_t* __restrict__ touched) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int cnt[256];
   __shared__ int off[257];
   __shared__ int running[256];
@@ -218,7 +224,7 @@ __global__ void __launch_bounds__(1024) router_permute_kernel(const int32_t* __r
 
 void launch_router_permute(const int32_t* ids, int n_items, int e, int tile, int32_t* cnt, int32_t* off,
                            int32_t* perm, int32_t* work, int32_t* n_work, int32_t* touched, cudaStream_t s) {
-  router_permute_kernel<<<1, 1024, 0, s>>>(ids, n_items, e, tile, cnt, off, perm, work, n_work, touched);
+  launch_k(router_permute_kernel, dim3(1), dim3(1024), 0, s, ids, n_items, e, tile, cnt, off, perm, work, n_work, touched);
 }
 
 }  // namespace dg

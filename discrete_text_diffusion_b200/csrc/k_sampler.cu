@@ -71,6 +71,8 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 // of 262144-term sums.
 __global__ void __launch_bounds__(kThreads) sampler_pass1(const float* __restrict__ logits, int vocab, float scale,
                                                           int argmax_mode, Partial* __restrict__ part) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red_m[kThreads / 32];
   __shared__ double red_s[kThreads / 32];
   __shared__ double red_a[kThreads / 32];
@@ -142,6 +144,8 @@ __global__ void __launch_bounds__(kThreads) sampler_pass2(const float* __restric
                                                           uint64_t seed, uint32_t step, uint32_t block,
                                                           const Partial* __restrict__ part, int32_t* __restrict__ x_hat,
                                                           float* __restrict__ pmax, float* __restrict__ ent) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sh_M;
   __shared__ double sh_target, sh_P0;
   __shared__ int sh_c;
@@ -253,8 +257,8 @@ void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const 
   const int argmax_mode = a.temperature == 0.f;
   const float scale = argmax_mode ? a.logit_scale : a.logit_scale / a.temperature;
   Partial* part = reinterpret_cast<Partial*>(ws);
-  sampler_pass1<<<dim3(n_chunks, rows), kThreads, 0, s>>>(logits, vocab, scale, argmax_mode, part);
-  sampler_pass2<<<rows, kThreads, 0, s>>>(logits, n, vocab, scale, argmax_mode, req_ids, a.seed, a.step, a.block,
+  launch_k(sampler_pass1, dim3(dim3(n_chunks, rows)), dim3(kThreads), 0, s, logits, vocab, scale, argmax_mode, part);
+  launch_k(sampler_pass2, dim3(rows), dim3(kThreads), 0, s, logits, n, vocab, scale, argmax_mode, req_ids, a.seed, a.step, a.block,
                                           part, x_hat, pmax, ent);
 }
 
@@ -265,6 +269,8 @@ __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const f
                                       int32_t* __restrict__ canvas, int32_t* __restrict__ keep_out,
                                       float* __restrict__ mean_h, int32_t* __restrict__ stop_out,
                                       int32_t* __restrict__ done, int32_t* __restrict__ out_tokens, int final_step) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float pm[];
   __shared__ float red[32];
   __shared__ int sh_stop;
@@ -314,7 +320,7 @@ void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float*
                            int32_t* stop, int32_t* done, int32_t* out_tokens, int final_step, cudaStream_t s) {
   if (B <= 0) return;
   const int threads = ((n + 31) / 32) * 32;
-  sampler_finish_kernel<<<B, threads, n * sizeof(float), s>>>(x_hat, pmax, ent, n, vocab, req_ids, a.seed, a.step,
+  launch_k(sampler_finish_kernel, dim3(B), dim3(threads), n * sizeof(float), s, x_hat, pmax, ent, n, vocab, req_ids, a.seed, a.step,
                                                               a.block, a.keep_k, a.stop_threshold, canvas, keep,
                                                               mean_h, stop, done, out_tokens, final_step);
 }
@@ -322,6 +328,8 @@ void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float*
 // ------------------------------------------------------------ self test
 __global__ void philox_selftest_kernel(const uint32_t* ctr, const uint32_t* key, uint32_t* out,
                                        uint32_t* out_curand, int n) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= n) return;
   const Philox4 o = philox4x32_10(ctr[4 * t], ctr[4 * t + 1], ctr[4 * t + 2], ctr[4 * t + 3], key[2 * t],
@@ -341,7 +349,7 @@ __global__ void philox_selftest_kernel(const uint32_t* ctr, const uint32_t* key,
 void launch_philox_selftest(const uint32_t* ctr, const uint32_t* key, uint32_t* out, uint32_t* out_curand, int n,
                             cudaStream_t s) {
   if (n <= 0) return;
-  philox_selftest_kernel<<<(n + 127) / 128, 128, 0, s>>>(ctr, key, out, out_curand, n);
+  launch_k(philox_selftest_kernel, dim3((n + 127) / 128), dim3(128), 0, s, ctr, key, out, out_curand, n);
 }
 
 }  // namespace dg

@@ -30,6 +30,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const T* __restrict__ x, const T* __restrict__ w, int n_tok,
                                                         int n_out, int kdim, int epi, void* out, int ld_out,
                                                         const float* __restrict__ bias) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float xs[TK][TS + 1];
   __shared__ float ws[TK][TS + 1];
   const int t0 = blockIdx.y * TS, n0 = blockIdx.x * TS;
@@ -73,7 +75,7 @@ void launch_gemm_simt(const T* x, const T* w, int n_tok, int n_out, int kdim, Ep
                       const float* bias, cudaStream_t s) {
   if (n_tok <= 0 || n_out <= 0) return;
   dim3 grid((n_out + TS - 1) / TS, (n_tok + TS - 1) / TS);
-  gemm_simt_kernel<T><<<grid, 256, 0, s>>>(x, w, n_tok, n_out, kdim, (int)epi, out, ld_out, bias);
+  launch_k(gemm_simt_kernel<T>, dim3(grid), dim3(256), 0, s, x, w, n_tok, n_out, kdim, (int)epi, out, ld_out, bias);
 }
 
 // ----------------------------------------------------------- grouped GEMM
@@ -86,6 +88,8 @@ __global__ void __launch_bounds__(256) grouped_simt_kernel(const T* __restrict__
                                                            const int32_t* __restrict__ n_work,
                                                            const int32_t* __restrict__ perm, int up, void* out,
                                                            int ld_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float xs[TK][TS + 1];
   __shared__ float as[TK][TS + 1];
   __shared__ float bs[TK][TS + 1];
@@ -146,7 +150,7 @@ void launch_grouped_simt(const T* x, const T* wa, const T* wb, int n_out, int kd
                          cudaStream_t s) {
   if (n_work_max <= 0) return;
   dim3 grid((n_out + TS - 1) / TS, n_work_max);
-  grouped_simt_kernel<T><<<grid, 256, 0, s>>>(x, wa, wb, n_out, kdim, work, n_work, perm, up ? 1 : 0, out, ld_out);
+  launch_k(grouped_simt_kernel<T>, dim3(grid), dim3(256), 0, s, x, wa, wb, n_out, kdim, work, n_work, perm, up ? 1 : 0, out, ld_out);
 }
 
 // -------------------------------------------------------------- attention
@@ -164,6 +168,8 @@ template <typename T>
 __global__ void __launch_bounds__(AW * 32) attn_simt_kernel(const T* __restrict__ q, const T* __restrict__ kc,
                                                             const T* __restrict__ vt, T* __restrict__ out,
                                                             AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float smem[];
   const int hd = a.hd, pitch = hd + 1;
   float* ks = smem;                         // [AKT][pitch]
@@ -259,7 +265,7 @@ void launch_attn_simt(const T* q, const T* kc, const T* vt, T* out, const AttnAr
     cudaFuncSetAttribute(attn_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
     attr_set = true;
   }
-  attn_simt_kernel<T><<<grid, AW * 32, smem, s>>>(q, kc, vt, out, a);
+  launch_k(attn_simt_kernel<T>, dim3(grid), dim3(AW * 32), smem, s, q, kc, vt, out, a);
 }
 
 #define DG_INST(T)                                                                                           \
