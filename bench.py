@@ -30,6 +30,11 @@ if ROOT not in sys.path:
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one canvas-step attention launch (prompt 8192,
+# canvas 256, 16 heads of 256), from the ncu capture summarised in
+# profiles/attn_tc_canvas_over_8192_cache.md (same shapes as one layer of the
+# full_b1 canvas step); set to None when the kernel changes.
+ATTN_TRAFFIC = 75321088
 
 
 def parse_args(argv=None):
@@ -40,7 +45,6 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["full_b1", "full_b16"], default="full_b1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--layers", type=int, default=0, help=argparse.SUPPRESS)  # debugging only (0 = as specified)
     return ap.parse_args(argv)
 
 
@@ -141,13 +145,24 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload(name, layers_override=0):
+def workload(name):
     from discrete_text_diffusion_b200 import synth
     W = dict(synth.WORKLOADS[name])
     W["model"] = dict(W["model"])
-    if layers_override:
-        W["model"]["n_layers"] = layers_override
     return W
+
+
+def attention_flops(model, batch, canvas, blocks):
+    """Algorithmic flops of the attention launches of the given blocks, all
+    layers.  blocks: (prompt length, denoise steps) per block.  Each denoise
+    step has every canvas query attend to prompt + canvas keys (QK^T and PV:
+    4 hd flops per query-key pair per head); the block's hand-off pass is
+    causal over the block (query i sees prompt + i + 1 keys)."""
+    hq, hd, L = model["n_heads"], model["head_dim"], model["n_layers"]
+    pairs = 0
+    for prompt, steps in blocks:
+        pairs += steps * canvas * (prompt + canvas) + sum(prompt + i + 1 for i in range(canvas))
+    return 4.0 * hd * hq * pairs * L * batch
 
 
 def moe_up_bytes(model, n_rows, touched):
@@ -169,7 +184,7 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dist = init_dist("nccl")
     dev = torch.device("cuda", local)
-    W = workload(args.workload, args.layers)
+    W = workload(args.workload)
     model, S = W["model"], W["sampler"]
     B, n, P0 = W["batch"], model["canvas"], W["prompt_len"]
     blocks = W.get("blocks", 1)
@@ -195,6 +210,7 @@ def run_ours(args):
     out = torch.zeros((B, n), dtype=torch.int32, device=dev)
     out_host = torch.zeros((B, n), dtype=torch.int32).pin_memory()
     steps_seen = []
+    block_log = []   # (prompt length, denoise steps) of every block run
 
     def one_step(host=False):
         total = 0
@@ -206,9 +222,11 @@ def run_ours(args):
                              logit_scale_growth=S["logit_scale_growth"], stop_threshold=S["stop_threshold"],
                              seed=S["seed"], block=blk)
             if host:
-                total += m.dg_generate_block_host(h, a, out_host)
+                used = m.dg_generate_block_host(h, a, out_host)
             else:
-                total += m.dg_generate_block(h, a, out)
+                used = m.dg_generate_block(h, a, out)
+            block_log.append((P0 + blk * n, used))
+            total += used
         steps_seen.append(total)
 
     for _ in range(args.warmup):
@@ -219,9 +237,10 @@ def run_ours(args):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # inside the timed region only the roofline kernel's launches carry events
     m.dg_profile_reset(h)
-    m.dg_profile_enable(h, True, classes=["moe_up"])
+    m.dg_profile_enable(h, True, classes=["attention"])
     launches0 = m.dg_launch_count(h)
     steps_seen.clear()
+    block_log.clear()
     with ClockSampler(local) as clk:
         barrier(dist)
         torch.cuda.synchronize(dev)
@@ -237,6 +256,7 @@ def run_ours(args):
     m.dg_profile_enable(h, False)
     clocks = clk.summary()
     denoise_steps = sum(steps_seen)
+    timed_blocks = list(block_log)
     units = args.steps * blocks * B * n
     elapsed_max, units_all = aggregate(dist, elapsed, units, device=dev)
 
@@ -260,16 +280,31 @@ def run_ours(args):
 
     peaks, peak_kind = load_peaks()
     roof = None
-    if "moe_up" in prof:
-        nl, ms = prof["moe_up"]
+    if "attention" in prof:
+        # the dominant kernel: tcgen05 attention (+ its split combine), timed on
+        # the library's stream over the whole timed region; tensor-bound, so
+        # against the sustained bf16 peak (it runs inside a long step)
+        nl, ms = prof["attention"]
+        fl = attention_flops(model, B, n, timed_blocks)
+        ach = fl / (ms / 1e3) / 1e12
+        pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"kernel": "attn_tc_kernel (+ split combine)", "bound": "tensor", "achieved": round(ach, 1),
+                "peak": pk, "peak_kind": peak_kind + " sustained", "unit": "TFLOP/s", "frac": round(ach / pk, 4),
+                "traffic": ATTN_TRAFFIC, "traffic_per": "canvas-step launch (ncu capture)",
+                "flops_timed": fl, "launches": nl,
+                "avg_launch_us": round(ms / nl * 1e3, 2)}
+    roof_moe = None
+    if "moe_up" in breakdown:
+        # from the separately profiled step (every class timed), not the timed region
+        nl, ms = breakdown["moe_up"]
         per_launch_s = ms / nl / 1e3
         byt = moe_up_bytes(model, B * n * model["top_k"], touched_mean)
         ach = byt / per_launch_s / 1e9
-        roof = {"kernel": "gemm_tc_kernel (grouped gate/up + SwiGLU)", "bound": "hbm", "achieved": round(ach, 1),
+        roof_moe = {"kernel": "gemm_tc_kernel (grouped gate/up + SwiGLU)", "bound": "hbm", "achieved": round(ach, 1),
                 "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
                 "bytes_per_launch": int(byt), "avg_launch_us": round(per_launch_s * 1e6, 2),
-                "experts_touched_mean": round(touched_mean, 2)}
+                "experts_touched_mean": round(touched_mean, 2), "timed": "profiled step"}
     line = {
         "metric": "canvas tokens/s (block generation, adaptive stop)",
         "value": round(units_all / (elapsed_max / 1e3), 2),
@@ -293,6 +328,7 @@ def run_ours(args):
                 "h2d_bytes_per_step": 4 * B * blocks, "d2h_bytes_per_step": 4 * B * n * blocks},
         "gpu_launches": int(launches),
         "roofline": roof,
+        "roofline_moe_up": roof_moe,
         "clocks": clocks,
         "prefill_s": round(prefill_s, 2),
         "kernel_ms_one_step": {k: round(v[1], 3) for k, v in breakdown.items()},

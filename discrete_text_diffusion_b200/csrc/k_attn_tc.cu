@@ -8,8 +8,11 @@
 //     the K tile (64 keys x 256) and the transposed V tile (256 x 64 keys)
 //     into one of two stages.
 //   warp 1 lane 0: MMA issuer.  S_j = Q K_j^T (M 128, N 64, K 256) into one of
-//     two TMEM score buffers, one tile ahead of O += P_j V_j (M 128, N 256,
-//     K 64) with O resident in TMEM (256 columns).
+//     kSBuf TMEM score buffers, queued kSBuf tiles ahead: S_{j+kSBuf} right
+//     behind O += P_j V_j (M 128, N 256, K 64), O resident in TMEM (256
+//     columns).  Per-tile timers show the tensor pipe busy ~1500 of ~2850
+//     cycles: the 16 S instructions (N = 64, both operands in shared memory)
+//     run at about half the rate of the 4 PV instructions.
 //   warps 2-9: softmax, two threads per query row (32 keys each).  Scores
 //     are scaled to log2 units; the running max is only raised when a tile
 //     exceeds it by more than 8 (then O and the running sum are rescaled
@@ -35,8 +38,12 @@ constexpr int kHd = 256;
 constexpr int kQBytes = kQTile * kHd * 2;   // 64 KB
 constexpr int kKBytes = kKTile * kHd * 2;   // 32 KB
 constexpr int kVBytes = kHd * kKTile * 2;   // 32 KB
+constexpr int kSBuf = 2;                      // TMEM score buffers (64 columns each; O uses [256, 512)); 3 measured no faster
 constexpr int kRedBytes = 256 * 4;           // per-row exchange between the two halves
-constexpr int kAttnSmem = 1008 + kQBytes + kKStages * kKBytes + kVStages * kVBytes + kRedBytes + 160;
+constexpr int kBarBytes = 192;               // mbarriers and the TMEM slot
+constexpr int kAttnSmem = 1008 + kQBytes + kKStages * kKBytes + kVStages * kVBytes + kRedBytes + kBarBytes;
+static_assert((1 + 2 * kKStages + 2 * kVStages + 3 * kSBuf) * 8 + 4 <= kBarBytes, "barrier area");
+static_assert(kSBuf * kKTile <= 256, "score buffers must stay below the O columns");
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct AttnTcParams {
@@ -92,14 +99,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* red = reinterpret_cast<float*>(sV + kVStages * kVBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kVStages * kVBytes + kRedBytes);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;      // [3]
-  uint64_t* k_empty = bars + 4;     // [3]
-  uint64_t* v_full = bars + 7;      // [2]
-  uint64_t* v_empty = bars + 9;     // [2]
-  uint64_t* s_full = bars + 11;     // [2]
-  uint64_t* p_full = bars + 13;     // [2]
-  uint64_t* pv_done = bars + 15;    // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* k_full = q_full + 1;          // [kKStages]
+  uint64_t* k_empty = k_full + kKStages;  // [kKStages]
+  uint64_t* v_full = k_empty + kKStages;  // [kVStages]
+  uint64_t* v_empty = v_full + kVStages;  // [kVStages]
+  uint64_t* s_full = v_empty + kVStages;  // [kSBuf]
+  uint64_t* p_full = s_full + kSBuf;      // [kSBuf]
+  uint64_t* pv_done = p_full + kSBuf;     // [kSBuf]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + kSBuf);
   int* err = P.t.err;
 
   if (threadIdx.x == 0) {
@@ -108,9 +115,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 256);
       mbar_init(&pv_done[i], 1);
@@ -128,7 +137,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // the set-up above touches no global memory: it overlaps the previous kernel
   pdl_wait();
   pdl_trigger();
-  const uint32_t tS = tmem;          // two score buffers: columns [0, 64), [64, 128)
+  const uint32_t tS = tmem;          // score buffers: columns [64 s, 64 s + 64), s < kSBuf
   const uint32_t tO = tmem + 256;    // output accumulator: columns [256, 512)
 
   if (warp == 0 && lane == 0) {
@@ -167,10 +176,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t q_base = smem_u32(sQ);
     bool ok = mbar_wait(q_full, 0, err, kErrTimeoutAttn);
     auto issue_s = [&](int j) -> bool {
-      const int s = j & 1;
+      const int s = j % kSBuf;
       const int ks = j % kKStages;
-      // S_j reuses the TMEM columns of P_{j-2}; PV_{j-2} was issued earlier,
-      // and tcgen05.mma of one thread run in issue order.
+      // S_j reuses the TMEM columns of P_{j-kSBuf}; PV_{j-kSBuf} was issued
+      // earlier, and the tcgen05.mma of one thread run in issue order.
       if (!mbar_wait(&k_full[ks], (uint32_t)(j / kKStages) & 1u, err, kErrTimeoutAttn)) return false;
       tc_fence_after();
       const uint32_t k_base = smem_u32(sK + ks * kKBytes);
@@ -184,21 +193,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       umma_commit(&k_empty[ks]);
       return true;
     };
-    if (ok) ok = issue_s(0);
+    for (int j = 0; j < min(ntiles, kSBuf) && ok; ++j) ok = issue_s(j);
     for (int j = 0; j < ntiles && ok; ++j) {
-      if (j + 1 < ntiles && !issue_s(j + 1)) break;
-      const int s = j & 1;
-      if (!mbar_wait(&p_full[s], (uint32_t)(j >> 1) & 1u, err, kErrTimeoutAttn)) break;
-      if (!mbar_wait(&v_full[s], (uint32_t)(j >> 1) & 1u, err, kErrTimeoutAttn)) break;
+      const int s = j % kSBuf;
+      const int vs = j % kVStages;
+      if (!mbar_wait(&p_full[s], (uint32_t)(j / kSBuf) & 1u, err, kErrTimeoutAttn)) break;
+      if (!mbar_wait(&v_full[vs], (uint32_t)(j / kVStages) & 1u, err, kErrTimeoutAttn)) break;
       tc_fence_after();
       // O += P_j V_j with P_j (bf16, 32 columns) read from TMEM where S_j was
-      const uint32_t v_base = smem_u32(sV + s * kVBytes);
+      const uint32_t v_base = smem_u32(sV + vs * kVBytes);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
         umma_bf16_ts(tO, tS + (uint32_t)(s * kKTile + 8 * k), sdesc_k_sw128(v_base + 32u * k), idesc_o,
                      (j > 0 || k > 0) ? 1u : 0u);
       umma_commit(&pv_done[s]);
-      umma_commit(&v_empty[s]);
+      umma_commit(&v_empty[vs]);
+      if (j + kSBuf < ntiles && !issue_s(j + kSBuf)) break;
     }
   } else if (warp >= 2 && warp < 10) {
     // ----------------------------------------------------------- softmax
@@ -214,8 +224,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+      const int s = j % kSBuf;
+      const uint32_t ph = (uint32_t)(j / kSBuf) & 1u;
       if (!mbar_wait(&s_full[s], ph, err, kErrTimeoutAttn)) { ok = false; break; }
       tc_fence_after();
       uint32_t sv[32];
@@ -245,7 +255,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float alpha = (raise && m_run > -INFINITY) ? fast_exp2(m_run - m_new) : 1.f;
       if (__any_sync(0xffffffffu, alpha != 1.f) && j > 0) {
         // O of rows in this warp must be rescaled: wait until PV_{j-1} landed
-        if (!mbar_wait(&pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, err, kErrTimeoutAttn)) {
+        if (!mbar_wait(&pv_done[(j - 1) % kSBuf], (uint32_t)((j - 1) / kSBuf) & 1u, err, kErrTimeoutAttn)) {
           ok = false;
           break;
         }
@@ -291,7 +301,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       named_barrier_sync(1, 256);
       l_run += red[(hf ^ 1) * 128 + r];
     }
-    if (ok) ok = mbar_wait(&pv_done[(ntiles - 1) & 1], (uint32_t)((ntiles - 1) >> 1) & 1u, err, kErrTimeoutAttn);
+    if (ok)
+      ok = mbar_wait(&pv_done[(ntiles - 1) % kSBuf], (uint32_t)((ntiles - 1) / kSBuf) & 1u, err, kErrTimeoutAttn);
     if (ok) {
       tc_fence_after();
       const bool valid = qi < a.nq;
