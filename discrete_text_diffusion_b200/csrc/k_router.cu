@@ -222,8 +222,133 @@ __global__ void __launch_bounds__(1024) router_permute_kernel(const int32_t* __r
   }
 }
 
+// Single-pass form for up to kPermChunks x 1024 items (a canvas step).  Per
+// chunk of 1024 items, each warp counts its items per expert with
+// __match_any_sync (no atomics); the per-expert exclusive scan over the 32
+// warps (4 threads per expert) gives every item its slot inside its expert,
+// kept in registers.  One warp then scans the expert counts into offsets and
+// writes the work list with a warp prefix sum, and the items go to
+// perm[off[e] + slot].  Same stable order as router_permute_kernel.
+constexpr int kPermChunks = 8;
+
+__global__ void __launch_bounds__(1024) router_permute_scan_kernel(const int32_t* __restrict__ ids, int n_items,
+                                                                  int e, int tile, int32_t* __restrict__ cnt_out,
+                                                                  int32_t* __restrict__ off_out,
+                                                                  int32_t* __restrict__ perm,
+                                                                  int32_t* __restrict__ work,
+                                                                  int32_t* __restrict__ n_work,
+                                                                  int32_t* __restrict__ touched) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int wc[32][256];  // this chunk: per-warp counts, then per-warp exclusive starts
+  __shared__ int running[256];
+  __shared__ int off[257];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  const int nch = (n_items + 1023) / 1024;
+  for (int x = tid; x < e; x += 1024) running[x] = 0;
+  __syncthreads();
+  int my_ex[kPermChunks], my_pos[kPermChunks];
+#pragma unroll
+  for (int c = 0; c < kPermChunks; ++c) {
+    my_ex[c] = -1;
+    my_pos[c] = 0;
+    if (c >= nch) continue;
+    const int i = c * 1024 + tid;
+    const bool valid = i < n_items;
+    const int ex = valid ? ids[i] : -1 - lane;  // invalid lanes never match a real expert
+    const unsigned peers = __match_any_sync(0xffffffffu, ex);
+    const int rank = __popc(peers & lt);
+    for (int x = lane; x < e; x += 32) wc[w][x] = 0;
+    __syncwarp();
+    if (valid && rank == 0) wc[w][ex] = __popc(peers);
+    __syncthreads();
+    {
+      // exclusive scan over the 32 warps of expert x, 4 threads x 8 warps each
+      const int x = tid >> 2, q = tid & 3;
+      int sum = 0;
+      if (x < e) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int v = wc[q * 8 + k][x];
+          wc[q * 8 + k][x] = sum;
+          sum += v;
+        }
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o, 4);
+        if (q >= o) incl += v;
+      }
+      if (x < e) {
+        const int start = running[x] + incl - sum;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) wc[q * 8 + k][x] += start;
+      }
+      __syncthreads();  // every thread has read running[x] before it moves
+      if (x < e && q == 3) running[x] += incl;
+    }
+    __syncthreads();
+    if (valid) {
+      my_ex[c] = ex;
+      my_pos[c] = wc[w][ex] + rank;
+    }
+  }
+  __syncthreads();
+  // offsets, tile counts and the work list: warp 0, experts lane*per .. lane*per+per-1
+  if (w == 0) {
+    const int per = (e + 31) / 32;
+    int c_loc = 0, t_loc = 0, nz = 0;
+    for (int u = 0; u < per; ++u) {
+      const int x = lane * per + u;
+      const int c = x < e ? running[x] : 0;
+      c_loc += c;
+      t_loc += (c + tile - 1) / tile;
+      nz += c > 0;
+    }
+    int c_in = c_loc, t_in = t_loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, c_in, o), b = __shfl_up_sync(0xffffffffu, t_in, o);
+      if (lane >= o) { c_in += a; t_in += b; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xffffffffu, nz, o);
+    int c_ex = c_in - c_loc, t_ex = t_in - t_loc;
+    for (int u = 0; u < per; ++u) {
+      const int x = lane * per + u;
+      if (x >= e) break;
+      const int c = running[x];
+      off[x] = c_ex;
+      for (int r0 = 0; r0 < c; r0 += tile, ++t_ex) {
+        work[3 * t_ex + 0] = x;
+        work[3 * t_ex + 1] = c_ex + r0;
+        work[3 * t_ex + 2] = min(tile, c - r0);
+      }
+      c_ex += c;
+    }
+    if (lane == 31) {
+      off[e] = c_in;
+      *n_work = t_in;
+    }
+    if (lane == 0) *touched = nz;
+  }
+  __syncthreads();
+  for (int x = tid; x < e; x += 1024) cnt_out[x] = running[x];
+  for (int x = tid; x <= e; x += 1024) off_out[x] = off[x];
+#pragma unroll
+  for (int c = 0; c < kPermChunks; ++c)
+    if (my_ex[c] >= 0) perm[off[my_ex[c]] + my_pos[c]] = c * 1024 + tid;
+}
+
 void launch_router_permute(const int32_t* ids, int n_items, int e, int tile, int32_t* cnt, int32_t* off,
                            int32_t* perm, int32_t* work, int32_t* n_work, int32_t* touched, cudaStream_t s) {
+  if (n_items <= kPermChunks * 1024 && e <= 256) {
+    launch_k(router_permute_scan_kernel, dim3(1), dim3(1024), 0, s, ids, n_items, e, tile, cnt, off, perm, work,
+             n_work, touched);
+    return;
+  }
   launch_k(router_permute_kernel, dim3(1), dim3(1024), 0, s, ids, n_items, e, tile, cnt, off, perm, work, n_work, touched);
 }
 
