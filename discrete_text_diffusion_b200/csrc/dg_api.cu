@@ -321,7 +321,10 @@ int grouped_tile(const dg_handle* H, int T) {
 #ifndef DG_NARROW_CTAS
 #define DG_NARROW_CTAS 2      // CTAs per SM when the token tile is <= 64 rows
 #endif
-int ksub_for(int mode, int ntile) { return (mode == 1 || ntile > 64) ? 2 : DG_NARROW_KSUB; }
+#ifndef DG_WIDE_KSUB
+#define DG_WIDE_KSUB 2        // chunks per weight box when the token tile is > 64 rows
+#endif
+int ksub_for(int mode, int ntile) { return (mode == 1) ? 2 : (ntile > 64 ? DG_WIDE_KSUB : DG_NARROW_KSUB); }
 constexpr int kMaxKSplit = 16;   // K slices of a split-K projection (router logits)
 constexpr int kMaxDenseSplit = 8;      // K slices of the split-K dense projections
 constexpr int kDenseSplitRows = 256;   // token rows up to which they take the split-K form
@@ -412,8 +415,11 @@ int dense_gemm(dg_handle* H, int cls, const void* x, const void* w, const WMap* 
 #ifndef DG_DENSE_MAXN
 #define DG_DENSE_MAXN 256     // token-tile cap (rows of the N operand)
 #endif
+#ifndef DG_SPLIT_KSUB
+#define DG_SPLIT_KSUB 2       // chunks per stage of the split-K dense projections
+#endif
 struct SplitPlan {
-  int ntile = 0, ksub = 2, split = 0;
+  int ntile = 0, ksub = DG_SPLIT_KSUB, split = 0;
 };
 
 SplitPlan split_plan(int num_sms, int T, int n_out, int K, size_t cap_floats) {
