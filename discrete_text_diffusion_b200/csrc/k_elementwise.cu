@@ -83,6 +83,21 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* o, int j4, 
   reinterpret_cast<uint2*>(o)[j4] = u;
 }
 
+// Four consecutive elements j4*4 .. j4*4+3 of a row as floats (16- or 8-byte load).
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* p, size_t j4);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p, size_t j4) {
+  return reinterpret_cast<const float4*>(p)[j4];
+}
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p, size_t j4) {
+  const uint2 u = reinterpret_cast<const uint2*>(p)[j4];
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+  return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+}
+
 template <typename T>
 __global__ void rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ w, T* __restrict__ xn,
                                int d, float eps) {
@@ -265,7 +280,7 @@ void launch_add_rmsnorm(float* h, const float* part, int nsplit, size_t split_st
 // thread and summed in slot order: no atomics, bitwise reproducible.  The
 // float4 path issues the k slot loads of a column group together.
 template <typename T>
-__global__ void combine_kernel(float* __restrict__ h, const float* __restrict__ y, const float* __restrict__ wts,
+__global__ void combine_kernel(float* __restrict__ h, const T* __restrict__ y, const float* __restrict__ wts,
                                int k, const float* __restrict__ norm_w, T* __restrict__ xn, int d, float eps) {
   pdl_wait();
   pdl_trigger();
@@ -275,17 +290,17 @@ __global__ void combine_kernel(float* __restrict__ h, const float* __restrict__ 
   if (threadIdx.x < k) ws[threadIdx.x] = wts[(size_t)t * k + threadIdx.x];
   __syncthreads();
   float* hr = h + (size_t)t * d;
-  const float* yr = y + (size_t)t * k * d;
+  const T* yr = y + (size_t)t * k * d;
   float ss = 0.f;
   if ((d & 3) == 0) {
     const int d4 = d / 4;
     float4* h4 = reinterpret_cast<float4*>(hr);
-    const float4* y4 = reinterpret_cast<const float4*>(yr);
+
     for (int j = threadIdx.x; j < d4; j += blockDim.x) {
       float4 yv[16];
 #pragma unroll
       for (int s = 0; s < 16; ++s)
-        if (s < k) yv[s] = y4[(size_t)s * d4 + j];
+        if (s < k) yv[s] = load4<T>(yr, (size_t)s * d4 + j);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int s = 0; s < 16; ++s)
@@ -313,7 +328,7 @@ __global__ void combine_kernel(float* __restrict__ h, const float* __restrict__ 
   }
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
     float acc = 0.f;
-    for (int s = 0; s < k; ++s) acc += ws[s] * yr[(size_t)s * d + j];
+    for (int s = 0; s < k; ++s) acc += ws[s] * to_f32(yr[(size_t)s * d + j]);
     const float v = hr[j] + acc;
     hr[j] = v;
     ss += v * v;
@@ -330,7 +345,7 @@ __global__ void combine_kernel(float* __restrict__ h, const float* __restrict__ 
 // in slot order.
 template <typename T, int VPT>
 __global__ void __launch_bounds__(kRowThreadsMax) combine_reg_kernel(float* __restrict__ h,
-                                                                     const float* __restrict__ y,
+                                                                     const T* __restrict__ y,
                                                                      const float* __restrict__ wts, int k,
                                                                      const float* __restrict__ norm_w,
                                                                      T* __restrict__ xn, int d, float eps) {
@@ -342,7 +357,7 @@ __global__ void __launch_bounds__(kRowThreadsMax) combine_reg_kernel(float* __re
   if (threadIdx.x < k) ws[threadIdx.x] = wts[(size_t)t * k + threadIdx.x];
   __syncthreads();
   float4* h4 = reinterpret_cast<float4*>(h + (size_t)t * d);
-  const float4* y4 = reinterpret_cast<const float4*>(y + (size_t)t * k * d);
+  const T* yt = y + (size_t)t * k * d;
   float4 v[VPT];
   float ss = 0.f;
 #pragma unroll
@@ -355,7 +370,7 @@ __global__ void __launch_bounds__(kRowThreadsMax) combine_reg_kernel(float* __re
         float4 yv[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          if (s0 + q < k) yv[q] = y4[(size_t)(s0 + q) * d4 + j];
+          if (s0 + q < k) yv[q] = load4<T>(yt, (size_t)(s0 + q) * d4 + j);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           if (s0 + q < k) {
@@ -389,7 +404,7 @@ __global__ void __launch_bounds__(kRowThreadsMax) combine_reg_kernel(float* __re
 }
 
 template <typename T>
-void launch_combine(float* h, const float* y, const float* wts, int k, const float* norm_w, T* xn, int n_tok,
+void launch_combine(float* h, const T* y, const float* wts, int k, const float* norm_w, T* xn, int n_tok,
                     int d, float eps, cudaStream_t s) {
   if (n_tok <= 0) return;
   const int vpt = k <= 16 ? row_vpt(d) : 0;
@@ -621,7 +636,7 @@ void launch_set_kv(const T* k, const T* v, T* kc, T* vt, int hkv, int n, int hd,
   template void launch_embed<T>(const int32_t*, const int32_t*, const T*, float*, T*, int, int, int, int*,    \
                                 cudaStream_t);                                                             \
   template void launch_rmsnorm<T>(const float*, const float*, T*, int, int, float, cudaStream_t);            \
-  template void launch_combine<T>(float*, const float*, const float*, int, const float*, T*, int, int, float, \
+  template void launch_combine<T>(float*, const T*, const float*, int, const float*, T*, int, int, float,     \
                                   cudaStream_t);                                                             \
   template void launch_rope_scatter<T>(const float*, int, size_t, T*, T*, T*, const float*, const BatchInfo&,  \
                                        int, int, int, int, int, cudaStream_t);                               \

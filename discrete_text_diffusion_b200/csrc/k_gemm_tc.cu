@@ -22,7 +22,8 @@
 //     weights of expert e both multiply the same token tile into two
 //     accumulators; the epilogue writes silu(gate) * up as bf16.
 //   2 grouped down: expert e's down projection; the epilogue writes row r to
-//     out[row_map[r]] (the token-slot order), fp32.
+//     out[row_map[r]] (the token-slot order) as bf16 (the combine adds the
+//     slots in fp32).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int te = threadIdx.x - 64;  // 0..127 over the epilogue warps
     float* stg = reinterpret_cast<float*>(base + P.stages * P.stage_bytes + 1024);
     __nv_bfloat16* stg_b = reinterpret_cast<__nv_bfloat16*>(stg);
-    const bool f32out = g.mode == 2 || g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32;
+    const bool f32out = g.mode == 0 && (g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32);
     float* out_f = reinterpret_cast<float*>(g.out);
     __nv_bfloat16* out_b = reinterpret_cast<__nv_bfloat16*>(g.out);
     int it = 0;
@@ -328,7 +329,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 if (c0 + j < rows) {
                   const float acc = __uint_as_float(v[j]) + bv;
                   const int tok = row0 + c0 + j;
-                  if (g.mode == 2) out_f[(size_t)g.row_map[tok] * g.ld_out + m] = acc;
+                  if (g.mode == 2) out_b[(size_t)g.row_map[tok] * g.ld_out + m] = __float2bfloat16_rn(acc);
                   else if (g.epi == EPI_STORE_F32) out_f[(size_t)ks * g.split_stride + (size_t)tok * g.ld_out + m] = acc;
                   else if (g.epi == EPI_ADD_F32) out_f[(size_t)tok * g.ld_out + m] += acc;
                   else out_b[(size_t)tok * g.ld_out + m] = __float2bfloat16_rn(acc);
@@ -365,8 +366,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             const int mm = m0 + c4 * 4;
             if (row < nrow && mm < g.M) {
               const int tok = row0 + c0 + row;
-              float* dst = (g.mode == 2) ? out_f + (size_t)g.row_map[tok] * g.ld_out + mm
-                                         : out_f + (size_t)ks * g.split_stride + (size_t)tok * g.ld_out + mm;
+              float* dst = out_f + (size_t)ks * g.split_stride + (size_t)tok * g.ld_out + mm;
               const float4 val = *reinterpret_cast<const float4*>(stg + row * kBM + c4 * 4);
               const bool add = g.mode == 0 && g.epi == EPI_ADD_F32;
               if (P.vec && mm + 3 < g.M) {
@@ -390,7 +390,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             const int idx = it2 * 128 + te, row = idx >> 4, c8 = idx & 15;
             const int mm = m0 + c8 * 8;
             if (row < nrow && mm < g.M) {
-              __nv_bfloat16* dst = out_b + (size_t)(row0 + c0 + row) * g.ld_out + mm;
+              const int tok = row0 + c0 + row;
+              __nv_bfloat16* dst = out_b + (size_t)(g.mode == 2 ? g.row_map[tok] : tok) * g.ld_out + mm;
               const __nv_bfloat16* src = stg_b + row * kBM + c8 * 8;
               if (P.vec && mm + 7 < g.M) {
                 *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
@@ -442,7 +443,7 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
     while (P.box_levels < 3 && (32 << P.box_levels) < g.ntile) ++P.box_levels;
   {
     // 16-byte output vectors need aligned rows (and slices) in elements of the output type
-    const bool f32out = g.mode == 2 || g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32;
+    const bool f32out = g.mode == 0 && (g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32);
     const int per_vec = f32out ? 4 : 8;
     P.vec = ((uintptr_t)g.out % 16 == 0) && g.ld_out % per_vec == 0 &&
             (g.ksplit <= 1 || g.split_stride % (size_t)per_vec == 0);

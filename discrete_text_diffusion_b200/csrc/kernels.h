@@ -27,9 +27,10 @@ void launch_embed(const int32_t* tok, const int32_t* prev, const T* embed, float
 // xn[t,:] = h[t,:] * w / sqrt(mean(h^2) + eps)
 template <typename T>
 void launch_rmsnorm(const float* h, const float* w, T* xn, int n_tok, int d, float eps, cudaStream_t s);
-// h[t,:] += sum_s wts[t,s] * y[t*k+s,:] (slot order), then optional xn = rmsnorm(h, norm_w)
+// h[t,:] += sum_s wts[t,s] * y[t*k+s,:] (slot order, fp32), then optional xn = rmsnorm(h, norm_w).
+// y holds the expert outputs in the activation type T.
 template <typename T>
-void launch_combine(float* h, const float* y, const float* wts, int k, const float* norm_w, T* xn,
+void launch_combine(float* h, const T* y, const float* wts, int k, const float* norm_w, T* xn,
                     int n_tok, int d, float eps, cudaStream_t s);
 // h[t,:] += sum over s < nsplit (in order) of part[s*split_stride + t*d + :]; then
 // xn = rmsnorm(h, w).  Sums the K slices of a split-K projection into the residual.
@@ -87,7 +88,7 @@ void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float*
                            int final_step, cudaStream_t s);
 
 // ---- GEMMs
-enum Epi { EPI_STORE_F32 = 0, EPI_ADD_F32 = 1, EPI_STORE_ACT = 2, EPI_SWIGLU_ACT = 3, EPI_SCATTER_F32 = 4 };
+enum Epi { EPI_STORE_F32 = 0, EPI_ADD_F32 = 1, EPI_STORE_ACT = 2, EPI_SWIGLU_ACT = 3, EPI_SCATTER_ACT = 4 };
 
 // SIMT fp32/generic path: out[t, n] (op)= sum_k x[t,k] w[n,k].
 template <typename T>
