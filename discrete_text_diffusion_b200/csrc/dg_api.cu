@@ -83,19 +83,6 @@ bool tmap_chunks4(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-// 3D bf16 map over [n2, rows, cols], box (64, box_rows, 1).
-bool tmap_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t n2, uint32_t box_rows) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {cols, rows, n2};
-  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
-  cuuint32_t box[3] = {64, box_rows, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 enum ProfClass {
   PC_EMBED, PC_DENSE, PC_ROPE, PC_ATTN, PC_NORM, PC_ROUTER, PC_GATHER, PC_MOE_UP, PC_MOE_DOWN, PC_COMBINE,
   PC_LMHEAD, PC_SAMPLER, PC_FINISH, PC_COUNT

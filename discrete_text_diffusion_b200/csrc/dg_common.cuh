@@ -101,37 +101,17 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// One poll of an mbarrier phase.  Mode 1 (default): try_wait with an explicit
-// suspend-time hint, so a thread that arrives early sleeps until the phase
-// completes (or the hint expires) instead of for a default time slice.
-// Mode 0: try_wait without a hint.  Mode 2: non-blocking test_wait.
-#ifndef DG_WAIT_MODE
-#define DG_WAIT_MODE 1
-#endif
+// One poll of an mbarrier phase: try_wait with an explicit suspend-time hint,
+// so a thread that arrives early sleeps until the phase completes (or the
+// hint expires) instead of for a default time slice.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
-#if DG_WAIT_MODE == 1
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       " selp.b32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)   // 1 ms hint
       : "memory");
-#elif DG_WAIT_MODE == 2
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.b32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-#else
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.b32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-#endif
   return ok != 0;
 }
 // Bounded wait for the phase of the given parity.  Gives up after
