@@ -313,7 +313,10 @@ int grouped_tile(const dg_handle* H, int T) {
                               // chunk, 4 stages measured 16% faster than 2 chunks, 2 stages)
 #endif
 int ksub_for(int mode, int ntile) { return (mode == 1) ? 2 : (ntile > 64 ? DG_WIDE_KSUB : DG_NARROW_KSUB); }
-constexpr int kMaxKSplit = 16;   // K slices of a split-K projection (router logits)
+#ifndef DG_ROUTER_SPLIT
+#define DG_ROUTER_SPLIT 16
+#endif
+constexpr int kMaxKSplit = DG_ROUTER_SPLIT;   // K slices of a split-K projection (router logits)
 constexpr int kMaxDenseSplit = 8;      // K slices of the split-K dense projections
 constexpr int kDenseSplitRows = 256;   // token rows up to which they take the split-K form
 int ctas_for(int ntile) { return ntile <= 64 ? DG_NARROW_CTAS : 1; }
@@ -595,6 +598,9 @@ void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
       const double cost = waves * ((tiles + n - 1) / n + 2.0) + 0.5 * n;
       if (cost < best - 1e-9) { best = cost; n_split = n; }
     }
+#ifdef DG_ATTN_SPLIT
+    n_split = std::min(DG_ATTN_SPLIT, std::max(1, tiles / 4));   // build-time override for measurements
+#endif
     if ((size_t)n_split * bi.B * c.n_heads * nq > H->part_rows_cap) n_split = 1;
     AttnTcArgs t{};
     t.a = a;
