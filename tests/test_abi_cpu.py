@@ -124,3 +124,51 @@ def test_profile_classes_follow_header():
     count = vals.pop("count")
     assert count == len(B.PROFILE_CLASSES)
     assert [c for c, _ in sorted(vals.items(), key=lambda x: x[1])] == list(B.PROFILE_CLASSES)
+
+
+def _noalloc(lib, logits, B, n, V, req, sp, canvas):
+    err = C.create_string_buffer(256)
+    rc = lib.dg_sample_noalloc(logits, B, n, V, (C.c_int * max(1, len(req)))(*req), 1,
+                               C.byref(sp) if sp is not None else None, canvas, None, None, err, 256)
+    return rc, err.value.decode()
+
+
+def test_noalloc_sampler_refuses_bad_arguments_on_host(lib):
+    """Every check of dg_sample_noalloc runs before its first CUDA call: these
+    refusals need no GPU (the pointers are never dereferenced)."""
+    fake = C.c_void_p(0x10000)        # 16-byte aligned, never touched
+    sp = B.sampler_params(temperature=1.0, keep_k=8)
+    assert _noalloc(lib, None, 1, 256, 1024, [0], sp, fake)[0] == 1            # null logits
+    assert _noalloc(lib, fake, 1, 256, 1024, [0], None, fake)[0] == 1          # null params
+    rc, msg = _noalloc(lib, C.c_void_p(0x10004), 1, 256, 1024, [0], sp, fake)  # unaligned logits
+    assert rc == 1 and "aligned" in msg
+    assert _noalloc(lib, fake, 0, 256, 1024, [], sp, fake)[0] == 1             # empty batch
+    assert _noalloc(lib, fake, 65, 256, 1024, list(range(65)), sp, fake)[0] == 1
+    assert _noalloc(lib, fake, 1, 1025, 1024, [0], sp, fake)[0] == 1           # canvas too long
+    assert _noalloc(lib, fake, 1, 256, 1024, [-1], sp, fake)[0] == 1           # negative request id
+    assert _noalloc(lib, fake, 1, 4, 1024, [0], sp, fake)[0] == 1              # keep_k > n
+    bad_t = B.sampler_params(temperature=-1.0, keep_k=1)
+    assert _noalloc(lib, fake, 1, 256, 1024, [0], bad_t, fake)[0] == 1
+    # 64 canvases of 256 over 262144 tokens exceed the fixed scratch: capacity error, nothing launched
+    rc, msg = _noalloc(lib, fake, 64, 256, 262144, list(range(64)), sp, fake)
+    assert rc == 4 and "scratch" in msg
+
+
+def test_bench_algorithmic_counts_match_brute_force():
+    """The flop and byte formulas behind bench.py's rooflines, against direct
+    counts on tiny shapes."""
+    import bench
+    model = dict(n_heads=2, head_dim=4, n_layers=3, d_model=8, d_ff=6)
+    prompt, canvas, steps = 5, 3, 2
+    pairs = 0
+    for _ in range(steps):                      # canvas step: every query sees prompt + canvas
+        pairs += canvas * (prompt + canvas)
+    pairs += sum(prompt + i + 1 for i in range(canvas))     # causal hand-off
+    want = 2 * 2 * model["head_dim"] * model["n_heads"] * pairs * model["n_layers"]   # QK^T + PV, 2 flops/MAC
+    assert bench.attention_flops(model, 1, canvas, [(prompt, steps)]) == want
+    assert bench.attention_flops(model, 2, canvas, [(prompt, steps), (prompt + canvas, 1)]) == 2 * (
+        want + 4 * model["head_dim"] * model["n_heads"] * model["n_layers"] *
+        (1 * canvas * (prompt + 2 * canvas) + sum(prompt + canvas + i + 1 for i in range(canvas))))
+    # gate+up bytes: touched experts' two [F, d] bf16 matrices, the rows read, the bf16 SwiGLU rows written
+    d, f = model["d_model"], model["d_ff"]
+    assert bench.moe_up_bytes(model, 10, 3) == 3 * 2 * f * d * 2 + 10 * d * 2 + 10 * f * 2
