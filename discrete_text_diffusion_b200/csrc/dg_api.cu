@@ -70,6 +70,20 @@ bool tmap_chunks(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, 
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// fp32 output [slices][rows][cols] (row pitch ld elements) for TMA-store
+// epilogues: dims (cols, rows, slices), boxes of (128, 32, 1), no swizzle.
+// Rows past `rows` of a slice are clipped by the store, never written.
+bool tmap_out3d(CUtensorMap* m, void* ptr, uint64_t cols, uint64_t rows, uint64_t slices, uint64_t ld) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, slices};
+  cuuint64_t strides[2] = {ld * 4, rows * ld * 4};
+  cuuint32_t box[3] = {128, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 // The same for n2 stacked matrices [n2][rows][cols]: dims (64, rows, cols/64, n2).
 bool tmap_chunks4(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t n2, uint32_t box_rows,
                   uint32_t nz) {
@@ -113,6 +127,11 @@ struct BMapEntry {
   int ntile, ksub;
   CUtensorMap m;
 };
+struct OMapEntry {
+  const void* p;
+  uint64_t cols, rows, slices, ld;
+  CUtensorMap m;
+};
 
 struct dg_handle {
   dg_config c{};
@@ -130,6 +149,7 @@ struct dg_handle {
   std::vector<LayerMaps> lmaps;
   WMap m_embed{}, m_wsc{};
   std::vector<BMapEntry> bmaps;   // token-operand maps, built on first use
+  std::vector<OMapEntry> omaps;   // fp32 output maps of the TMA-store epilogue, built on first use
   bool bad_launch = false;        // a tensor map or GEMM tiling was rejected
   // KV cache (owned)
   void* kc = nullptr;
@@ -343,8 +363,30 @@ const CUtensorMap* bmap(dg_handle* H, const void* p, uint64_t cols, uint64_t row
 }
 
 void run_tc(dg_handle* H, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap* b,
-            TcGemm& g, const CUtensorMap* bsub = nullptr) {
-  if (!b || launch_gemm_tc(a0, a1, a2, *b, bsub, g, H->num_sms, H->stream) != 0) H->bad_launch = true;
+            TcGemm& g, const CUtensorMap* bsub = nullptr, const CUtensorMap* tout = nullptr) {
+  if (!b || launch_gemm_tc(a0, a1, a2, *b, bsub, g, H->num_sms, H->stream, tout) != 0) H->bad_launch = true;
+}
+
+// Output map of a dense fp32 store (slices of rows x cols, pitch ld), cached;
+// returns false when it cannot be built (the launch then uses plain stores).
+bool omap(dg_handle* H, void* p, uint64_t cols, uint64_t rows, uint64_t slices, uint64_t ld, CUtensorMap* out) {
+  for (const auto& e : H->omaps)
+    if (e.p == p && e.cols == cols && e.rows == rows && e.slices == slices && e.ld == ld) {
+      *out = e.m;
+      return true;
+    }
+  if (((uintptr_t)p & 15u) != 0 || ld % 4 != 0) return false;
+  OMapEntry e;
+  e.p = p;
+  e.cols = cols;
+  e.rows = rows;
+  e.slices = slices;
+  e.ld = ld;
+  if (!tmap_out3d(&e.m, p, cols, rows, slices, ld)) return false;
+  if (H->omaps.size() >= 64) H->omaps.clear();   // callers passing fresh output buffers each step
+  H->omaps.push_back(e);
+  *out = e.m;
+  return true;
 }
 
 // Token maps of a grouped GEMM's activation rows: boxes of 32, 64 and 128
@@ -392,7 +434,9 @@ int dense_gemm(dg_handle* H, int cls, const void* x, const void* w, const WMap* 
   g.ksplit = split;
   g.split_stride = (size_t)T * ld_out;
   const CUtensorMap& a = pick(*mw, g.ksub);
-  run_tc(H, a, a, a, bmap(H, x, K, H->T_max, g.ntile, g.ksub), g);
+  CUtensorMap to;
+  const bool tma_out = epi == EPI_STORE_F32 && omap(H, out, n_out, T, split, ld_out, &to);
+  run_tc(H, a, a, a, bmap(H, x, K, H->T_max, g.ntile, g.ksub), g, nullptr, tma_out ? &to : nullptr);
   return split;
 }
 
@@ -445,7 +489,9 @@ void run_split(dg_handle* H, const CUtensorMap& a0, const CUtensorMap& a1, const
   g.ctas_per_sm = 1;
   g.ksplit = p.split;
   g.split_stride = (size_t)T * n_out;
-  run_tc(H, a0, a1, a2, b, g);
+  CUtensorMap to;
+  const bool tma_out = omap(H, part, n_out, T, p.split, n_out, &to);
+  run_tc(H, a0, a1, a2, b, g, nullptr, tma_out ? &to : nullptr);
 }
 
 // The layers' use of the split-K form: up to three weight maps stacked along
@@ -1246,7 +1292,9 @@ int dg_selftest_gemm(dg_handle* H, const void* x, const void* w, int T, int M, i
   if (!tmap_chunks(&mx, x, K, T, K, (uint32_t)g.ntile, (uint32_t)g.ksub) ||
       !tmap_chunks(&mw, w, K, M, K, 128, (uint32_t)g.ksub))
     return fail(H, DG_ECUDA, "tensor map encode failed");
-  if (launch_gemm_tc(mw, mw, mw, mx, nullptr, g, H->num_sms, H->stream) != 0)
+  CUtensorMap to;
+  const bool tma_out = tmap_out3d(&to, out, M, T, 1, M);
+  if (launch_gemm_tc(mw, mw, mw, mx, nullptr, g, H->num_sms, H->stream, tma_out ? &to : nullptr) != 0)
     return fail(H, DG_EINVAL, "GEMM tiling rejected");
   H->launches += 1;
   return check_launch(H, "selftest gemm");

@@ -75,7 +75,8 @@ static TcLayout tc_layout(const TcGemm& p) {
   L.per_sm = std::max(1, std::min(3, p.ctas_per_sm > 0 ? p.ctas_per_sm : DG_GEMM_CTAS_PER_SM));
   // the tensor maps are built for this chunk count: it is never changed here
   L.ksub = std::max(1, std::min(4, p.ksub > 0 ? p.ksub : DG_GEMM_KSUB));
-  const int overhead = 1024 /*align*/ + 1024 /*barriers*/ + (((DG_EPI_STAGE_MODES >> p.mode) & 1) ? kEpiBytes : 0);
+  const int n_stg = ((DG_EPI_STAGE_MODES >> p.mode) & 1) ? (p.tma_out ? 2 : 1) : 0;   // staging tiles
+  const int overhead = 1024 /*align*/ + 1024 /*barriers*/ + n_stg * kEpiBytes;
   for (;;) {
     // TMEM: every co-resident CTA holds its accumulators
     L.n_acc_buf = (L.per_sm * 2 * L.acc_cols <= 512) ? 2 : 1;
@@ -148,7 +149,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap ta1,
                    const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb,
                    const __grid_constant__ CUtensorMap tbs0, const __grid_constant__ CUtensorMap tbs1,
-                   const __grid_constant__ CUtensorMap tbs2, const TcKParams P) {
+                   const __grid_constant__ CUtensorMap tbs2, const __grid_constant__ CUtensorMap tout,
+                   const TcKParams P) {
   extern __shared__ uint8_t smem_raw[];
   const TcGemm& g = P.g;
   const uint32_t raw = smem_u32(smem_raw);
@@ -291,6 +293,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const bool f32out = g.mode == 0 && (g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32);
     float* out_f = reinterpret_cast<float*>(g.out);
     __nv_bfloat16* out_b = reinterpret_cast<__nv_bfloat16*>(g.out);
+    // TMA-store form (dense fp32 stores): two staging tiles used in turn; the
+    // thread that issues the stores (te 0) frees a tile by waiting for the
+    // store issued from it two chunks earlier.
+    const bool tstore = g.tma_out != 0;
+    uint32_t chunk_no = 0;
     int it = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
       int m0, e, row0, rows, j0, j1, ks;
@@ -348,6 +355,21 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             const float gt = __uint_as_float(v[j]), up = __uint_as_float(u[j]);
             stg_b[j * kBM + r] = __float2bfloat16_rn(gt / (1.f + expf(-gt)) * up);
           }
+        } else if (tstore) {
+          tmem_ld_wait();
+          float* tile = stg + (chunk_no & 1u) * (kEpiBytes / 4);
+          if (te == 0 && chunk_no >= 2) bulk_wait_read_1();
+          named_barrier_sync(1, 128);  // the tile's previous store has finished reading it
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tile[j * kBM + r] = __uint_as_float(v[j]) + bv;
+          fence_proxy_async_smem();
+          named_barrier_sync(1, 128);
+          if (te == 0) {
+            tma_store_3d(&tout, tile, m0, row0 + c0, ks);
+            bulk_commit();
+          }
+          ++chunk_no;
+          continue;
         } else if (f32out) {
           tmem_ld_wait();
 #pragma unroll
@@ -406,6 +428,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);
     }
+    if (tstore && te == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -425,7 +448,9 @@ static void set_smem_attr() {
 }
 
 int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
-                   const CUtensorMap* bsub, const TcGemm& g, int num_sms, cudaStream_t s) {
+                   const CUtensorMap* bsub, const TcGemm& g_in, int num_sms, cudaStream_t s, const CUtensorMap* tout) {
+  TcGemm g = g_in;
+  g.tma_out = (tout != nullptr && g.mode == 0 && g.epi == EPI_STORE_F32 && ((DG_EPI_STAGE_MODES & 1) != 0)) ? 1 : 0;
   const TcLayout L = tc_layout(g);
   if (L.stages < 2) return -1;   // the tile does not fit a two-stage pipeline
   TcKParams P;
@@ -456,7 +481,8 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   const CUtensorMap& s0 = P.box_levels > 0 ? bsub[0] : b;
   const CUtensorMap& s1 = P.box_levels > 1 ? bsub[1] : b;
   const CUtensorMap& s2 = P.box_levels > 2 ? bsub[2] : b;
-  launch_k(gemm_tc_kernel, dim3(grid), dim3(kTcThreads), L.smem_bytes, s, a0, a1, a2, b, s0, s1, s2, P);
+  launch_k(gemm_tc_kernel, dim3(grid), dim3(kTcThreads), L.smem_bytes, s, a0, a1, a2, b, s0, s1, s2,
+           g.tma_out ? *tout : b, P);
   return 0;
 }
 

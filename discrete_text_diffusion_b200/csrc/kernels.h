@@ -123,13 +123,17 @@ struct TcGemm {
   int ksplit;        // dense EPI_STORE_F32 only: K split into ksplit slices, slice s
                      // writes its partial sums at out + s * split_stride (floats)
   size_t split_stride;
+  int tma_out;       // set by the launcher: the output goes out through TMA stores
 };
 // Returns 0, or -1 when the tile does not fit a two-stage pipeline (nothing launched).
 // b: token map with boxes of ntile rows.  bsub (grouped modes, or NULL): maps of the
 // same tokens with boxes of 32, 64, 128 rows (those below ntile), used for work
 // items with fewer rows.
+// tout (dense EPI_STORE_F32, or NULL): fp32 map of the output as (M, T, ksplit) with boxes of
+// (128, 32, 1); the epilogue then writes each 32-row chunk with one TMA store.
 int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
-                   const CUtensorMap* bsub, const TcGemm& p, int num_sms, cudaStream_t s);
+                   const CUtensorMap* bsub, const TcGemm& p, int num_sms, cudaStream_t s,
+                   const CUtensorMap* tout = nullptr);
 int gemm_tc_smem_bytes(const TcGemm& p, int* stages);
 
 // ---- attention
