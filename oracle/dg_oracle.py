@@ -41,6 +41,15 @@ Readings of points the pages leave open (each is a named reading, R-x):
             softmax over the k selected logits.
   R-append  a finished canvas is appended by one causal encode pass over its
             tokens (no self-conditioning).
+  The page's own sampler variants ([P1 四]; the CUDA path has them next):
+  R-budget  entropy-ordered locking: positions sorted by entropy ascending
+            (ties -> lower index) are kept while the inclusive cumulative
+            entropy stays <= the budget (0.1); the position that crosses it and
+            all after it are re-noised.
+  R-anneal  the temperature falls linearly from 0.8 at round 1 to 0.4 at the
+            last round of the step budget.
+  R-stop2   stop after round t when the mean entropy of rounds t-1 and t is
+            below 0.005 and the argmax sequence of round t equals round t-1's.
 
 Parity pins: every public function here is pinned by ``tests/test_oracle_*.py``
 against library routines, closed forms, invariants or brute force.  Parity
@@ -263,6 +272,48 @@ def keep_set(pmax, k):
     else:
         margin = math.inf
     return keep, margin
+
+
+def keep_entropy_budget(ent, budget):
+    """Entropy-ordered locking of [P1 四] (R-budget).
+
+    Positions are taken in order of increasing entropy (ties -> lower index)
+    and kept while the running sum of their entropies, this position
+    included, is <= budget.  Returns (bool mask [N], relative margin: the
+    distance of the running sum at the first rejected position from the
+    budget, inf if none is rejected)."""
+    ent = np.asarray(ent, dtype=np.float64)
+    n = len(ent)
+    order = np.lexsort((np.arange(n), ent))
+    keep = np.zeros(n, dtype=bool)
+    run = 0.0
+    for i in order:
+        if run + ent[i] > budget:
+            return keep, ((run + ent[i]) - budget) / max(abs(budget), 1e-300)
+        run += ent[i]
+        keep[i] = True
+    return keep, math.inf
+
+
+def anneal_temperature(t: int, t_total: int, t_start: float = 0.8, t_end: float = 0.4) -> float:
+    """Linear temperature anneal of [P1 四] (R-anneal): t_start at round 1,
+    t_end at round t_total."""
+    if t_total <= 1:
+        return float(t_end)
+    return float(t_start + (t_end - t_start) * (t - 1) / (t_total - 1))
+
+
+def argmax_tokens(logits):
+    """The most likely token per position, ties -> lower index: [N, V] -> [N]."""
+    return np.argmax(np.asarray(logits), axis=-1).astype(np.int64)
+
+
+def stop_two_rounds(mean_h_prev, mean_h, argmax_prev, argmax, tau=0.005):
+    """Adaptive stop of [P1 四] (R-stop2): both rounds' mean entropy below tau
+    and an unchanged argmax sequence.  The first round has no previous one."""
+    if argmax_prev is None or mean_h_prev is None:
+        return False
+    return bool(mean_h_prev < tau and mean_h < tau and np.array_equal(argmax_prev, argmax))
 
 
 def sample_canvas(logits, *, seed, step, block, req, temperature, logit_scale,

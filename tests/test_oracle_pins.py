@@ -386,3 +386,62 @@ def test_self_conditioning_term():
     want = torch.from_numpy(E[toks]) + F.linear(torch.from_numpy(E[prev]), torch.from_numpy(W))
     assert np.allclose(got, want.numpy())
     assert np.allclose(m.embed_tokens(toks), E[toks])
+
+
+# ------------------------------------------------ the page's sampler variants
+
+def test_entropy_budget_keep_worked_example():
+    # sorted: 0.01 (pos 1), 0.03 (pos 3), 0.05 (pos 0) -> running 0.01, 0.04, 0.09 <= 0.1; +0.2 crosses
+    keep, margin = O.keep_entropy_budget([0.05, 0.01, 0.2, 0.03], 0.1)
+    assert keep.tolist() == [True, True, False, True]
+    assert margin == pytest.approx((0.29 - 0.1) / 0.1)
+    # a tie at the boundary goes to the lower index
+    keep, _ = O.keep_entropy_budget([0.04, 0.05, 0.05, 0.0], 0.1)
+    assert keep.tolist() == [True, True, False, True]
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_entropy_budget_keep_invariants(seed):
+    rng = np.random.default_rng(seed)
+    ent = np.round(rng.exponential(0.02, 64), 3)          # rounding makes ties
+    for budget in (0.0, 0.05, 0.1, 0.3, 10.0):
+        keep, _ = O.keep_entropy_budget(ent, budget)
+        kept, rest = np.nonzero(keep)[0], np.nonzero(~keep)[0]
+        assert ent[kept].sum() <= budget + 1e-12
+        if len(rest):
+            # every kept position precedes every rejected one in (entropy, index) order ...
+            first = min(rest, key=lambda i: (ent[i], i))
+            assert all((ent[i], i) < (ent[first], first) for i in kept)
+            # ... and the first rejected one does not fit the budget
+            assert ent[kept].sum() + ent[first] > budget
+        else:
+            assert ent.sum() <= budget
+    assert O.keep_entropy_budget(ent, -1.0)[0].sum() == 0
+
+
+def test_anneal_is_linear_from_08_to_04():
+    assert O.anneal_temperature(1, 48) == pytest.approx(0.8)
+    assert O.anneal_temperature(48, 48) == pytest.approx(0.4)
+    mid = O.anneal_temperature(1, 3), O.anneal_temperature(2, 3), O.anneal_temperature(3, 3)
+    assert mid == pytest.approx((0.8, 0.6, 0.4))
+    ts = [O.anneal_temperature(t, 48) for t in range(1, 49)]
+    steps = np.diff(ts)
+    assert np.allclose(steps, steps[0]) and steps[0] < 0
+
+
+def test_two_round_stop_truth_table():
+    a = np.array([3, 1, 4])
+    b = np.array([3, 1, 5])
+    assert O.stop_two_rounds(0.001, 0.002, a, a.copy())
+    assert not O.stop_two_rounds(0.001, 0.002, a, b)          # argmax changed
+    assert not O.stop_two_rounds(0.01, 0.002, a, a.copy())    # previous round too uncertain
+    assert not O.stop_two_rounds(0.001, 0.006, a, a.copy())   # this round too uncertain
+    assert not O.stop_two_rounds(None, 0.001, None, a)        # first round
+
+
+def test_argmax_tokens_takes_the_lower_index_on_ties():
+    lg = np.array([[0.0, 2.0, 2.0, 1.0], [5.0, 5.0, 5.0, 5.0]])
+    assert O.argmax_tokens(lg).tolist() == [1, 0]
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((16, 50))
+    assert np.array_equal(O.argmax_tokens(x), torch.from_numpy(x).argmax(-1).numpy())
