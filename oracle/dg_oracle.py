@@ -41,7 +41,8 @@ Readings of points the pages leave open (each is a named reading, R-x):
             softmax over the k selected logits.
   R-append  a finished canvas is appended by one causal encode pass over its
             tokens (no self-conditioning).
-  The page's own sampler variants ([P1 四]; the CUDA path has them next):
+  The page's own sampler variants ([P1 四]; the CUDA path has R-budget and
+  R-anneal, R-stop2 is here only):
   R-budget  entropy-ordered locking: positions sorted by entropy ascending
             (ties -> lower index) are kept while the inclusive cumulative
             entropy stays <= the budget (0.1); the position that crosses it and
@@ -317,12 +318,14 @@ def stop_two_rounds(mean_h_prev, mean_h, argmax_prev, argmax, tau=0.005):
 
 
 def sample_canvas(logits, *, seed, step, block, req, temperature, logit_scale,
-                  keep_k, stop_threshold):
+                  keep_k, stop_threshold, keep_budget=None):
     """Sampler for one canvas: stats, Philox sample, keep, re-noise, stop.
 
     logits [N, V].  Returns dict with x_hat, pmax, H, keep, x_new, mean_H, stop
     and the decision margins (sample_margin [N], keep_margin, stop_margin).
-    stop_threshold < 0 disables the stop test.
+    stop_threshold < 0 disables the stop test.  keep_budget=None keeps the
+    keep_k most confident positions; a number keeps the entropy-budget set
+    (R-budget) and ignores keep_k.
     """
     n, vocab = logits.shape
     words = sampler_words(seed, np.arange(n), step, block, req)
@@ -340,7 +343,10 @@ def sample_canvas(logits, *, seed, step, block, req, temperature, logit_scale,
             smargin[i] = math.inf
         else:
             x_hat[i], smargin[i] = inverse_cdf(st["e"], st["S"], u[i])
-    keep, kmargin = keep_set(pmax, keep_k)
+    if keep_budget is None:
+        keep, kmargin = keep_set(pmax, keep_k)
+    else:
+        keep, kmargin = keep_entropy_budget(ent, keep_budget)
     x_new = np.where(keep, x_hat, renoise)
     mean_h = float(ent.mean())
     stop = bool(stop_threshold >= 0 and mean_h < stop_threshold)
@@ -469,33 +475,41 @@ class OracleModel:
         return (logits, h) if return_hidden else logits
 
     def denoise_step(self, req, canvas, prev_pred, *, step, block, seed, temperature,
-                     logit_scale, keep_k, stop_threshold):
+                     logit_scale, keep_k, stop_threshold, keep_budget=None):
         logits = self.denoise_forward(req, canvas, prev_pred)
         out = sample_canvas(logits, seed=seed, step=step, block=block, req=req,
                             temperature=temperature, logit_scale=logit_scale,
-                            keep_k=keep_k, stop_threshold=stop_threshold)
+                            keep_k=keep_k, stop_threshold=stop_threshold,
+                            keep_budget=keep_budget)
         out["logits"] = logits
         return out
 
     def generate_block(self, req, *, seed, block, max_steps, schedule_steps,
                        temperature, logit_scale_growth=1.0, stop_threshold=-1.0,
-                       append=True):
+                       append=True, keep_budget=None, temperature_end=None):
         """One block ([P1 一/四], [P2 运作机制], [P3]): random canvas, up to
         max_steps denoise steps with the linear keep schedule over
         schedule_steps, stop on mean entropy, output the last x_hat, then the
-        causal hand-off of the block into the cache.  Returns (tokens, steps, trace)."""
+        causal hand-off of the block into the cache.  Returns (tokens, steps, trace).
+        keep_budget: the entropy-budget keep (R-budget) instead of the schedule.
+        temperature_end: the linear anneal (R-anneal) from `temperature` at
+        step 1 to it at step max_steps; each step's temperature is recorded in
+        its trace entry."""
         n, vocab = self.cfg["canvas"], self.cfg["vocab"]
         canvas = init_canvas(seed, n, vocab, block, req)
         prev = None
         trace = []
         out_tokens, steps = None, 0
         for t in range(1, max_steps + 1):
+            temp = temperature if temperature_end is None else \
+                anneal_temperature(t, max_steps, temperature, temperature_end)
             r = self.denoise_step(req, canvas, prev, step=t, block=block, seed=seed,
-                                  temperature=temperature,
+                                  temperature=temp,
                                   logit_scale=logit_scale_growth ** (t - 1),
                                   keep_k=linear_keep_count(n, t, schedule_steps),
-                                  stop_threshold=stop_threshold)
+                                  stop_threshold=stop_threshold, keep_budget=keep_budget)
             r["canvas_in"] = canvas.copy()
+            r["temperature"] = temp
             trace.append(r)
             steps = t
             if r["stop"] or t == max_steps:

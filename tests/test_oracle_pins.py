@@ -445,3 +445,47 @@ def test_argmax_tokens_takes_the_lower_index_on_ties():
     rng = np.random.default_rng(3)
     x = rng.standard_normal((16, 50))
     assert np.array_equal(O.argmax_tokens(x), torch.from_numpy(x).argmax(-1).numpy())
+
+
+def test_sampler_with_entropy_budget_keeps_the_budget_set_of_its_own_entropies():
+    rng = np.random.default_rng(23)
+    logits = rng.standard_normal((12, 40)) * rng.uniform(0.1, 6.0, (12, 1))   # mixed confidence
+    kw = dict(seed=3, step=2, block=1, req=0, temperature=0.9, logit_scale=1.0, keep_k=5, stop_threshold=-1.0)
+    base = O.sample_canvas(logits, **kw)
+    for budget in (0.0, 1.0, 4.0, 1e9):
+        out = O.sample_canvas(logits, keep_budget=budget, **kw)
+        keep, _ = O.keep_entropy_budget(out["H"], budget)
+        assert np.array_equal(out["keep"], keep)
+        # keep_k is ignored; the sample, the statistics and the re-noise tokens are the top-k run's
+        assert np.array_equal(out["x_hat"], base["x_hat"]) and np.allclose(out["H"], base["H"])
+        assert np.array_equal(out["x_new"], np.where(keep, out["x_hat"], base["renoise"]))
+    assert O.sample_canvas(logits, keep_budget=1e9, **kw)["keep"].all()
+    assert not O.sample_canvas(logits, keep_budget=0.0, **kw)["keep"].any()   # every H > 0 here
+
+
+def test_block_with_anneal_runs_each_step_at_the_annealed_temperature():
+    def run(**extra):
+        m = _tiny_model(seed=24, n_layers=1)
+        m.encode_causal(0, np.arange(4))
+        return m.generate_block(0, seed=1, block=0, max_steps=4, schedule_steps=4, temperature=0.8,
+                                stop_threshold=-1.0, append=False, **extra)
+    toks, steps, trace = run(temperature_end=0.4)
+    assert steps == 4
+    assert [r["temperature"] for r in trace] == pytest.approx([0.8, 0.8 - 0.4 / 3, 0.8 - 0.8 / 3, 0.4])
+    # each step equals a plain step at that temperature from the same canvas and self-conditioning
+    m = _tiny_model(seed=24, n_layers=1)
+    m.encode_causal(0, np.arange(4))
+    prev = None
+    for t, r in enumerate(trace, start=1):
+        one = m.denoise_step(0, r["canvas_in"], prev, step=t, block=0, seed=1, temperature=r["temperature"],
+                             logit_scale=1.0, keep_k=O.linear_keep_count(m.cfg["canvas"], t, 4),
+                             stop_threshold=-1.0)
+        assert np.array_equal(one["x_new"], r["x_new"]) and np.allclose(one["H"], r["H"])
+        prev = r["x_hat"]
+    # an anneal whose ends are equal is the constant-temperature block
+    a = run(temperature_end=0.8)
+    b = run()
+    assert a[1] == b[1] and np.array_equal(a[0], b[0])
+    # the budget keep plugs into the block: a budget of 0 keeps nothing until the last step's output
+    toks, steps, trace = run(keep_budget=0.0)
+    assert all(not r["keep"].any() for r in trace) and np.array_equal(toks, trace[-1]["x_hat"])
