@@ -794,6 +794,8 @@ SamplerArgs sampler_args(const dg_sampler_params& sp, int step) {
   a.seed = sp.seed;
   a.block = sp.block;
   a.step = (uint32_t)step;
+  a.keep_mode = sp.keep_mode;
+  a.entropy_budget = sp.entropy_budget;
   return a;
 }
 
@@ -803,6 +805,10 @@ int check_sampler_params(dg_handle* H, const dg_sampler_params* sp) {
     return fail(H, DG_EINVAL, "temperature must be finite and >= 0");
   if (!(sp->logit_scale > 0.f) || !std::isfinite(sp->logit_scale)) return fail(H, DG_EINVAL, "logit_scale must be > 0");
   if (sp->keep_k < 0 || sp->keep_k > H->c.canvas) return fail(H, DG_EINVAL, "keep_k out of [0, N]");
+  if (sp->keep_mode != DG_KEEP_TOPK && sp->keep_mode != DG_KEEP_ENTROPY_BUDGET)
+    return fail(H, DG_EINVAL, "unknown keep_mode %d", sp->keep_mode);
+  if (sp->keep_mode == DG_KEEP_ENTROPY_BUDGET && !(sp->entropy_budget >= 0.f && std::isfinite(sp->entropy_budget)))
+    return fail(H, DG_EINVAL, "entropy_budget must be finite and >= 0");
   return DG_OK;
 }
 
@@ -1158,6 +1164,13 @@ static int generate_block_impl(dg_handle* H, const dg_block_args* a, int32_t* ou
   if (rc) return rc;
   if (a->max_steps < 1 || a->schedule_steps < 1) return fail(H, DG_EINVAL, "max_steps and schedule_steps must be >= 1");
   if (!(a->temperature >= 0.f) || !(a->logit_scale_growth > 0.f)) return fail(H, DG_EINVAL, "bad temperature / growth");
+  if (a->anneal && !(a->temperature > 0.f && a->temperature_end > 0.f && std::isfinite(a->temperature) &&
+                     std::isfinite(a->temperature_end)))
+    return fail(H, DG_EINVAL, "an annealed temperature needs finite ends > 0");
+  if (a->keep_mode != DG_KEEP_TOPK && a->keep_mode != DG_KEEP_ENTROPY_BUDGET)
+    return fail(H, DG_EINVAL, "unknown keep_mode %d", a->keep_mode);
+  if (a->keep_mode == DG_KEEP_ENTROPY_BUDGET && !(a->entropy_budget >= 0.f && std::isfinite(a->entropy_budget)))
+    return fail(H, DG_EINVAL, "entropy_budget must be finite and >= 0");
   for (int b = 0; b < bi.B; ++b)
     if (bi.len[b] + c.canvas > c.max_ctx) return fail(H, DG_ECAPACITY, "cache + canvas exceeds max_ctx");
   if ((rc = upload_req(H, bi))) return rc;
@@ -1172,11 +1185,20 @@ static int generate_block_impl(dg_handle* H, const dg_block_args* a, int32_t* ou
   for (int t = 1; t <= a->max_steps; ++t) {
     dg_sampler_params sp;
     sp.temperature = a->temperature;
+    if (a->anneal) {
+      // linear from T at step 1 to T_end at step max_steps, in double ([P1 四])
+      const double t0 = a->temperature, t1 = a->temperature_end;
+      sp.temperature = a->max_steps <= 1 ? a->temperature_end
+                                         : (float)(t0 + (t1 - t0) * (double)(t - 1) / (double)(a->max_steps - 1));
+    }
     sp.logit_scale = (float)std::pow((double)a->logit_scale_growth, (double)(t - 1));
     sp.stop_threshold = a->stop_threshold;
     sp.keep_k = std::min(n, (int)(((long long)n * t + a->schedule_steps - 1) / a->schedule_steps));
     sp.seed = a->seed;
     sp.block = a->block;
+    sp.keep_mode = a->keep_mode;
+    sp.entropy_budget = a->entropy_budget;
+    if ((rc = check_sampler_params(H, &sp))) return rc;
     run_layers(H, bi, n, false, H->canvas, prev, true, H->logits, nullptr);
     int32_t* xh = H->xh[t & 1];
     run_sampler(H, H->logits, bi, sampler_args(sp, t), H->canvas, xh, H->pmax, H->ent, H->keep, H->meanh, H->stop,

@@ -66,6 +66,10 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
   if (!(sp->logit_scale > 0.f) || !std::isfinite(sp->logit_scale))
     return report(err, err_len, DG_EINVAL, "logit_scale must be > 0");
   if (sp->keep_k < 0 || sp->keep_k > n) return report(err, err_len, DG_EINVAL, "keep_k out of [0, N]");
+  if (sp->keep_mode != DG_KEEP_TOPK && sp->keep_mode != DG_KEEP_ENTROPY_BUDGET)
+    return report(err, err_len, DG_EINVAL, "unknown keep_mode %d", sp->keep_mode);
+  if (sp->keep_mode == DG_KEEP_ENTROPY_BUDGET && !(sp->entropy_budget >= 0.f && std::isfinite(sp->entropy_budget)))
+    return report(err, err_len, DG_EINVAL, "entropy_budget must be finite and >= 0");
 
   // scratch layout: request ids | x_hat | pmax | entropy | chunk partials
   const size_t rows = (size_t)batch * n;
@@ -116,6 +120,8 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
   a.seed = sp->seed;
   a.block = sp->block;
   a.step = (uint32_t)step;
+  a.keep_mode = sp->keep_mode;
+  a.entropy_budget = sp->entropy_budget;
   launch_sampler_rows(logits, (int)rows, n, vocab, req_dev, a, base + off_ws, xh, pmax, ent, s);
   launch_sampler_finish(xh, pmax, ent, batch, n, vocab, req_dev, a, canvas, o ? o->keep : nullptr,
                         o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0, s);

@@ -262,24 +262,49 @@ void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const 
                                           part, x_hat, pmax, ent);
 }
 
-// Pass 3: per canvas.  rank_i = #{j : pmax_j > pmax_i or (pmax_j == pmax_i and j < i)}.
+// Pass 3: per canvas.  Top-k keep: rank_i = #{j : pmax_j > pmax_i or
+// (pmax_j == pmax_i and j < i)}, kept iff rank_i < keep_k.  Entropy budget:
+// r_i = #{j : H_j < H_i or (H_j == H_i and j < i)} orders the positions by
+// entropy; C_i = sum of H_j over r_j <= r_i (fp64) is the running sum that
+// reaches position i, and the positions kept are those ranked before the first
+// one whose C exceeds the budget (a running sum of H >= 0 only grows, so that
+// is also where it stays above).
 __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const float* __restrict__ pmax,
                                       const float* __restrict__ ent, int n, int vocab, const int* __restrict__ req_ids,
-                                      uint64_t seed, uint32_t step, uint32_t block, int keep_k, float stop_thr,
+                                      uint64_t seed, uint32_t step, uint32_t block, int keep_k, int keep_mode,
+                                      float budget, float stop_thr,
                                       int32_t* __restrict__ canvas, int32_t* __restrict__ keep_out,
                                       float* __restrict__ mean_h, int32_t* __restrict__ stop_out,
                                       int32_t* __restrict__ done, int32_t* __restrict__ out_tokens, int final_step) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ float pm[];
+  extern __shared__ float pm[];  // [n] pmax, then [n] entropy for the budget keep
+  float* eh = pm + n;
   __shared__ float red[32];
   __shared__ int sh_stop;
+  __shared__ int sh_cut;         // budget keep: entropy rank of the first position re-noised
   const int b = blockIdx.x;
   const int req = req_ids[b];
   const int i = threadIdx.x;
-  for (int j = i; j < n; j += blockDim.x) pm[j] = pmax[(size_t)b * n + j];
+  for (int j = i; j < n; j += blockDim.x) {
+    pm[j] = pmax[(size_t)b * n + j];
+    if (keep_mode == 1) eh[j] = ent[(size_t)b * n + j];
+  }
+  if (i == 0) sh_cut = n;
   const int was_done = (done != nullptr) ? done[b] : 0;
   __syncthreads();
+  int hrank = 0;
+  if (keep_mode == 1 && i < n) {
+    const float h = eh[i];
+    double run = 0.0;
+    for (int j = 0; j < n; ++j) {
+      const float q = eh[j];
+      const int before = (q < h || (q == h && j < i)) ? 1 : 0;
+      hrank += before;
+      if (before || j == i) run += (double)q;
+    }
+    if (run > (double)budget) atomicMin(&sh_cut, hrank);
+  }
   float hsum = 0.f;
   if (i < n) hsum = ent[(size_t)b * n + i];
   // deterministic block sum over positions
@@ -297,13 +322,18 @@ __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const f
   }
   __syncthreads();
   if (i < n) {
-    const float p = pm[i];
-    int rank = 0;
-    for (int j = 0; j < n; ++j) {
-      const float q = pm[j];
-      rank += (q > p || (q == p && j < i)) ? 1 : 0;
+    int kept;
+    if (keep_mode == 1) {
+      kept = hrank < sh_cut;
+    } else {
+      const float p = pm[i];
+      int rank = 0;
+      for (int j = 0; j < n; ++j) {
+        const float q = pm[j];
+        rank += (q > p || (q == p && j < i)) ? 1 : 0;
+      }
+      kept = rank < keep_k;
     }
-    const int kept = rank < keep_k;
     const int32_t xh = x_hat[(size_t)b * n + i];
     const Philox4 w = sampler_words(seed, (uint32_t)i, step, block, (uint32_t)req);
     const int32_t tok = kept ? xh : uniform_token(w.w[1], (uint32_t)vocab);
@@ -320,8 +350,11 @@ void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float*
                            int32_t* stop, int32_t* done, int32_t* out_tokens, int final_step, cudaStream_t s) {
   if (B <= 0) return;
   const int threads = ((n + 31) / 32) * 32;
-  launch_k(sampler_finish_kernel, dim3(B), dim3(threads), n * sizeof(float), s, x_hat, pmax, ent, n, vocab, req_ids, a.seed, a.step,
-                                                              a.block, a.keep_k, a.stop_threshold, canvas, keep,
+  const int keep_mode = a.keep_mode == 1 ? 1 : 0;
+  const size_t smem = (size_t)n * sizeof(float) * (keep_mode ? 2 : 1);
+  launch_k(sampler_finish_kernel, dim3(B), dim3(threads), smem, s, x_hat, pmax, ent, n, vocab, req_ids, a.seed, a.step,
+                                                              a.block, a.keep_k, keep_mode, a.entropy_budget,
+                                                              a.stop_threshold, canvas, keep,
                                                               mean_h, stop, done, out_tokens, final_step);
 }
 

@@ -75,6 +75,8 @@ struct SamplerArgs {
   uint64_t seed;
   uint32_t block;
   uint32_t step;
+  int keep_mode = 0;            // 0: top keep_k by pmax; 1: entropy budget
+  float entropy_budget = 0.f;   // nats, keep_mode 1
 };
 size_t sampler_workspace_bytes(int rows, int vocab);
 // rows = B*N logits rows; writes x_hat, pmax, H (workspace-sized arrays).

@@ -46,7 +46,12 @@ class DgWeights(C.Structure):
 
 class DgSamplerParams(C.Structure):
     _fields_ = [("temperature", C.c_float), ("logit_scale", C.c_float), ("stop_threshold", C.c_float),
-                ("keep_k", C.c_int), ("seed", C.c_uint64), ("block", C.c_uint32)]
+                ("keep_k", C.c_int), ("seed", C.c_uint64), ("block", C.c_uint32), ("keep_mode", C.c_int),
+                ("entropy_budget", C.c_float)]
+
+
+DG_KEEP_TOPK = 0
+DG_KEEP_ENTROPY_BUDGET = 1
 
 
 class DgStepOut(C.Structure):
@@ -63,7 +68,9 @@ class DgStepArgs(C.Structure):
 class DgBlockArgs(C.Structure):
     _fields_ = [("batch", C.c_int), ("req", C.POINTER(C.c_int)), ("max_steps", C.c_int),
                 ("schedule_steps", C.c_int), ("temperature", C.c_float), ("logit_scale_growth", C.c_float),
-                ("stop_threshold", C.c_float), ("seed", C.c_uint64), ("block", C.c_uint32)]
+                ("stop_threshold", C.c_float), ("seed", C.c_uint64), ("block", C.c_uint32),
+                ("keep_mode", C.c_int), ("entropy_budget", C.c_float), ("anneal", C.c_int),
+                ("temperature_end", C.c_float)]
 
 
 class DgProfileEntry(C.Structure):
@@ -210,8 +217,12 @@ def dg_get_length(h: Handle, req: int) -> int:
     return v.value
 
 
-def sampler_params(temperature=1.0, logit_scale=1.0, stop_threshold=-1.0, keep_k=0, seed=0, block=0):
-    return DgSamplerParams(temperature, logit_scale, stop_threshold, keep_k, seed, block)
+def sampler_params(temperature=1.0, logit_scale=1.0, stop_threshold=-1.0, keep_k=0, seed=0, block=0,
+                   entropy_budget=None):
+    """entropy_budget=None keeps the top keep_k by pmax; a number selects the entropy-budget keep."""
+    mode = DG_KEEP_TOPK if entropy_budget is None else DG_KEEP_ENTROPY_BUDGET
+    return DgSamplerParams(temperature, logit_scale, stop_threshold, keep_k, seed, block, mode,
+                           0.0 if entropy_budget is None else entropy_budget)
 
 
 def step_out(x_hat=None, pmax=None, entropy=None, keep=None, mean_entropy=None, stop=None, experts_touched=None):
@@ -246,9 +257,13 @@ def dg_sample_noalloc(logits, req, step, sp: DgSamplerParams, canvas, out: DgSte
 
 
 def block_args(req, max_steps, schedule_steps, temperature=1.0, logit_scale_growth=1.0, stop_threshold=-1.0,
-               seed=0, block=0):
+               seed=0, block=0, entropy_budget=None, temperature_end=None):
+    """entropy_budget: None = the k_t schedule, else the entropy-budget keep.
+    temperature_end: None = constant temperature, else the linear anneal to it."""
+    mode = DG_KEEP_TOPK if entropy_budget is None else DG_KEEP_ENTROPY_BUDGET
     return DgBlockArgs(len(req), _ints(req), max_steps, schedule_steps, temperature, logit_scale_growth,
-                       stop_threshold, seed, block)
+                       stop_threshold, seed, block, mode, 0.0 if entropy_budget is None else entropy_budget,
+                       0 if temperature_end is None else 1, 0.0 if temperature_end is None else temperature_end)
 
 
 def dg_generate_block(h: Handle, a: DgBlockArgs, out_tokens: torch.Tensor) -> int:

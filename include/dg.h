@@ -111,7 +111,19 @@ typedef struct dg_sampler_params {
   int keep_k;            /* positions kept this step (0..N) */
   uint64_t seed;         /* Philox key */
   uint32_t block;        /* Philox counter word 2 (block index) */
+  int keep_mode;         /* DG_KEEP_TOPK (0, the default when zeroed) or DG_KEEP_ENTROPY_BUDGET */
+  float entropy_budget;  /* nats, >= 0; read only by DG_KEEP_ENTROPY_BUDGET */
 } dg_sampler_params;
+
+/* Which positions a step keeps ([P1 四]).
+ * DG_KEEP_TOPK: the keep_k positions of highest pmax (ties -> lower index).
+ * DG_KEEP_ENTROPY_BUDGET: the page's entropy-ordered locking.  Positions are
+ *   taken by increasing entropy (ties -> lower index) and kept while the
+ *   running sum of their entropies, the position itself included, is
+ *   <= entropy_budget; the first position that crosses it and every later
+ *   one are re-noised.  keep_k is ignored.  The sum is taken in fp64 over the
+ *   fp32 per-position entropies. */
+enum { DG_KEEP_TOPK = 0, DG_KEEP_ENTROPY_BUDGET = 1 };
 
 /* Outputs of one sampler step; every pointer may be NULL (not written). */
 typedef struct dg_step_out {
@@ -148,6 +160,13 @@ typedef struct dg_block_args {
   float stop_threshold;       /* < 0 disables the adaptive stop */
   uint64_t seed;
   uint32_t block;
+  int keep_mode;              /* DG_KEEP_TOPK (schedule k_t) or DG_KEEP_ENTROPY_BUDGET */
+  float entropy_budget;       /* nats, for DG_KEEP_ENTROPY_BUDGET */
+  int anneal;                 /* nonzero: linear temperature anneal ([P1 四]) */
+  float temperature_end;      /* with anneal: step t runs at
+                                 T_t = T + (T_end - T) (t-1) / (max_steps-1)
+                                 (in double, then rounded to float; T_end when
+                                 max_steps == 1).  Both ends > 0. */
 } dg_block_args;
 
 /* Kernel-class timing, filled when profiling is on. */
@@ -204,10 +223,12 @@ int dg_denoise_step(dg_handle* h, const dg_step_args* a, const dg_step_out* o);
  * z = s*l/T; pmax = max softmax(z); H = entropy(softmax(z));
  * x_hat = inverse-CDF sample in vocabulary order with u from Philox word 0 of
  * counter (i, step, block, req[b]) under key seed (u = (w0 >> 8) * 2^-24);
- * keep = top keep_k positions by pmax (ties to the lower index);
+ * keep = top keep_k positions by pmax (ties to the lower index), or the
+ * entropy-budget set when sp->keep_mode is DG_KEEP_ENTROPY_BUDGET;
  * canvas[b,i] = keep ? x_hat : (w1 * V) >> 32 (uniform re-noise from word 1);
  * mean entropy and stop = mean < stop_threshold.
- * logits must be 16-byte aligned (DG_EINVAL otherwise).
+ * logits must be 16-byte aligned (DG_EINVAL otherwise); an unknown keep_mode
+ * or a negative or non-finite entropy_budget is DG_EINVAL.
  */
 int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int step,
               const dg_sampler_params* sp, int32_t* canvas, const dg_step_out* o);
@@ -259,12 +280,15 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
 
 /*
  * One block per request: canvas from Philox word 1 of counter (i, 0, block,
- * req); steps t = 1..max_steps with keep_k = ceil(N t / schedule_steps) and
- * logit scale growth^(t-1), self-conditioning on the previous x_hat; a request
+ * req); steps t = 1..max_steps with keep_k = ceil(N t / schedule_steps) (or
+ * the entropy budget, per keep_mode), logit scale growth^(t-1), temperature T
+ * or the annealed T_t, self-conditioning on the previous x_hat; a request
  * finishes at its first stop (or at max_steps) with output x_hat; the loop ends
  * when every request has finished.  Then the causal hand-off: the output tokens
  * are encoded causally and their K/V appended (P += N) ([P2], [P3]).
  * out_tokens: [B, N] device int32.  steps_used: HOST int, steps run.
+ * DG_EINVAL for an unknown keep_mode, a negative or non-finite budget, or an
+ * anneal end that is not > 0 (when anneal is set, the start must be > 0 too).
  */
 int dg_generate_block(dg_handle* h, const dg_block_args* a, int32_t* out_tokens, int* steps_used);
 

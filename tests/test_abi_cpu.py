@@ -149,6 +149,13 @@ def test_noalloc_sampler_refuses_bad_arguments_on_host(lib):
     assert _noalloc(lib, fake, 1, 4, 1024, [0], sp, fake)[0] == 1              # keep_k > n
     bad_t = B.sampler_params(temperature=-1.0, keep_k=1)
     assert _noalloc(lib, fake, 1, 256, 1024, [0], bad_t, fake)[0] == 1
+    bad_mode = B.sampler_params(temperature=1.0, keep_k=1)
+    bad_mode.keep_mode = 2
+    rc, msg = _noalloc(lib, fake, 1, 256, 1024, [0], bad_mode, fake)
+    assert rc == 1 and "keep_mode" in msg
+    for budget in (-0.5, float("nan"), float("inf")):
+        rc, msg = _noalloc(lib, fake, 1, 256, 1024, [0], B.sampler_params(entropy_budget=budget), fake)
+        assert rc == 1 and "budget" in msg
     # 64 canvases of 256 over 262144 tokens exceed the fixed scratch: capacity error, nothing launched
     rc, msg = _noalloc(lib, fake, 64, 256, 262144, list(range(64)), sp, fake)
     assert rc == 4 and "scratch" in msg
