@@ -268,7 +268,7 @@ void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const 
 // entropy; C_i = sum of H_j over r_j <= r_i (fp64) is the running sum that
 // reaches position i, and the positions kept are those ranked before the first
 // one whose C exceeds the budget (a running sum of H >= 0 only grows, so that
-// is also where it stays above).
+// is also where it stays above).  Rank 0, where locking starts, is always kept.
 __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const float* __restrict__ pmax,
                                       const float* __restrict__ ent, int n, int vocab, const int* __restrict__ req_ids,
                                       uint64_t seed, uint32_t step, uint32_t block, int keep_k, int keep_mode,
@@ -324,7 +324,7 @@ __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const f
   if (i < n) {
     int kept;
     if (keep_mode == 1) {
-      kept = hrank < sh_cut;
+      kept = hrank < max(sh_cut, 1);
     } else {
       const float p = pm[i];
       int rank = 0;

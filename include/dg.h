@@ -118,11 +118,11 @@ typedef struct dg_sampler_params {
 /* Which positions a step keeps ([P1 四]).
  * DG_KEEP_TOPK: the keep_k positions of highest pmax (ties -> lower index).
  * DG_KEEP_ENTROPY_BUDGET: the page's entropy-ordered locking.  Positions are
- *   taken by increasing entropy (ties -> lower index) and kept while the
- *   running sum of their entropies, the position itself included, is
- *   <= entropy_budget; the first position that crosses it and every later
- *   one are re-noised.  keep_k is ignored.  The sum is taken in fp64 over the
- *   fp32 per-position entropies. */
+ *   taken by increasing entropy (ties -> lower index); the first is always
+ *   kept, and each later one while the running sum of entropies, the
+ *   position itself included, is <= entropy_budget; the first position that
+ *   crosses it and every later one are re-noised.  keep_k is ignored.  The
+ *   sum is taken in fp64 over the fp32 per-position entropies. */
 enum { DG_KEEP_TOPK = 0, DG_KEEP_ENTROPY_BUDGET = 1 };
 
 /* Outputs of one sampler step; every pointer may be NULL (not written). */

@@ -46,7 +46,8 @@ Readings of points the pages leave open (each is a named reading, R-x):
   R-budget  entropy-ordered locking: positions sorted by entropy ascending
             (ties -> lower index) are kept while the inclusive cumulative
             entropy stays <= the budget (0.1); the position that crosses it and
-            all after it are re-noised.
+            all after it are re-noised.  Locking starts from the most certain
+            position, so that one is kept whatever its entropy.
   R-anneal  the temperature falls linearly from 0.8 at round 1 to 0.4 at the
             last round of the step budget.
   R-stop2   stop after round t when the mean entropy of rounds t-1 and t is
@@ -278,18 +279,19 @@ def keep_set(pmax, k):
 def keep_entropy_budget(ent, budget):
     """Entropy-ordered locking of [P1 四] (R-budget).
 
-    Positions are taken in order of increasing entropy (ties -> lower index)
-    and kept while the running sum of their entropies, this position
-    included, is <= budget.  Returns (bool mask [N], relative margin: the
-    distance of the running sum at the first rejected position from the
-    budget, inf if none is rejected)."""
+    Positions are taken in order of increasing entropy (ties -> lower index);
+    the first (most certain) one is always locked, and each later one while
+    the running sum of entropies, this position included, is <= budget.
+    Returns (bool mask [N], relative margin: the distance of the running sum
+    at the first rejected position from the budget, inf if none is
+    rejected)."""
     ent = np.asarray(ent, dtype=np.float64)
     n = len(ent)
     order = np.lexsort((np.arange(n), ent))
     keep = np.zeros(n, dtype=bool)
     run = 0.0
-    for i in order:
-        if run + ent[i] > budget:
+    for pos, i in enumerate(order):
+        if pos > 0 and run + ent[i] > budget:
             return keep, ((run + ent[i]) - budget) / max(abs(budget), 1e-300)
         run += ent[i]
         keep[i] = True

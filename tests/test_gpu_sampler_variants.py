@@ -89,6 +89,7 @@ def test_entropy_budget_keep_full_vocab(dg):
         alt = _sample(dg, g, [0], 2, sp, noalloc=True)
         for k in ("keep", "canvas", "x_hat"):
             assert np.array_equal(alt[k], got[k]), k
+    assert counts[0] == 1                          # a zero budget locks only the most certain position
     assert counts[-1] == n                         # an unbounded budget keeps every position
     assert counts == sorted(counts)                # a larger budget never keeps fewer
 

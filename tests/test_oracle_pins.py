@@ -407,7 +407,8 @@ def test_entropy_budget_keep_invariants(seed):
     for budget in (0.0, 0.05, 0.1, 0.3, 10.0):
         keep, _ = O.keep_entropy_budget(ent, budget)
         kept, rest = np.nonzero(keep)[0], np.nonzero(~keep)[0]
-        assert ent[kept].sum() <= budget + 1e-12
+        assert len(kept) >= 1                                   # the most certain position is always locked
+        assert len(kept) == 1 or ent[kept].sum() <= budget + 1e-12
         if len(rest):
             # every kept position precedes every rejected one in (entropy, index) order ...
             first = min(rest, key=lambda i: (ent[i], i))
@@ -416,7 +417,11 @@ def test_entropy_budget_keep_invariants(seed):
             assert ent[kept].sum() + ent[first] > budget
         else:
             assert ent.sum() <= budget
-    assert O.keep_entropy_budget(ent, -1.0)[0].sum() == 0
+    # a budget nothing fits keeps exactly the most certain position (ties -> lower index)
+    keep, _ = O.keep_entropy_budget(ent, -1.0)
+    assert np.nonzero(keep)[0].tolist() == [int(np.lexsort((np.arange(len(ent)), ent))[0])]
+    assert O.keep_entropy_budget([0.5, 0.2, 0.2, 0.9], 0.0)[0].tolist() == [False, True, False, False]
+    assert O.keep_entropy_budget([], 0.1)[0].size == 0
 
 
 def test_anneal_is_linear_from_08_to_04():
@@ -460,7 +465,8 @@ def test_sampler_with_entropy_budget_keeps_the_budget_set_of_its_own_entropies()
         assert np.array_equal(out["x_hat"], base["x_hat"]) and np.allclose(out["H"], base["H"])
         assert np.array_equal(out["x_new"], np.where(keep, out["x_hat"], base["renoise"]))
     assert O.sample_canvas(logits, keep_budget=1e9, **kw)["keep"].all()
-    assert not O.sample_canvas(logits, keep_budget=0.0, **kw)["keep"].any()   # every H > 0 here
+    zero = O.sample_canvas(logits, keep_budget=0.0, **kw)                    # every H > 0 here
+    assert np.nonzero(zero["keep"])[0].tolist() == [int(np.argmin(zero["H"]))]
 
 
 def test_block_with_anneal_runs_each_step_at_the_annealed_temperature():
@@ -486,6 +492,6 @@ def test_block_with_anneal_runs_each_step_at_the_annealed_temperature():
     a = run(temperature_end=0.8)
     b = run()
     assert a[1] == b[1] and np.array_equal(a[0], b[0])
-    # the budget keep plugs into the block: a budget of 0 keeps nothing until the last step's output
+    # the budget keep plugs into the block: a budget of 0 locks one position a step
     toks, steps, trace = run(keep_budget=0.0)
-    assert all(not r["keep"].any() for r in trace) and np.array_equal(toks, trace[-1]["x_hat"])
+    assert all(r["keep"].sum() == 1 for r in trace) and np.array_equal(toks, trace[-1]["x_hat"])
