@@ -190,6 +190,8 @@ struct dg_handle {
   // sampler workspace
   void* sws = nullptr;
   int32_t* xh[2] = {nullptr, nullptr};
+  int32_t* amax[2] = {nullptr, nullptr};   // argmax rows of two rounds (two-round stop)
+  float* mh2[2] = {nullptr, nullptr};      // mean entropies of two rounds (two-round stop)
   float* pmax = nullptr;
   float* ent = nullptr;
   int32_t* keep = nullptr;
@@ -796,6 +798,9 @@ SamplerArgs sampler_args(const dg_sampler_params& sp, int step) {
   a.step = (uint32_t)step;
   a.keep_mode = sp.keep_mode;
   a.entropy_budget = sp.entropy_budget;
+  a.stop_mode = sp.stop_mode;
+  a.prev_argmax = sp.prev_argmax;
+  a.prev_mean_h = sp.prev_mean_entropy;
   return a;
 }
 
@@ -809,22 +814,24 @@ int check_sampler_params(dg_handle* H, const dg_sampler_params* sp) {
     return fail(H, DG_EINVAL, "unknown keep_mode %d", sp->keep_mode);
   if (sp->keep_mode == DG_KEEP_ENTROPY_BUDGET && !(sp->entropy_budget >= 0.f && std::isfinite(sp->entropy_budget)))
     return fail(H, DG_EINVAL, "entropy_budget must be finite and >= 0");
+  if (sp->stop_mode != DG_STOP_MEAN_ENTROPY && sp->stop_mode != DG_STOP_TWO_ROUNDS)
+    return fail(H, DG_EINVAL, "unknown stop_mode %d", sp->stop_mode);
   return DG_OK;
 }
 
 // sampler over logits rows of the batch, then keep / re-noise / stop
 void run_sampler(dg_handle* H, const float* logits, const BatchInfo& bi, const SamplerArgs& a, int32_t* canvas,
                  int32_t* xh, float* pmax, float* ent, int32_t* keep, float* meanh, int32_t* stop, int32_t* done,
-                 int32_t* out_tokens, int final_step) {
+                 int32_t* out_tokens, int final_step, int32_t* argmax) {
   const int n = H->c.canvas;
   {
     ProfScope ps(H, PC_SAMPLER, 2);
-    launch_sampler_rows(logits, bi.B * n, n, H->c.vocab, H->req_dev, a, H->sws, xh, pmax, ent, H->stream);
+    launch_sampler_rows(logits, bi.B * n, n, H->c.vocab, H->req_dev, a, H->sws, xh, pmax, ent, H->stream, argmax);
   }
   {
     ProfScope ps(H, PC_FINISH);
     launch_sampler_finish(xh, pmax, ent, bi.B, n, H->c.vocab, H->req_dev, a, canvas, keep, meanh, stop, done,
-                          out_tokens, final_step, H->stream);
+                          out_tokens, final_step, H->stream, argmax);
   }
 }
 
@@ -961,6 +968,10 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
   H->sws = dalloc<char>(sampler_workspace_bytes(nrow, c.vocab), &ok);
   H->xh[0] = dalloc<int32_t>(nrow, &ok);
   H->xh[1] = dalloc<int32_t>(nrow, &ok);
+  H->amax[0] = dalloc<int32_t>(nrow, &ok);
+  H->amax[1] = dalloc<int32_t>(nrow, &ok);
+  H->mh2[0] = dalloc<float>(c.max_batch, &ok);
+  H->mh2[1] = dalloc<float>(c.max_batch, &ok);
   H->pmax = dalloc<float>(nrow, &ok);
   H->ent = dalloc<float>(nrow, &ok);
   H->keep = dalloc<int32_t>(nrow, &ok);
@@ -1058,7 +1069,8 @@ void dg_destroy(dg_handle* H) {
   void* ps[] = {H->kc, H->vt, H->h, H->xn, H->eprev, H->qkv, H->q, H->attn, H->glog, H->ids, H->wts, H->cnt,
                 H->off, H->perm, H->work, H->n_work, H->touched, H->xp, H->hb, H->y, H->logits, H->rope, H->sws,
                 H->xh[0], H->xh[1], H->pmax, H->ent, H->keep, H->meanh, H->stop, H->done, H->canvas, H->out_tok,
-                H->req_dev, H->tok_ws, H->d_err, H->part_o, H->part_ml, H->kpart};
+                H->req_dev, H->tok_ws, H->d_err, H->part_o, H->part_ml, H->kpart, H->amax[0], H->amax[1],
+                H->mh2[0], H->mh2[1]};
   for (void* p : ps)
     if (p) cudaFree(p);
   if (H->h_done) cudaFreeHost(H->h_done);
@@ -1113,6 +1125,12 @@ int dg_prefill_prompt(dg_handle* H, int batch, const int* req, const int32_t* to
   return encode_causal(H, bi, tokens, n, n);
 }
 
+// where a step writes its argmax rows: the caller's buffer, else (the two-round stop needs them) the handle's
+static int32_t* argmax_target(dg_handle* H, const SamplerArgs& a, const dg_step_out* o) {
+  if (o && o->argmax) return o->argmax;
+  return a.stop_mode == DG_STOP_TWO_ROUNDS ? H->amax[0] : nullptr;
+}
+
 int dg_sample(dg_handle* H, const float* logits, int batch, const int* req, int step, const dg_sampler_params* sp,
               int32_t* canvas, const dg_step_out* o) {
   if (!H) return DG_EINVAL;
@@ -1126,7 +1144,7 @@ int dg_sample(dg_handle* H, const float* logits, int batch, const int* req, int 
   const SamplerArgs a = sampler_args(*sp, step);
   run_sampler(H, logits, bi, a, canvas, (o && o->x_hat) ? o->x_hat : H->xh[0], (o && o->pmax) ? o->pmax : H->pmax,
               (o && o->entropy) ? o->entropy : H->ent, o ? o->keep : nullptr, o ? o->mean_entropy : nullptr,
-              o ? o->stop : nullptr, nullptr, nullptr, 0);
+              o ? o->stop : nullptr, nullptr, nullptr, 0, argmax_target(H, a, o));
   return check_launch(H, "sample");
 }
 
@@ -1149,7 +1167,7 @@ int dg_denoise_step(dg_handle* H, const dg_step_args* a, const dg_step_out* o) {
   const SamplerArgs sa = sampler_args(a->sp, a->step);
   run_sampler(H, logits, bi, sa, a->canvas, (o && o->x_hat) ? o->x_hat : H->xh[0],
               (o && o->pmax) ? o->pmax : H->pmax, (o && o->entropy) ? o->entropy : H->ent, o ? o->keep : nullptr,
-              o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0);
+              o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0, argmax_target(H, sa, o));
   if (o && o->experts_touched)
     cudaMemcpyAsync(o->experts_touched, H->touched, c.n_layers * sizeof(int32_t), cudaMemcpyDeviceToDevice,
                     H->stream);
@@ -1171,6 +1189,9 @@ static int generate_block_impl(dg_handle* H, const dg_block_args* a, int32_t* ou
     return fail(H, DG_EINVAL, "unknown keep_mode %d", a->keep_mode);
   if (a->keep_mode == DG_KEEP_ENTROPY_BUDGET && !(a->entropy_budget >= 0.f && std::isfinite(a->entropy_budget)))
     return fail(H, DG_EINVAL, "entropy_budget must be finite and >= 0");
+  if (a->stop_mode != DG_STOP_MEAN_ENTROPY && a->stop_mode != DG_STOP_TWO_ROUNDS)
+    return fail(H, DG_EINVAL, "unknown stop_mode %d", a->stop_mode);
+  const bool two_rounds = a->stop_mode == DG_STOP_TWO_ROUNDS;
   for (int b = 0; b < bi.B; ++b)
     if (bi.len[b] + c.canvas > c.max_ctx) return fail(H, DG_ECAPACITY, "cache + canvas exceeds max_ctx");
   if ((rc = upload_req(H, bi))) return rc;
@@ -1198,11 +1219,16 @@ static int generate_block_impl(dg_handle* H, const dg_block_args* a, int32_t* ou
     sp.block = a->block;
     sp.keep_mode = a->keep_mode;
     sp.entropy_budget = a->entropy_budget;
+    // the two-round stop compares with the previous round's argmax and mean entropy (double-buffered)
+    sp.stop_mode = a->stop_mode;
+    sp.prev_argmax = (two_rounds && t > 1) ? H->amax[(t - 1) & 1] : nullptr;
+    sp.prev_mean_entropy = (two_rounds && t > 1) ? H->mh2[(t - 1) & 1] : nullptr;
     if ((rc = check_sampler_params(H, &sp))) return rc;
     run_layers(H, bi, n, false, H->canvas, prev, true, H->logits, nullptr);
     int32_t* xh = H->xh[t & 1];
-    run_sampler(H, H->logits, bi, sampler_args(sp, t), H->canvas, xh, H->pmax, H->ent, H->keep, H->meanh, H->stop,
-                H->done, out_dev, t == a->max_steps ? 1 : 0);
+    run_sampler(H, H->logits, bi, sampler_args(sp, t), H->canvas, xh, H->pmax, H->ent, H->keep,
+                two_rounds ? H->mh2[t & 1] : H->meanh, H->stop, H->done, out_dev, t == a->max_steps ? 1 : 0,
+                two_rounds ? H->amax[t & 1] : nullptr);
     if ((rc = check_launch(H, "block step"))) return rc;
     steps = t;
     cudaMemcpyAsync(H->h_done, H->done, bi.B * sizeof(int32_t), cudaMemcpyDeviceToHost, H->stream);

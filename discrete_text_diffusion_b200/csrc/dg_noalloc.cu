@@ -70,13 +70,16 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
     return report(err, err_len, DG_EINVAL, "unknown keep_mode %d", sp->keep_mode);
   if (sp->keep_mode == DG_KEEP_ENTROPY_BUDGET && !(sp->entropy_budget >= 0.f && std::isfinite(sp->entropy_budget)))
     return report(err, err_len, DG_EINVAL, "entropy_budget must be finite and >= 0");
+  if (sp->stop_mode != DG_STOP_MEAN_ENTROPY && sp->stop_mode != DG_STOP_TWO_ROUNDS)
+    return report(err, err_len, DG_EINVAL, "unknown stop_mode %d", sp->stop_mode);
 
-  // scratch layout: request ids | x_hat | pmax | entropy | chunk partials
+  // scratch layout: request ids | x_hat | pmax | entropy | argmax | chunk partials
   const size_t rows = (size_t)batch * n;
   const size_t off_xh = round256(kMaxReq * sizeof(int32_t));
   const size_t off_pm = off_xh + round256(rows * sizeof(int32_t));
   const size_t off_en = off_pm + round256(rows * sizeof(float));
-  const size_t off_ws = off_en + round256(rows * sizeof(float));
+  const size_t off_am = off_en + round256(rows * sizeof(float));
+  const size_t off_ws = off_am + round256(rows * sizeof(int32_t));
   const size_t need = off_ws + round256(sampler_workspace_bytes((int)rows, vocab));
   if (need > kScratchBytes)
     return report(err, err_len, DG_ECAPACITY,
@@ -122,9 +125,15 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
   a.step = (uint32_t)step;
   a.keep_mode = sp->keep_mode;
   a.entropy_budget = sp->entropy_budget;
-  launch_sampler_rows(logits, (int)rows, n, vocab, req_dev, a, base + off_ws, xh, pmax, ent, s);
+  a.stop_mode = sp->stop_mode;
+  a.prev_argmax = sp->prev_argmax;
+  a.prev_mean_h = sp->prev_mean_entropy;
+  int32_t* amax = (o && o->argmax) ? o->argmax
+                                   : (sp->stop_mode == DG_STOP_TWO_ROUNDS ? reinterpret_cast<int32_t*>(base + off_am)
+                                                                          : nullptr);
+  launch_sampler_rows(logits, (int)rows, n, vocab, req_dev, a, base + off_ws, xh, pmax, ent, s, amax);
   launch_sampler_finish(xh, pmax, ent, batch, n, vocab, req_dev, a, canvas, o ? o->keep : nullptr,
-                        o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0, s);
+                        o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0, s, amax);
   e = cudaGetLastError();
   if (e != cudaSuccess) return report(err, err_len, DG_ECUDA, "sampler launch: %s", cudaGetErrorString(e));
   return DG_OK;

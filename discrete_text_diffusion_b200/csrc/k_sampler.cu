@@ -10,6 +10,8 @@
 // in vocabulary order.
 // Pass 3: one CTA per canvas ranks positions by pmax, keeps the top-k,
 // re-noises the rest with Philox, and forms the mean entropy / stop flag.
+// On request, passes 1 and 2 also carry the first arg-max of z per row, for
+// the two-round stop.
 #include <curand_kernel.h>
 
 #include "dg_common.cuh"
@@ -23,7 +25,7 @@ constexpr int kPerThread = kChunk / kThreads;  // 16
 
 struct Partial {
   float m;    // chunk max of z (T > 0) / of the scaled logit (T == 0)
-  int idx;    // T == 0: first arg-max index in the chunk
+  int idx;    // first arg-max index in the chunk (T == 0, or when requested; else 0)
   double s;   // sum exp(z - m)             | T == 0: count of maxima
   double a;   // sum exp(z - m) * (z - m)
 };
@@ -70,7 +72,7 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 // in fp64 so the CDF that decides the sample is not limited by fp32 rounding
 // of 262144-term sums.
 __global__ void __launch_bounds__(kThreads) sampler_pass1(const float* __restrict__ logits, int vocab, float scale,
-                                                          int argmax_mode, Partial* __restrict__ part) {
+                                                          int argmax_mode, int want_idx, Partial* __restrict__ part) {
   pdl_wait();
   pdl_trigger();
   __shared__ float red_m[kThreads / 32];
@@ -117,6 +119,22 @@ __global__ void __launch_bounds__(kThreads) sampler_pass1(const float* __restric
     }
     return;
   }
+  int first = 0;
+  if (want_idx) {  // uniform over the block
+    int best = 0x7fffffff;
+#pragma unroll
+    for (int r = 0; r < kPerThread; ++r) {
+      const int j = reg_index(c0, r, vec4);
+      if (z[r] == m && j < vocab) best = min(best, j);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if (lane == 0) red_i[w] = best;
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int x = 0; x < kThreads / 32; ++x) best = min(best, red_i[x]);
+    first = best;
+  }
   double s = 0.0, a = 0.0;
   if (m > -INFINITY) {
 #pragma unroll
@@ -134,7 +152,7 @@ __global__ void __launch_bounds__(kThreads) sampler_pass1(const float* __restric
   if (threadIdx.x == 0) {
     s = 0.0; a = 0.0;
     for (int x = 0; x < kThreads / 32; ++x) { s += red_s[x]; a += red_a[x]; }
-    p.m = m; p.idx = 0; p.s = s; p.a = a;
+    p.m = m; p.idx = first; p.s = s; p.a = a;
     part[(size_t)row * n_chunks + c] = p;
   }
 }
@@ -143,7 +161,8 @@ __global__ void __launch_bounds__(kThreads) sampler_pass2(const float* __restric
                                                           float scale, int argmax_mode, const int* __restrict__ req_ids,
                                                           uint64_t seed, uint32_t step, uint32_t block,
                                                           const Partial* __restrict__ part, int32_t* __restrict__ x_hat,
-                                                          float* __restrict__ pmax, float* __restrict__ ent) {
+                                                          float* __restrict__ pmax, float* __restrict__ ent,
+                                                          int32_t* __restrict__ argmax) {
   pdl_wait();
   pdl_trigger();
   __shared__ float sh_M;
@@ -169,6 +188,7 @@ __global__ void __launch_bounds__(kThreads) sampler_pass2(const float* __restric
           cntm += pr[c].s;
         }
       x_hat[row] = idx;
+      if (argmax) argmax[row] = idx;
       pmax[row] = (float)(1.0 / cntm);
       ent[row] = (float)log(cntm);
     }
@@ -177,6 +197,12 @@ __global__ void __launch_bounds__(kThreads) sampler_pass2(const float* __restric
   if (threadIdx.x == 0) {
     float M = -INFINITY;
     for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pr[c].m);
+    if (argmax) {  // chunks are in vocabulary order: the first holding M has the first arg-max
+      int idx = -1;
+      for (int c = 0; c < n_chunks && idx < 0; ++c)
+        if (pr[c].m == M) idx = pr[c].idx;
+      argmax[row] = idx;
+    }
     double S = 0.0, A = 0.0;
     for (int c = 0; c < n_chunks; ++c) {
       const double f = exp((double)pr[c].m - (double)M);
@@ -251,15 +277,17 @@ __global__ void __launch_bounds__(kThreads) sampler_pass2(const float* __restric
 }
 
 void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const int* req_ids, const SamplerArgs& a,
-                         void* ws, int32_t* x_hat, float* pmax, float* ent, cudaStream_t s) {
+                         void* ws, int32_t* x_hat, float* pmax, float* ent, cudaStream_t s, int32_t* argmax) {
   if (rows <= 0) return;
   const int n_chunks = (vocab + kChunk - 1) / kChunk;
   const int argmax_mode = a.temperature == 0.f;
   const float scale = argmax_mode ? a.logit_scale : a.logit_scale / a.temperature;
   Partial* part = reinterpret_cast<Partial*>(ws);
-  launch_k(sampler_pass1, dim3(dim3(n_chunks, rows)), dim3(kThreads), 0, s, logits, vocab, scale, argmax_mode, part);
+  const int want_idx = (argmax != nullptr && !argmax_mode) ? 1 : 0;
+  launch_k(sampler_pass1, dim3(dim3(n_chunks, rows)), dim3(kThreads), 0, s, logits, vocab, scale, argmax_mode, want_idx,
+           part);
   launch_k(sampler_pass2, dim3(rows), dim3(kThreads), 0, s, logits, n, vocab, scale, argmax_mode, req_ids, a.seed, a.step, a.block,
-                                          part, x_hat, pmax, ent);
+                                          part, x_hat, pmax, ent, argmax);
 }
 
 // Pass 3: per canvas.  Top-k keep: rank_i = #{j : pmax_j > pmax_i or
@@ -269,10 +297,15 @@ void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const 
 // reaches position i, and the positions kept are those ranked before the first
 // one whose C exceeds the budget (a running sum of H >= 0 only grows, so that
 // is also where it stays above).  Rank 0, where locking starts, is always kept.
+// Two-round stop: this round's and the previous round's mean entropies below
+// the threshold and every position's arg-max unchanged; no previous round, no
+// stop.
 __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const float* __restrict__ pmax,
                                       const float* __restrict__ ent, int n, int vocab, const int* __restrict__ req_ids,
                                       uint64_t seed, uint32_t step, uint32_t block, int keep_k, int keep_mode,
-                                      float budget, float stop_thr,
+                                      float budget, float stop_thr, int stop_mode,
+                                      const int32_t* __restrict__ amax_cur, const int32_t* __restrict__ amax_prev,
+                                      const float* __restrict__ mh_prev,
                                       int32_t* __restrict__ canvas, int32_t* __restrict__ keep_out,
                                       float* __restrict__ mean_h, int32_t* __restrict__ stop_out,
                                       int32_t* __restrict__ done, int32_t* __restrict__ out_tokens, int final_step) {
@@ -293,6 +326,12 @@ __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const f
   if (i == 0) sh_cut = n;
   const int was_done = (done != nullptr) ? done[b] : 0;
   __syncthreads();
+  int same = 1;
+  if (stop_mode == 1) {  // uniform over the block
+    int eq = 1;
+    if (amax_prev != nullptr && i < n) eq = amax_cur[(size_t)b * n + i] == amax_prev[(size_t)b * n + i];
+    same = __syncthreads_and(eq);
+  }
   int hrank = 0;
   if (keep_mode == 1 && i < n) {
     const float h = eh[i];
@@ -315,7 +354,12 @@ __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const f
     float t = 0.f;
     for (int x = 0; x < (int)((blockDim.x + 31) >> 5); ++x) t += red[x];
     const float mh = t / (float)n;
-    const int st = (stop_thr >= 0.f && mh < stop_thr) ? 1 : 0;
+    int st;
+    if (stop_mode == 1)
+      st = (stop_thr >= 0.f && amax_prev != nullptr && mh_prev != nullptr && mh_prev[b] < stop_thr &&
+            mh < stop_thr && same) ? 1 : 0;
+    else
+      st = (stop_thr >= 0.f && mh < stop_thr) ? 1 : 0;
     if (mean_h) mean_h[b] = mh;
     if (stop_out) stop_out[b] = st;
     sh_stop = st;
@@ -347,14 +391,17 @@ __global__ void sampler_finish_kernel(const int32_t* __restrict__ x_hat, const f
 
 void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float* ent, int B, int n, int vocab,
                            const int* req_ids, const SamplerArgs& a, int32_t* canvas, int32_t* keep, float* mean_h,
-                           int32_t* stop, int32_t* done, int32_t* out_tokens, int final_step, cudaStream_t s) {
+                           int32_t* stop, int32_t* done, int32_t* out_tokens, int final_step, cudaStream_t s,
+                           const int32_t* argmax) {
   if (B <= 0) return;
   const int threads = ((n + 31) / 32) * 32;
   const int keep_mode = a.keep_mode == 1 ? 1 : 0;
+  const int stop_mode = (a.stop_mode == 1 && argmax != nullptr) ? 1 : 0;
   const size_t smem = (size_t)n * sizeof(float) * (keep_mode ? 2 : 1);
   launch_k(sampler_finish_kernel, dim3(B), dim3(threads), smem, s, x_hat, pmax, ent, n, vocab, req_ids, a.seed, a.step,
                                                               a.block, a.keep_k, keep_mode, a.entropy_budget,
-                                                              a.stop_threshold, canvas, keep,
+                                                              a.stop_threshold, stop_mode, argmax, a.prev_argmax,
+                                                              a.prev_mean_h, canvas, keep,
                                                               mean_h, stop, done, out_tokens, final_step);
 }
 

@@ -77,17 +77,22 @@ struct SamplerArgs {
   uint32_t step;
   int keep_mode = 0;            // 0: top keep_k by pmax; 1: entropy budget
   float entropy_budget = 0.f;   // nats, keep_mode 1
+  int stop_mode = 0;            // 0: mean entropy; 1: two rounds (mean entropies and argmax)
+  const int32_t* prev_argmax = nullptr;   // stop_mode 1: previous round [B, N], or null
+  const float* prev_mean_h = nullptr;     // stop_mode 1: previous round [B], or null
 };
 size_t sampler_workspace_bytes(int rows, int vocab);
-// rows = B*N logits rows; writes x_hat, pmax, H (workspace-sized arrays).
+// rows = B*N logits rows; writes x_hat, pmax, H (workspace-sized arrays) and,
+// when argmax is not null, the argmax of z per row (ties -> lower index).
 void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const int* req_ids,
                          const SamplerArgs& a, void* ws, int32_t* x_hat, float* pmax, float* ent,
-                         cudaStream_t s);
+                         cudaStream_t s, int32_t* argmax = nullptr);
 // Per canvas: keep set, re-noise, mean entropy, stop; optional block-loop outputs.
+// argmax: this round's argmax rows (required by stop_mode 1).
 void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float* ent, int B, int n,
                            int vocab, const int* req_ids, const SamplerArgs& a, int32_t* canvas,
                            int32_t* keep, float* mean_h, int32_t* stop, int32_t* done, int32_t* out_tokens,
-                           int final_step, cudaStream_t s);
+                           int final_step, cudaStream_t s, const int32_t* argmax = nullptr);
 
 // ---- GEMMs
 enum Epi { EPI_STORE_F32 = 0, EPI_ADD_F32 = 1, EPI_STORE_ACT = 2, EPI_SWIGLU_ACT = 3, EPI_SCATTER_ACT = 4 };

@@ -47,16 +47,19 @@ class DgWeights(C.Structure):
 class DgSamplerParams(C.Structure):
     _fields_ = [("temperature", C.c_float), ("logit_scale", C.c_float), ("stop_threshold", C.c_float),
                 ("keep_k", C.c_int), ("seed", C.c_uint64), ("block", C.c_uint32), ("keep_mode", C.c_int),
-                ("entropy_budget", C.c_float)]
+                ("entropy_budget", C.c_float), ("stop_mode", C.c_int), ("prev_argmax", C.c_void_p),
+                ("prev_mean_entropy", C.c_void_p)]
 
 
 DG_KEEP_TOPK = 0
 DG_KEEP_ENTROPY_BUDGET = 1
+DG_STOP_MEAN_ENTROPY = 0
+DG_STOP_TWO_ROUNDS = 1
 
 
 class DgStepOut(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("x_hat", "pmax", "entropy", "keep", "mean_entropy", "stop",
-                                          "experts_touched")]
+                                          "experts_touched", "argmax")]
 
 
 class DgStepArgs(C.Structure):
@@ -70,7 +73,7 @@ class DgBlockArgs(C.Structure):
                 ("schedule_steps", C.c_int), ("temperature", C.c_float), ("logit_scale_growth", C.c_float),
                 ("stop_threshold", C.c_float), ("seed", C.c_uint64), ("block", C.c_uint32),
                 ("keep_mode", C.c_int), ("entropy_budget", C.c_float), ("anneal", C.c_int),
-                ("temperature_end", C.c_float)]
+                ("temperature_end", C.c_float), ("stop_mode", C.c_int)]
 
 
 class DgProfileEntry(C.Structure):
@@ -218,16 +221,22 @@ def dg_get_length(h: Handle, req: int) -> int:
 
 
 def sampler_params(temperature=1.0, logit_scale=1.0, stop_threshold=-1.0, keep_k=0, seed=0, block=0,
-                   entropy_budget=None):
-    """entropy_budget=None keeps the top keep_k by pmax; a number selects the entropy-budget keep."""
+                   entropy_budget=None, two_round_stop=False, prev_argmax=None, prev_mean_entropy=None):
+    """entropy_budget=None keeps the top keep_k by pmax; a number selects the entropy-budget keep.
+    two_round_stop selects the stop on two rounds' mean entropies and argmax; prev_argmax [B, N] int32 and
+    prev_mean_entropy [B] float32 (device tensors) are the previous round's outputs, None at the first round."""
     mode = DG_KEEP_TOPK if entropy_budget is None else DG_KEEP_ENTROPY_BUDGET
     return DgSamplerParams(temperature, logit_scale, stop_threshold, keep_k, seed, block, mode,
-                           0.0 if entropy_budget is None else entropy_budget)
+                           0.0 if entropy_budget is None else entropy_budget,
+                           DG_STOP_TWO_ROUNDS if two_round_stop else DG_STOP_MEAN_ENTROPY,
+                           None if prev_argmax is None else prev_argmax.data_ptr(),
+                           None if prev_mean_entropy is None else prev_mean_entropy.data_ptr())
 
 
-def step_out(x_hat=None, pmax=None, entropy=None, keep=None, mean_entropy=None, stop=None, experts_touched=None):
+def step_out(x_hat=None, pmax=None, entropy=None, keep=None, mean_entropy=None, stop=None, experts_touched=None,
+             argmax=None):
     return DgStepOut(*[None if t is None else t.data_ptr() for t in
-                       (x_hat, pmax, entropy, keep, mean_entropy, stop, experts_touched)])
+                       (x_hat, pmax, entropy, keep, mean_entropy, stop, experts_touched, argmax)])
 
 
 def dg_denoise_step(h: Handle, req, canvas, prev_pred, step, sp: DgSamplerParams, out: DgStepOut,
@@ -257,13 +266,15 @@ def dg_sample_noalloc(logits, req, step, sp: DgSamplerParams, canvas, out: DgSte
 
 
 def block_args(req, max_steps, schedule_steps, temperature=1.0, logit_scale_growth=1.0, stop_threshold=-1.0,
-               seed=0, block=0, entropy_budget=None, temperature_end=None):
+               seed=0, block=0, entropy_budget=None, temperature_end=None, two_round_stop=False):
     """entropy_budget: None = the k_t schedule, else the entropy-budget keep.
-    temperature_end: None = constant temperature, else the linear anneal to it."""
+    temperature_end: None = constant temperature, else the linear anneal to it.
+    two_round_stop: stop on two rounds' mean entropies (< stop_threshold) and an unchanged argmax."""
     mode = DG_KEEP_TOPK if entropy_budget is None else DG_KEEP_ENTROPY_BUDGET
     return DgBlockArgs(len(req), _ints(req), max_steps, schedule_steps, temperature, logit_scale_growth,
                        stop_threshold, seed, block, mode, 0.0 if entropy_budget is None else entropy_budget,
-                       0 if temperature_end is None else 1, 0.0 if temperature_end is None else temperature_end)
+                       0 if temperature_end is None else 1, 0.0 if temperature_end is None else temperature_end,
+                       DG_STOP_TWO_ROUNDS if two_round_stop else DG_STOP_MEAN_ENTROPY)
 
 
 def dg_generate_block(h: Handle, a: DgBlockArgs, out_tokens: torch.Tensor) -> int:

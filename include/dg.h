@@ -113,7 +113,23 @@ typedef struct dg_sampler_params {
   uint32_t block;        /* Philox counter word 2 (block index) */
   int keep_mode;         /* DG_KEEP_TOPK (0, the default when zeroed) or DG_KEEP_ENTROPY_BUDGET */
   float entropy_budget;  /* nats, >= 0; read only by DG_KEEP_ENTROPY_BUDGET */
+  int stop_mode;         /* DG_STOP_MEAN_ENTROPY (0, the default) or DG_STOP_TWO_ROUNDS */
+  const int32_t* prev_argmax;      /* DG_STOP_TWO_ROUNDS: device [B, N], the previous round's argmax
+                                      output, or NULL at the first round */
+  const float* prev_mean_entropy;  /* DG_STOP_TWO_ROUNDS: device [B], the previous round's mean
+                                      entropy, or NULL at the first round */
 } dg_sampler_params;
+
+/* The stop test of a round ([P1 四]).
+ * DG_STOP_MEAN_ENTROPY: stop when this round's mean entropy < stop_threshold.
+ * DG_STOP_TWO_ROUNDS: the page's adaptive stop.  Stop when this round's and
+ *   the previous round's mean entropies are both < stop_threshold (0.005 on
+ *   the page) and this round's argmax sequence equals the previous round's.
+ *   The argmax is that of z = s*l/T in fp32 (ties -> lower index; for T == 0
+ *   it is x_hat).  A round without a previous round (prev_* NULL) does not
+ *   stop.
+ * stop_threshold < 0 disables either test. */
+enum { DG_STOP_MEAN_ENTROPY = 0, DG_STOP_TWO_ROUNDS = 1 };
 
 /* Which positions a step keeps ([P1 四]).
  * DG_KEEP_TOPK: the keep_k positions of highest pmax (ties -> lower index).
@@ -134,6 +150,8 @@ typedef struct dg_step_out {
   float* mean_entropy;       /* [B] */
   int32_t* stop;             /* [B] 1 = stop test passed */
   int32_t* experts_touched;  /* [n_layers] distinct experts routed to */
+  int32_t* argmax;           /* [B, N] argmax of z (ties -> lower index); pass it as the next
+                                round's prev_argmax for DG_STOP_TWO_ROUNDS */
 } dg_step_out;
 
 /* One denoising step ([P1 一/二/四]). */
@@ -167,6 +185,8 @@ typedef struct dg_block_args {
                                  T_t = T + (T_end - T) (t-1) / (max_steps-1)
                                  (in double, then rounded to float; T_end when
                                  max_steps == 1).  Both ends > 0. */
+  int stop_mode;              /* DG_STOP_MEAN_ENTROPY or DG_STOP_TWO_ROUNDS (the loop keeps
+                                 the previous round's argmax and mean entropy) */
 } dg_block_args;
 
 /* Kernel-class timing, filled when profiling is on. */
@@ -228,7 +248,8 @@ int dg_denoise_step(dg_handle* h, const dg_step_args* a, const dg_step_out* o);
  * canvas[b,i] = keep ? x_hat : (w1 * V) >> 32 (uniform re-noise from word 1);
  * mean entropy and stop = mean < stop_threshold.
  * logits must be 16-byte aligned (DG_EINVAL otherwise); an unknown keep_mode
- * or a negative or non-finite entropy_budget is DG_EINVAL.
+ * or stop_mode, or a negative or non-finite entropy_budget, is DG_EINVAL.
+ * With DG_STOP_TWO_ROUNDS the stop follows that mode's definition.
  */
 int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int step,
               const dg_sampler_params* sp, int32_t* canvas, const dg_step_out* o);
@@ -252,15 +273,16 @@ int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int 
  *   n: canvas length, 1..1024.
  *   step, sp: as for dg_sample; sp->keep_k <= n.
  *   canvas: device [batch, n]; in: unused, out: the re-noised canvas.
- *   o: as for dg_sample, or NULL.  x_hat / pmax / entropy that o does not
- *      request are kept in the scratch; experts_touched is ignored.
+ *   o: as for dg_sample, or NULL.  x_hat / pmax / entropy (and the argmax a
+ *      two-round stop needs) that o does not request are kept in the
+ *      scratch; experts_touched is ignored.
  *   stream: a cudaStream_t of the current device (NULL = legacy default).
  *   err: buffer of err_len bytes for a message (may be NULL).
  *
  * Limits and behaviour:
  *   - The request must fit the scratch:
- *     ceil(vocab / 4096) * 24 bytes per row of logits, plus ~12 bytes per row
- *     and 1 KB.  At vocab = 262144 that is about 5400 rows (21 canvases of 256).
+ *     ceil(vocab / 4096) * 24 bytes per row of logits, plus ~16 bytes per row
+ *     and 1.3 KB.  At vocab = 262144 that is about 5400 rows (21 canvases of 256).
  *     A larger request returns DG_ECAPACITY before anything is launched.
  *   - The first call on a device does the setup (looks up the scratch's
  *     address, loading the module if needed); make it before any stream capture.
@@ -287,8 +309,9 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
  * when every request has finished.  Then the causal hand-off: the output tokens
  * are encoded causally and their K/V appended (P += N) ([P2], [P3]).
  * out_tokens: [B, N] device int32.  steps_used: HOST int, steps run.
- * DG_EINVAL for an unknown keep_mode, a negative or non-finite budget, or an
- * anneal end that is not > 0 (when anneal is set, the start must be > 0 too).
+ * DG_EINVAL for an unknown keep_mode or stop_mode, a negative or non-finite
+ * budget, or an anneal end that is not > 0 (when anneal is set, the start
+ * must be > 0 too).
  */
 int dg_generate_block(dg_handle* h, const dg_block_args* a, int32_t* out_tokens, int* steps_used);
 

@@ -41,8 +41,7 @@ Readings of points the pages leave open (each is a named reading, R-x):
             softmax over the k selected logits.
   R-append  a finished canvas is appended by one causal encode pass over its
             tokens (no self-conditioning).
-  The page's own sampler variants ([P1 四]; the CUDA path has R-budget and
-  R-anneal, R-stop2 is here only):
+  The page's own sampler variants ([P1 四]; the CUDA path has all three):
   R-budget  entropy-ordered locking: positions sorted by entropy ascending
             (ties -> lower index) are kept while the inclusive cumulative
             entropy stays <= the budget (0.1); the position that crosses it and
@@ -323,8 +322,10 @@ def sample_canvas(logits, *, seed, step, block, req, temperature, logit_scale,
                   keep_k, stop_threshold, keep_budget=None):
     """Sampler for one canvas: stats, Philox sample, keep, re-noise, stop.
 
-    logits [N, V].  Returns dict with x_hat, pmax, H, keep, x_new, mean_H, stop
-    and the decision margins (sample_margin [N], keep_margin, stop_margin).
+    logits [N, V].  Returns dict with x_hat, pmax, H, keep, x_new, mean_H, stop,
+    argmax (of z, ties -> lower index) and the decision margins (sample_margin
+    [N], keep_margin, stop_margin, argmax_margin [N]: the gap between the two
+    largest z relative to max(|z_max|, 1)).
     stop_threshold < 0 disables the stop test.  keep_budget=None keeps the
     keep_k most confident positions; a number keeps the entropy-budget set
     (R-budget) and ignores keep_k.
@@ -337,9 +338,14 @@ def sample_canvas(logits, *, seed, step, block, req, temperature, logit_scale,
     pmax = np.empty(n)
     ent = np.empty(n)
     smargin = np.empty(n)
+    amax = np.empty(n, dtype=np.int64)
+    amargin = np.empty(n)
     for i in range(n):
         st = position_stats(logits[i], temperature, logit_scale)
         pmax[i], ent[i] = st["pmax"], st["H"]
+        amax[i] = argmax_tokens(st["z"])
+        top2 = np.sort(st["z"])[-2:] if vocab > 1 else np.array([-np.inf, st["z"][0]])
+        amargin[i] = (top2[1] - top2[0]) / max(abs(top2[1]), 1.0)
         if temperature == 0.0:
             x_hat[i] = int(np.argmax(st["z"]))       # first maximum = lower index
             smargin[i] = math.inf
@@ -355,7 +361,7 @@ def sample_canvas(logits, *, seed, step, block, req, temperature, logit_scale,
     smg = abs(mean_h - stop_threshold) / max(abs(stop_threshold), 1e-300) if stop_threshold >= 0 else math.inf
     return dict(x_hat=x_hat, pmax=pmax, H=ent, keep=keep, x_new=x_new, renoise=renoise,
                 mean_H=mean_h, stop=stop, sample_margin=smargin, keep_margin=kmargin,
-                stop_margin=smg)
+                stop_margin=smg, argmax=amax, argmax_margin=amargin)
 
 
 # ----------------------------------------------------------------------------
@@ -488,7 +494,8 @@ class OracleModel:
 
     def generate_block(self, req, *, seed, block, max_steps, schedule_steps,
                        temperature, logit_scale_growth=1.0, stop_threshold=-1.0,
-                       append=True, keep_budget=None, temperature_end=None):
+                       append=True, keep_budget=None, temperature_end=None,
+                       two_round_stop=False):
         """One block ([P1 一/四], [P2 运作机制], [P3]): random canvas, up to
         max_steps denoise steps with the linear keep schedule over
         schedule_steps, stop on mean entropy, output the last x_hat, then the
@@ -496,7 +503,9 @@ class OracleModel:
         keep_budget: the entropy-budget keep (R-budget) instead of the schedule.
         temperature_end: the linear anneal (R-anneal) from `temperature` at
         step 1 to it at step max_steps; each step's temperature is recorded in
-        its trace entry."""
+        its trace entry.
+        two_round_stop: the stop of R-stop2 with tau = stop_threshold (< 0
+        disables it) in place of the one-round mean-entropy test."""
         n, vocab = self.cfg["canvas"], self.cfg["vocab"]
         canvas = init_canvas(seed, n, vocab, block, req)
         prev = None
@@ -512,6 +521,13 @@ class OracleModel:
                                   stop_threshold=stop_threshold, keep_budget=keep_budget)
             r["canvas_in"] = canvas.copy()
             r["temperature"] = temp
+            if two_round_stop:
+                prev_r = trace[-1] if trace else None
+                r["stop"] = stop_threshold >= 0 and prev_r is not None and stop_two_rounds(
+                    prev_r["mean_H"], r["mean_H"], prev_r["argmax"], r["argmax"], tau=stop_threshold)
+                r["stop_margin"] = math.inf if prev_r is None or stop_threshold < 0 else \
+                    min(abs(prev_r["mean_H"] - stop_threshold), abs(r["mean_H"] - stop_threshold)) / \
+                    max(stop_threshold, 1e-300)
             trace.append(r)
             steps = t
             if r["stop"] or t == max_steps:

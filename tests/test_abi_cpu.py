@@ -153,6 +153,10 @@ def test_noalloc_sampler_refuses_bad_arguments_on_host(lib):
     bad_mode.keep_mode = 2
     rc, msg = _noalloc(lib, fake, 1, 256, 1024, [0], bad_mode, fake)
     assert rc == 1 and "keep_mode" in msg
+    bad_stop = B.sampler_params(temperature=1.0, keep_k=1)
+    bad_stop.stop_mode = 7
+    rc, msg = _noalloc(lib, fake, 1, 256, 1024, [0], bad_stop, fake)
+    assert rc == 1 and "stop_mode" in msg
     for budget in (-0.5, float("nan"), float("inf")):
         rc, msg = _noalloc(lib, fake, 1, 256, 1024, [0], B.sampler_params(entropy_budget=budget), fake)
         assert rc == 1 and "budget" in msg

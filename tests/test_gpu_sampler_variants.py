@@ -10,7 +10,12 @@
 - Temperature anneal and the budget keep in the block loop (tiny fp32 model):
   each step checked against the oracle from the GPU's own canvas, then
   dg_generate_block must reproduce that trajectory token for token.
-- Argument errors: unknown keep_mode, bad budgets, bad anneal ends.
+- Two-round stop: the sampler on peaked logits over four rounds (argmax
+  unchanged, one position changed, a previous round above the threshold)
+  through dg_sample and dg_sample_noalloc; the argmax output against the
+  oracle's; in the tiny model's block (T = 0, every position kept) step by
+  step and through dg_generate_block.
+- Argument errors: unknown keep_mode and stop_mode, bad budgets, bad anneal ends.
 """
 import numpy as np
 import pytest
@@ -24,17 +29,20 @@ SW = synth.WORKLOADS["sampler"]
 TW = synth.WORKLOADS["tiny_fp32"]
 
 
-def _outs(B, n):
+def _outs(B, n, argmax=False):
     dev = "cuda"
-    return dict(x_hat=torch.zeros((B, n), dtype=torch.int32, device=dev),
-                pmax=torch.zeros((B, n), device=dev), entropy=torch.zeros((B, n), device=dev),
-                keep=torch.zeros((B, n), dtype=torch.int32, device=dev),
-                mean_entropy=torch.zeros(B, device=dev), stop=torch.zeros(B, dtype=torch.int32, device=dev))
+    o = dict(x_hat=torch.zeros((B, n), dtype=torch.int32, device=dev),
+             pmax=torch.zeros((B, n), device=dev), entropy=torch.zeros((B, n), device=dev),
+             keep=torch.zeros((B, n), dtype=torch.int32, device=dev),
+             mean_entropy=torch.zeros(B, device=dev), stop=torch.zeros(B, dtype=torch.int32, device=dev))
+    if argmax:
+        o["argmax"] = torch.full((B, n), -1, dtype=torch.int32, device=dev)
+    return o
 
 
-def _sample(dg, logits, req, step, sp, noalloc=False):
+def _sample(dg, logits, req, step, sp, noalloc=False, argmax=False, keep_tensors=False):
     B, n, V = logits.shape
-    outs = _outs(B, n)
+    outs = _outs(B, n, argmax)
     canvas = torch.full((B, n), -1, dtype=torch.int32, device="cuda")
     if noalloc:
         stream = torch.cuda.current_stream()
@@ -46,6 +54,8 @@ def _sample(dg, logits, req, step, sp, noalloc=False):
         dg.dg_synchronize(h)
         h.close()
     outs["canvas"] = canvas
+    if keep_tensors:
+        return outs
     return {k: to_np(v) for k, v in outs.items()}
 
 
@@ -181,14 +191,111 @@ def test_variant_argument_errors(dg):
     for budget in (-1.0, float("nan")):
         with pytest.raises(RuntimeError, match="budget"):
             dg.dg_sample(h, logits, [0], 1, dg.sampler_params(entropy_budget=budget), canvas, dg.step_out())
+    bad = dg.sampler_params(temperature=1.0, keep_k=1)
+    bad.stop_mode = 2
+    with pytest.raises(RuntimeError, match="stop_mode"):
+        dg.dg_sample(h, logits, [0], 1, bad, canvas, dg.step_out())
     h.close()
     om, ht, wd = _tiny(dg)
     S = TW["sampler"]
     out = torch.zeros((1, TW["model"]["canvas"]), dtype=torch.int32, device="cuda")
+    bad_stop = dg.block_args([0], 2, 2, seed=S["seed"])
+    bad_stop.stop_mode = 5
     for kw in (dict(temperature=0.8, temperature_end=0.0), dict(temperature=0.0, temperature_end=0.4),
-               dict(temperature=0.8, entropy_budget=-2.0)):
-        a = dg.block_args([0], 2, 2, seed=S["seed"], **kw)
+               dict(temperature=0.8, entropy_budget=-2.0), None):
+        a = bad_stop if kw is None else dg.block_args([0], 2, 2, seed=S["seed"], **kw)
         with pytest.raises(RuntimeError):
             dg.dg_generate_block(ht, a, out)
         assert dg.dg_get_length(ht, 0) == TW["prompt_len"]     # refused before anything ran
     ht.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("noalloc", [False, True])
+def test_two_round_stop_sampler(dg, noalloc):
+    B, n, V, tau = 2, 64, 5000, 0.005
+    gen = torch.Generator().manual_seed(31)
+    base = torch.randn((B, n, V), generator=gen)
+    peak = torch.randint(0, V, (B, n), generator=gen)
+    l1 = base.clone()
+    l1.scatter_(2, peak[..., None], 30.0)                    # H ~ 1e-8 nats per position
+    l2 = l1 * 1.01                                           # the same argmax
+    l3 = l2.clone()
+    l3[1, 7] = base[1, 7]
+    l3[1, 7, (int(peak[1, 7]) + 1) % V] = 30.0              # canvas 1 changes one position's argmax
+    rounds = [(l1, None, None), (l2, "prev", None), (l3, "prev", None), (l2, "prev", 1.0)]
+    want_stop = [[0, 0], [1, 1], [1, 0], [0, 0]]
+    prev = None
+    for r, ((lg, use_prev, prev_h), want) in enumerate(zip(rounds, want_stop)):
+        pa = pm = None
+        if use_prev:
+            pa = prev["argmax"]
+            pm = prev["mean_entropy"] if prev_h is None else torch.full((B,), prev_h, device="cuda")
+        sp = dg.sampler_params(temperature=1.0, keep_k=n, stop_threshold=tau, seed=5, block=0,
+                               two_round_stop=True, prev_argmax=pa, prev_mean_entropy=pm)
+        outs = _sample(dg, lg.cuda(), [0, 1], r + 1, sp, noalloc=noalloc, argmax=True, keep_tensors=True)
+        got = {k: to_np(v) for k, v in outs.items()}
+        for b in range(B):
+            ref = _oracle(lg[b].numpy(), seed=5, step=r + 1, block=0, req=b, temperature=1.0)
+            check_decisions(got["argmax"][b], ref["argmax"], ref["argmax_margin"], "argmax", thr=1e-6,
+                            max_low_margin=0)
+            assert got["mean_entropy"][b] < tau
+            # the stop is the oracle's rule on this round's and the previous round's GPU outputs
+            want_rule = O.stop_two_rounds(None if pm is None else float(to_np(pm)[b]), float(got["mean_entropy"][b]),
+                                          None if pa is None else to_np(pa)[b], got["argmax"][b], tau=tau)
+            assert bool(got["stop"][b]) == want_rule
+        assert got["stop"].tolist() == want, f"round {r + 1}"
+        prev = outs
+
+
+@pytest.mark.gpu
+def test_argmax_output_at_zero_temperature_is_x_hat(dg):
+    B, n, V = 2, 40, 3001
+    logits = torch.randn((B, n, V), generator=torch.Generator().manual_seed(33))
+    sp = dg.sampler_params(temperature=0.0, keep_k=5, seed=1)
+    got = _sample(dg, logits.cuda(), [0, 1], 1, sp, argmax=True)
+    assert np.array_equal(got["argmax"], got["x_hat"])
+    assert np.array_equal(got["argmax"], logits.argmax(-1).numpy())
+
+
+@pytest.mark.gpu
+def test_block_with_two_round_stop(dg):
+    om, h, wd = _tiny(dg)
+    M, S = TW["model"], TW["sampler"]
+    n, vocab, steps_max, tau = M["canvas"], M["vocab"], 8, 0.1
+    seed, block = S["seed"], 0
+    # 1) step by step at T = 0 with every position kept: the canvas becomes the argmax
+    canvas = torch.from_numpy(O.init_canvas(seed, n, vocab, block, 0).astype(np.int32)).cuda()[None]
+    prev_x = prev = None
+    traj = []
+    for t in range(1, steps_max + 1):
+        c_in = to_np(canvas)[0].copy()
+        logits = torch.zeros((1, n, vocab), device="cuda")
+        outs = _outs(1, n, argmax=True)
+        sp = dg.sampler_params(temperature=0.0, keep_k=n, stop_threshold=tau, seed=seed, block=block,
+                               two_round_stop=True, prev_argmax=None if prev is None else prev["argmax"],
+                               prev_mean_entropy=None if prev is None else prev["mean_entropy"])
+        dg.dg_denoise_step(h, [0], canvas, prev_x, t, sp, dg.step_out(**outs), logits_out=logits)
+        dg.dg_synchronize(h)
+        got = {k: to_np(v) for k, v in outs.items()}
+        ref_logits = om.denoise_forward(0, c_in, None if prev_x is None else to_np(prev_x)[0])
+        assert max_abs_rel(to_np(logits)[0], ref_logits) < 1e-4
+        assert np.array_equal(got["argmax"][0], got["x_hat"][0])
+        ref = _oracle(to_np(logits)[0], seed=seed, step=t, block=block, req=0, temperature=0.0)
+        assert np.array_equal(got["argmax"][0], ref["argmax"])
+        want = O.stop_two_rounds(None if prev is None else float(to_np(prev["mean_entropy"])[0]),
+                                 float(got["mean_entropy"][0]), None if prev is None else to_np(prev["argmax"])[0],
+                                 got["argmax"][0], tau=tau)
+        assert bool(got["stop"][0]) == want
+        traj.append(got)
+        if got["stop"][0] or t == steps_max:
+            break
+        prev, prev_x = outs, outs["x_hat"]
+    # 2) the block loop keeps the previous round itself: the same trajectory
+    a = dg.block_args([0], steps_max, 1, temperature=0.0, stop_threshold=tau, seed=seed, block=block,
+                      two_round_stop=True)
+    out = torch.zeros((1, n), dtype=torch.int32, device="cuda")
+    steps = dg.dg_generate_block(h, a, out)
+    assert steps == len(traj)
+    assert np.array_equal(to_np(out)[0], traj[-1]["x_hat"][0])
+    h.close()

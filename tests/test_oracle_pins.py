@@ -495,3 +495,44 @@ def test_block_with_anneal_runs_each_step_at_the_annealed_temperature():
     # the budget keep plugs into the block: a budget of 0 locks one position a step
     toks, steps, trace = run(keep_budget=0.0)
     assert all(r["keep"].sum() == 1 for r in trace) and np.array_equal(toks, trace[-1]["x_hat"])
+
+
+def test_sampler_reports_the_argmax_of_z():
+    rng = np.random.default_rng(25)
+    logits = rng.normal(size=(9, 70)).astype(np.float32)
+    logits[2, [5, 40]] = 9.0                                   # a tie: the lower index
+    for temperature, scale in ((1.0, 1.0), (0.7, 2.0), (0.0, 1.0)):
+        out = O.sample_canvas(logits, seed=2, step=1, block=0, req=0, temperature=temperature, logit_scale=scale,
+                              keep_k=3, stop_threshold=-1.0)
+        assert np.array_equal(out["argmax"], torch.from_numpy(logits).argmax(-1).numpy())
+        assert out["argmax"][2] == 5 and out["argmax_margin"][2] == 0.0
+        assert (out["argmax_margin"] >= 0).all()
+        if temperature == 0.0:
+            assert np.array_equal(out["argmax"], out["x_hat"])
+
+
+def test_block_with_two_round_stop_follows_the_rule_on_its_own_trace():
+    def run(tau, scale=50.0, **kw):
+        m = _tiny_model(seed=26, n_layers=1)
+        m.weights["embed"] = m.weights["embed"] * scale       # confident logits: mean H near 0
+        m.encode_causal(0, np.arange(4))
+        return m.generate_block(0, seed=2, block=0, max_steps=6, schedule_steps=1, temperature=0.0,
+                                stop_threshold=tau, append=False, two_round_stop=True, **kw)
+    toks, steps, trace = run(0.1)
+    assert not trace[0]["stop"]                                  # no previous round
+    for t in range(1, len(trace)):
+        want = O.stop_two_rounds(trace[t - 1]["mean_H"], trace[t]["mean_H"], trace[t - 1]["argmax"],
+                                 trace[t]["argmax"], tau=0.1)
+        assert trace[t]["stop"] == want
+    assert all(not r["stop"] for r in trace[:-1])                # the block ends at its first stop
+    assert np.array_equal(toks, trace[-1]["x_hat"])
+    # T = 0 and every position kept: the canvas becomes the argmax, so a stop means a fixed point
+    if trace[-1]["stop"]:
+        assert np.array_equal(trace[-1]["argmax"], trace[-2]["argmax"])
+    # a negative threshold disables the stop; the one-round test would stop at step 1 here
+    assert run(-1.0)[1] == 6
+    m = _tiny_model(seed=26, n_layers=1)
+    m.weights["embed"] = m.weights["embed"] * 50.0
+    m.encode_causal(0, np.arange(4))
+    assert m.generate_block(0, seed=2, block=0, max_steps=6, schedule_steps=1, temperature=0.0,
+                            stop_threshold=0.1, append=False)[1] == 1
