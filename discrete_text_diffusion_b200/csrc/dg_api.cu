@@ -1065,7 +1065,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
 
 void dg_destroy(dg_handle* H) {
   if (!H) return;
-  if (H->stream || true) cudaStreamSynchronize(H->stream);
+  cudaStreamSynchronize(H->stream);  // the legacy default stream when the handle has none
   void* ps[] = {H->kc, H->vt, H->h, H->xn, H->eprev, H->qkv, H->q, H->attn, H->glog, H->ids, H->wts, H->cnt,
                 H->off, H->perm, H->work, H->n_work, H->touched, H->xp, H->hb, H->y, H->logits, H->rope, H->sws,
                 H->xh[0], H->xh[1], H->pmax, H->ent, H->keep, H->meanh, H->stop, H->done, H->canvas, H->out_tok,
