@@ -21,6 +21,7 @@ from tests import test_oracle_pins as P
 # the unaltered functions, for planted versions that wrap them
 _philox, _router, _attention = O.philox4x32_10, O.router, O.attention
 _position_stats, _anneal = O.position_stats, O.anneal_temperature
+_quantize = N.quantize
 
 
 def _rope_sign(x, pos, base):
@@ -123,6 +124,30 @@ def _budget_exclusive(ent, budget):
     return keep, math.inf
 
 
+def _budget_may_keep_none(ent, budget):
+    ent = np.asarray(ent, dtype=np.float64)
+    order = np.lexsort((np.arange(len(ent)), ent))
+    keep = np.zeros(len(ent), dtype=bool)
+    run = 0.0
+    for i in order:
+        if run + ent[i] > budget:                                               # the most certain one not forced
+            break
+        run += ent[i]
+        keep[i] = True
+    return keep, math.inf
+
+
+def _argmax_last_tie(logits):
+    z = np.asarray(logits)
+    return (z.shape[-1] - 1 - np.argmax(z[..., ::-1], axis=-1)).astype(np.int64)  # ties -> higher index
+
+
+def _quantize_no_448(w):
+    q = _quantize(w)
+    amax = float(np.max(np.abs(w)))
+    return dict(q, g=float(np.float32(amax / 6.0)))                               # per-tensor scale without E4M3's range
+
+
 def _embed_sc_transposed(self, tokens, prev_pred=None):
     E = self.weights["embed"]
     h = E[np.asarray(tokens)].astype(np.float64)
@@ -197,6 +222,13 @@ CASES = {
     "e2m1 ties up": (N, "e2m1_encode", _e2m1_ties_up, [PN.test_e2m1_encode_is_nearest_with_ties_to_even_by_brute_force]),
     "block scale axis": (N, "dequantize", _dequant_tiled, [lambda: PN.test_quantize_reproduces_weights_built_from_codes(0)]),
     "nibble order": (N, "pack", _pack_swapped, [PN.test_pack_nibble_order_and_round_trip]),
+    "budget keeps none": (O, "keep_entropy_budget", _budget_may_keep_none,
+                          [lambda: P.test_entropy_budget_keep_invariants(0)]),
+    "argmax ties": (O, "argmax_tokens", _argmax_last_tie, [P.test_argmax_tokens_takes_the_lower_index_on_ties,
+                                                         P.test_sampler_reports_the_argmax_of_z]),
+    "global scale range": (N, "quantize", _quantize_no_448,
+                           [lambda: PN.test_quantize_reproduces_weights_built_from_codes(0),
+                            PN.test_quantize_error_bound_and_structure]),
 }
 
 

@@ -473,7 +473,8 @@ def test_block_with_anneal_runs_each_step_at_the_annealed_temperature():
     def run(**extra):
         m = _tiny_model(seed=24, n_layers=1)
         m.encode_causal(0, np.arange(4))
-        return m.generate_block(0, seed=1, block=0, max_steps=4, schedule_steps=4, temperature=0.8,
+        # the keep schedule (2 steps) is shorter than the step budget (4): the anneal runs over the budget
+        return m.generate_block(0, seed=1, block=0, max_steps=4, schedule_steps=2, temperature=0.8,
                                 stop_threshold=-1.0, append=False, **extra)
     toks, steps, trace = run(temperature_end=0.4)
     assert steps == 4
@@ -484,7 +485,7 @@ def test_block_with_anneal_runs_each_step_at_the_annealed_temperature():
     prev = None
     for t, r in enumerate(trace, start=1):
         one = m.denoise_step(0, r["canvas_in"], prev, step=t, block=0, seed=1, temperature=r["temperature"],
-                             logit_scale=1.0, keep_k=O.linear_keep_count(m.cfg["canvas"], t, 4),
+                             logit_scale=1.0, keep_k=O.linear_keep_count(m.cfg["canvas"], t, 2),
                              stop_threshold=-1.0)
         assert np.array_equal(one["x_new"], r["x_new"]) and np.allclose(one["H"], r["H"])
         prev = r["x_hat"]
