@@ -41,6 +41,10 @@ Readings of points the pages leave open (each is a named reading, R-x):
             softmax over the k selected logits.
   R-append  a finished canvas is appended by one causal encode pass over its
             tokens (no self-conditioning).
+  R-ar      AR mode ([P1 七]: the weights load unchanged as an autoregressive
+            model): a token is encoded causally at the end of the cache, as a
+            prompt token is, and the tied LM head of its final-norm output
+            gives the next token's logits.  No canvas, no self-conditioning.
   The page's own sampler variants ([P1 四]; the CUDA path has all three):
   R-budget  entropy-ordered locking: positions sorted by entropy ascending
             (ties -> lower index) are kept while the inclusive cumulative
@@ -481,6 +485,13 @@ class OracleModel:
         x = rms_norm(h, self.weights["final_norm"], c["rms_eps"])
         logits = lm_head(x, self.weights["embed"])
         return (logits, h) if return_hidden else logits
+
+    def ar_next_logits(self, req, token):
+        """AR mode (R-ar): append one token to the request's cache by a causal
+        pass and return the logits [V] of the token that follows it."""
+        h = self.encode_causal(req, [int(token)])
+        x = rms_norm(h, self.weights["final_norm"], self.cfg["rms_eps"])
+        return lm_head(x, self.weights["embed"])[0]
 
     def denoise_step(self, req, canvas, prev_pred, *, step, block, seed, temperature,
                      logit_scale, keep_k, stop_threshold, keep_budget=None):

@@ -148,6 +148,10 @@ def _quantize_no_448(w):
     return dict(q, g=float(np.float32(amax / 6.0)))                               # per-tensor scale without E4M3's range
 
 
+def _ar_no_append(self, req, token):
+    return self.denoise_forward(req, [int(token)])[0]                            # the token is never cached
+
+
 def _embed_sc_transposed(self, tokens, prev_pred=None):
     E = self.weights["embed"]
     h = E[np.asarray(tokens)].astype(np.float64)
@@ -226,6 +230,8 @@ CASES = {
                           [lambda: P.test_entropy_budget_keep_invariants(0)]),
     "argmax ties": (O, "argmax_tokens", _argmax_last_tie, [P.test_argmax_tokens_takes_the_lower_index_on_ties,
                                                          P.test_sampler_reports_the_argmax_of_z]),
+    "AR step not cached": (O.OracleModel, "ar_next_logits", _ar_no_append,
+                           [P.test_ar_decode_one_token_at_a_time_equals_one_causal_pass]),
     "global scale range": (N, "quantize", _quantize_no_448,
                            [lambda: PN.test_quantize_reproduces_weights_built_from_codes(0),
                             PN.test_quantize_error_bound_and_structure]),

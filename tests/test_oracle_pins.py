@@ -537,3 +537,21 @@ def test_block_with_two_round_stop_follows_the_rule_on_its_own_trace():
     m.encode_causal(0, np.arange(4))
     assert m.generate_block(0, seed=2, block=0, max_steps=6, schedule_steps=1, temperature=0.0,
                             stop_threshold=0.1, append=False)[1] == 1
+
+
+def test_ar_decode_one_token_at_a_time_equals_one_causal_pass():
+    m = _tiny_model(seed=27, n_layers=2)
+    rng = np.random.default_rng(28)
+    prompt = rng.integers(0, m.cfg["vocab"], 7)
+    cont = rng.integers(0, m.cfg["vocab"], 5)
+    m.encode_causal(0, prompt)
+    steps = np.stack([m.ar_next_logits(0, t) for t in cont])
+    ref = _tiny_model(seed=27, n_layers=2)
+    h = ref.encode_causal(0, np.concatenate([prompt, cont]))      # the whole sequence in one causal pass
+    x = O.rms_norm(h[len(prompt):], ref.weights["final_norm"], ref.cfg["rms_eps"])
+    want = torch.from_numpy(x) @ torch.from_numpy(ref.weights["embed"]).T
+    assert np.allclose(steps, want.numpy(), rtol=1e-10, atol=1e-10)
+    assert m.length(0) == len(prompt) + len(cont)
+    for li in range(2):
+        assert np.allclose(m.k_cache[0][li], ref.k_cache[0][li], atol=1e-12)
+        assert np.allclose(m.v_cache[0][li], ref.v_cache[0][li], atol=1e-12)
