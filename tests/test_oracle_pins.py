@@ -555,3 +555,24 @@ def test_ar_decode_one_token_at_a_time_equals_one_causal_pass():
     for li in range(2):
         assert np.allclose(m.k_cache[0][li], ref.k_cache[0][li], atol=1e-12)
         assert np.allclose(m.v_cache[0][li], ref.v_cache[0][li], atol=1e-12)
+
+
+def test_certain_and_stable_canvas_stops_after_round_two():
+    """[P1 六]: when every prediction is certain and no longer changes (the page's structured-output example),
+    the block needs two rounds.  With the layers reduced to the identity (zero O, expert down and
+    self-conditioning weights) and large embeddings, each position's logits peak at its own token, so at T = 0
+    with every position kept the round-1 argmax is the canvas itself and round 2 repeats it."""
+    m = _tiny_model(seed=29, n_layers=2, vocab=40)
+    m.weights["embed"] = m.weights["embed"] * 20.0
+    m.weights["w_sc"] = np.zeros_like(m.weights["w_sc"])
+    for L in m.weights["layers"]:
+        L["wo"] = np.zeros_like(L["wo"])
+        L["w_down"] = np.zeros_like(L["w_down"])
+    m.encode_causal(0, np.arange(5))
+    canvas0 = O.init_canvas(4, m.cfg["canvas"], m.cfg["vocab"], 0, 0)
+    logits = m.denoise_forward(0, canvas0)
+    assert np.array_equal(O.argmax_tokens(logits), canvas0)          # the fixed point the pin relies on
+    toks, steps, trace = m.generate_block(0, seed=4, block=0, max_steps=8, schedule_steps=1, temperature=0.0,
+                                          stop_threshold=0.005, append=False, two_round_stop=True)
+    assert steps == 2 and [r["stop"] for r in trace] == [False, True]
+    assert trace[0]["mean_H"] == 0.0 and np.array_equal(toks, canvas0)
