@@ -8,6 +8,15 @@ prompt already in the cache, up to 48 steps, linear keep over 48, stop 0.1 nats,
 logit scale 1.5^(t-1).  Before every block the request's cache length is reset
 to the prompt, so every step does the same work.  Weights (49 GB) exceed L2.
 
+With full_b1 the same run then measures the batch-16 workload (full_b16: 16
+requests with 4096-token prompts, 4 blocks of 12 fixed steps per bench step)
+and reports it under "workloads" (skip with --no-b16).  The JSON line carries
+the block-level roofline ("roofline_step": the sum over the block's passes of
+max(bytes / HBM, flops / bf16 peak) against the measured block time), the
+dominant kernel's roofline and every major kernel class's, from one extra
+profiled bench step after the timed region (the timed region itself carries no
+profiling events).
+
   python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
 
 N > 1 runs N independent replicas (one per GPU, no data-path collective; the
@@ -30,11 +39,11 @@ if ROOT not in sys.path:
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one canvas-step attention launch (prompt 8192,
-# canvas 256, 16 heads of 256), from the ncu capture summarised in
-# profiles/attn_tc_canvas_over_8192_cache.md (same shapes as one layer of the
-# full_b1 canvas step); set to None when the kernel changes.
-ATTN_TRAFFIC = 75321088
+CSRC = os.path.join(ROOT, "discrete_text_diffusion_b200", "csrc")
+# DRAM bytes (read + write) per launch measured by ncu for a kernel class, with
+# the source file and the sha256 prefix of that file when it was captured.  A
+# class whose source has changed since reports traffic null.
+NCU_TRAFFIC = {}
 
 
 def parse_args(argv=None):
@@ -44,6 +53,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["full_b1", "full_b16"], default="full_b1")
+    ap.add_argument("--no-b16", action="store_true", help="with full_b1: skip the batch-16 companion measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
@@ -152,6 +162,21 @@ def workload(name):
     return W
 
 
+def _src_sha(name):
+    import hashlib
+    with open(os.path.join(CSRC, name), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def ncu_traffic(cls):
+    """The ncu-measured DRAM bytes per launch of a kernel class, or None when
+    there is no capture of the current source."""
+    if cls not in NCU_TRAFFIC:
+        return None
+    byt, src, sha = NCU_TRAFFIC[cls]
+    return byt if _src_sha(src) == sha else None
+
+
 def attention_flops(model, batch, canvas, blocks):
     """Algorithmic flops of the attention launches of the given blocks, all
     layers.  blocks: (prompt length, denoise steps) per block.  Each denoise
@@ -172,19 +197,141 @@ def moe_up_bytes(model, n_rows, touched):
     return touched * 2 * f * d * 2 + n_rows * d * 2 + n_rows * f * 2
 
 
+def moe_down_bytes(model, n_rows, touched):
+    """One grouped down launch: the touched experts' down weights, the SwiGLU rows
+    read, the bf16 expert outputs written."""
+    d, f = model["d_model"], model["d_ff"]
+    return touched * f * d * 2 + n_rows * f * 2 + n_rows * d * 2
+
+
+def pass_cost(model, batch, canvas, prompt, touched, causal, head, self_cond):
+    """Algorithmic (bytes, flops) of one forward pass over batch x canvas tokens
+    at cache length `prompt`: every weight read once (experts only if touched,
+    `touched` distinct experts per layer), the KV cache read once and the
+    canvas K/V written and read, bf16 throughout; flops of every product.
+    causal: the hand-off pass (query i sees prompt + i + 1 keys) instead of the
+    bidirectional canvas step.  head: the LM head; self_cond: the W_sc product.
+    Activations and logits between kernels are not counted (a fused path need
+    not write them)."""
+    d, hq, hkv, hd = model["d_model"], model["n_heads"], model["n_kv_heads"], model["head_dim"]
+    E, k, F, V, L = model["n_experts"], model["top_k"], model["d_ff"], model["vocab"], model["n_layers"]
+    T = batch * canvas
+    attn_w = ((hq + 2 * hkv) * hd * d + d * hq * hd) * 2
+    router_w = E * d * 2
+    expert_w = 3 * F * d * 2
+    kv_pos = hkv * hd * 2 * 2                      # K and V, bf16, per position per layer
+    byt = L * (attn_w + router_w + touched * expert_w + batch * prompt * kv_pos + 2 * T * kv_pos)
+    if head:
+        byt += V * d * 2
+    if self_cond:
+        byt += d * d * 2
+    per_tok = 2 * d * (hq + 2 * hkv) * hd + 2 * hq * hd * d + 2 * d * E + k * 3 * 2 * d * F
+    keys = (canvas * (prompt + canvas) if not causal else sum(prompt + i + 1 for i in range(canvas))) * batch
+    fl = L * (T * per_tok + 4.0 * hq * hd * keys)
+    if head:
+        fl += T * 2.0 * d * V
+    if self_cond:
+        fl += T * 2.0 * d * d
+    return float(byt), float(fl)
+
+
+def block_roofline(model, batch, canvas, blocks, touched, block_ms, peaks, sustained=True):
+    """Roofline of whole blocks (denoise steps + hand-off): the bound time is the
+    sum over passes of max(bytes / HBM, flops / bf16 peak); frac = bound / measured."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    tf = (peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) if sustained else peaks["bf16_tflops"]) * 1e12
+    bound_s, byt_all, fl_all, steps_all, hbm_s, tc_s = 0.0, 0.0, 0.0, 0, 0.0, 0.0
+    for prompt, steps in blocks:
+        for t in range(1, steps + 1):
+            b, f = pass_cost(model, batch, canvas, prompt, touched, False, True, t > 1)
+            bound_s += max(b / hbm, f / tf)
+            hbm_s += b / hbm
+            tc_s += f / tf
+            byt_all += b
+            fl_all += f
+        b, f = pass_cost(model, batch, canvas, prompt, touched, True, False, False)
+        bound_s += max(b / hbm, f / tf)
+        hbm_s += b / hbm
+        tc_s += f / tf
+        byt_all += b
+        fl_all += f
+        steps_all += steps
+    nblk = max(1, len(blocks))
+    measured_s = block_ms / 1e3 * nblk
+    return {"bound": "hbm" if hbm_s >= tc_s else "tensor",
+            "bound_ms_per_block": round(bound_s * 1e3 / nblk, 3),
+            "measured_ms_per_block": round(block_ms, 3),
+            "bound_us_per_denoise_step": round(bound_s * 1e6 / max(1, steps_all), 1),
+            "measured_us_per_denoise_step": round(measured_s * 1e6 / max(1, steps_all), 1),
+            "frac": round(bound_s / measured_s, 4),
+            "gbytes_per_block": round(byt_all / 1e9 / nblk, 3), "tflop_per_block": round(fl_all / 1e12 / nblk, 3),
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+            "bf16_peak_tflops": round(tf / 1e12, 1),
+            "experts_touched_per_layer": round(touched, 2),
+            "includes": "denoise steps + the causal hand-off; weights, KV, canvas K/V; activations and logits "
+                        "between kernels not counted"}
+
+
+def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, peak_kind):
+    """Per-kernel-class roofline from one profiled block (every class timed on
+    the library's stream).  Returns {class: roofline} with algorithmic bytes or
+    flops per launch over the class's mean launch time."""
+    d, F, V, L = model["d_model"], model["d_ff"], model["vocab"], model["n_layers"]
+    hq, hkv, hd, k = model["n_heads"], model["n_kv_heads"], model["head_dim"], model["top_k"]
+    hbm = peaks["hbm_gbs"]
+    tfs = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    T = batch * canvas
+    rows = T * k
+    steps = sum(s for _, s in blocks)
+    passes = steps + len(blocks)
+    out = {}
+
+    def add(cls, name, bound, per_launch, launches_expected=None):
+        if cls not in breakdown:
+            return
+        nl, ms = breakdown[cls]
+        us = ms / nl * 1e3
+        if bound == "hbm":
+            ach = per_launch / (us * 1e-6) / 1e9
+            r = {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "peak_kind": peak_kind,
+                 "unit": "GB/s", "frac": round(ach / hbm, 4), "bytes_per_launch": int(per_launch)}
+        else:
+            ach = per_launch / (us * 1e-6) / 1e12
+            r = {"kernel": name, "bound": "tensor", "achieved": round(ach, 1), "peak": tfs,
+                 "peak_kind": peak_kind + " sustained", "unit": "TFLOP/s", "frac": round(ach / tfs, 4),
+                 "flops_per_launch": per_launch}
+        r.update({"launches": nl, "avg_launch_us": round(us, 2), "ms_per_block": round(ms / len(blocks), 3),
+                  "traffic": ncu_traffic(cls)})
+        out[cls] = r
+
+    if "attention" in breakdown:
+        nl, _ = breakdown["attention"]
+        add("attention", "attn_tc_kernel (+ split combine)", "tensor", attention_flops(model, batch, canvas, blocks) / nl)
+    if batch == 1:
+        add("moe_up", "gemm_tc_kernel (grouped gate/up + SwiGLU)", "hbm", moe_up_bytes(model, rows, touched))
+        add("moe_down", "gemm_tc_kernel (grouped down, scatter)", "hbm", moe_down_bytes(model, rows, touched))
+    else:
+        add("moe_up", "gemm_tc_kernel (grouped gate/up + SwiGLU)", "tensor", 2.0 * rows * 2 * F * d)
+        add("moe_down", "gemm_tc_kernel (grouped down, scatter)", "tensor", 2.0 * rows * F * d)
+    if "dense_gemm" in breakdown:
+        # QKV and O every pass, W_sc every step after the first: weights once each
+        nl, _ = breakdown["dense_gemm"]
+        byt = (passes * L * ((hq + 2 * hkv) * hd * d + d * hq * hd) + (steps - len(blocks)) * d * d) * 2
+        add("dense_gemm", "gemm_tc_kernel (split-K QKV / O / self-cond)", "hbm", byt / nl)
+    add("lm_head", "gemm_tc_kernel (tied LM head)", "hbm", V * d * 2 + T * V * 4)
+    add("sampler_rows", "sampler_pass1 + sampler_pass2", "hbm", 4.0 * V * T)
+    return out
+
+
 # -------------------------------------------------------------------- ours
 
-def run_ours(args):
+def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clocks=True):
+    """Build the workload's model, time `steps` bench steps after `warmup`, then
+    an end-to-end pass and one profiled block.  Returns a dict of results."""
     import torch
 
-    import discrete_text_diffusion_b200 as m
     from discrete_text_diffusion_b200 import synth
-
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dist = init_dist("nccl")
-    dev = torch.device("cuda", local)
-    W = workload(args.workload)
+    W = workload(name)
     model, S = W["model"], W["sampler"]
     B, n, P0 = W["batch"], model["canvas"], W["prompt_len"]
     blocks = W.get("blocks", 1)
@@ -229,35 +376,36 @@ def run_ours(args):
             total += used
         steps_seen.append(total)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         one_step()
     m.dg_synchronize(h)
 
+    # the timed region: no profiling events, only the two bracketing events
     stream = torch.cuda.current_stream(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # inside the timed region only the roofline kernel's launches carry events
-    m.dg_profile_reset(h)
-    m.dg_profile_enable(h, True, classes=["attention"])
+    m.dg_profile_enable(h, False)
     launches0 = m.dg_launch_count(h)
     steps_seen.clear()
     block_log.clear()
-    with ClockSampler(local) as clk:
-        barrier(dist)
-        torch.cuda.synchronize(dev)
-        ev0.record(stream)
-        for _ in range(args.steps):
-            one_step()
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(dist)
+    clk = ClockSampler(dev.index if dev.index is not None else 0) if with_clocks else None
+    if clk:
+        clk.__enter__()
+    barrier(dist)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(steps):
+        one_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist)
+    if clk:
+        clk.__exit__(None, None, None)
     elapsed = ev0.elapsed_time(ev1)
     launches = m.dg_launch_count(h) - launches0
-    prof = m.dg_profile_read(h)
-    m.dg_profile_enable(h, False)
-    clocks = clk.summary()
+    clocks = clk.summary() if clk else None
     denoise_steps = sum(steps_seen)
     timed_blocks = list(block_log)
-    units = args.steps * blocks * B * n
+    units = steps * blocks * B * n
     elapsed_max, units_all = aggregate(dist, elapsed, units, device=dev)
 
     # end to end: the same calls with the tokens landing in pinned host memory
@@ -265,56 +413,55 @@ def run_ours(args):
     barrier(dist)
     torch.cuda.synchronize(dev)
     e0 = time.perf_counter()
-    for _ in range(args.steps):
+    for _ in range(steps):
         one_step(host=True)
     torch.cuda.synchronize(dev)
     e2e_ms = (time.perf_counter() - e0) * 1e3
     e2e_max, _ = aggregate(dist, e2e_ms, units, device=dev)
 
-    # per-class kernel time from one extra, untimed step with every class profiled
+    # per-class kernel time from one extra, untimed bench step with every class profiled
     m.dg_profile_reset(h)
     m.dg_profile_enable(h, True)
+    block_log.clear()
     one_step()
     breakdown = m.dg_profile_read(h)
+    prof_blocks = list(block_log)
     m.dg_profile_enable(h, False)
+    h.close()
+    del w
+    torch.cuda.empty_cache()
+    return dict(W=W, model=model, B=B, n=n, P0=P0, blocks=blocks, elapsed_max=elapsed_max, units_all=units_all,
+                e2e_max=e2e_max, launches=launches, clocks=clocks, denoise_steps=denoise_steps,
+                timed_blocks=timed_blocks, breakdown=breakdown, prof_blocks=prof_blocks, touched=touched_mean,
+                prefill_s=prefill_s, steps=steps, warmup=warmup)
 
+
+def run_ours(args):
+    import torch
+
+    import discrete_text_diffusion_b200 as m
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = init_dist("nccl")
+    dev = torch.device("cuda", local)
     peaks, peak_kind = load_peaks()
-    roof = None
-    if "attention" in prof:
-        # the dominant kernel: tcgen05 attention (+ its split combine), timed on
-        # the library's stream over the whole timed region; tensor-bound, so
-        # against the sustained bf16 peak (it runs inside a long step)
-        nl, ms = prof["attention"]
-        fl = attention_flops(model, B, n, timed_blocks)
-        ach = fl / (ms / 1e3) / 1e12
-        pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        roof = {"kernel": "attn_tc_kernel (+ split combine)", "bound": "tensor", "achieved": round(ach, 1),
-                "peak": pk, "peak_kind": peak_kind + " sustained", "unit": "TFLOP/s", "frac": round(ach / pk, 4),
-                "traffic": ATTN_TRAFFIC, "traffic_per": "canvas-step launch (ncu capture)",
-                "flops_timed": fl, "launches": nl,
-                "avg_launch_us": round(ms / nl * 1e3, 2)}
-    roof_moe = None
-    if "moe_up" in breakdown:
-        # from the separately profiled step (every class timed), not the timed region
-        nl, ms = breakdown["moe_up"]
-        per_launch_s = ms / nl / 1e3
-        byt = moe_up_bytes(model, B * n * model["top_k"], touched_mean)
-        ach = byt / per_launch_s / 1e9
-        roof_moe = {"kernel": "gemm_tc_kernel (grouped gate/up + SwiGLU)", "bound": "hbm", "achieved": round(ach, 1),
-                "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
-                "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
-                "bytes_per_launch": int(byt), "avg_launch_us": round(per_launch_s * 1e6, 2),
-                "experts_touched_mean": round(touched_mean, 2), "timed": "profiled step"}
+    r = _measure_workload(m, args, args.workload, args.steps, args.warmup, dev, dist, world)
+    model, B, n, P0, blocks = r["model"], r["B"], r["n"], r["P0"], r["blocks"]
+    block_ms = r["elapsed_max"] / (args.steps * blocks)
+    roof_step = block_roofline(model, B, n, r["timed_blocks"][:blocks], r["touched"], block_ms, peaks)
+    kr = kernel_rooflines(model, B, n, r["prof_blocks"], r["touched"], r["breakdown"], peaks, peak_kind)
+    dominant = max(kr, key=lambda c: r["breakdown"][c][1]) if kr else None
     line = {
         "metric": "canvas tokens/s (block generation, adaptive stop)",
-        "value": round(units_all / (elapsed_max / 1e3), 2),
+        "value": round(r["units_all"] / (r["elapsed_max"] / 1e3), 2),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(elapsed_max / args.steps, 3),
-        "us_per_denoise_step": round(elapsed_max * 1e3 / max(1, denoise_steps), 1),
-        "denoise_steps_per_block": round(denoise_steps / max(1, args.steps * blocks), 2),
+        "ms_per_step": round(r["elapsed_max"] / args.steps, 3),
+        "us_per_denoise_step": round(r["elapsed_max"] * 1e3 / max(1, r["denoise_steps"]), 1),
+        "denoise_steps_per_block": round(r["denoise_steps"] / max(1, args.steps * blocks), 2),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -324,21 +471,44 @@ def run_ours(args):
                    "layers": model["n_layers"], "d_model": model["d_model"], "experts": model["n_experts"],
                    "top_k": model["top_k"], "vocab": model["vocab"], "blocks_per_step": blocks,
                    "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (49 GB of weights)"},
-        "e2e": {"value": round(units_all / (e2e_max / 1e3), 2), "unit": "tokens/s",
+        "e2e": {"value": round(r["units_all"] / (r["e2e_max"] / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": 4 * B * blocks, "d2h_bytes_per_step": 4 * B * n * blocks},
-        "gpu_launches": int(launches),
-        "roofline": roof,
-        "roofline_moe_up": roof_moe,
-        "clocks": clocks,
-        "prefill_s": round(prefill_s, 2),
-        "kernel_ms_one_step": {k: round(v[1], 3) for k, v in breakdown.items()},
+        "gpu_launches": int(r["launches"]),
+        "roofline": dict(kr[dominant], kernel_class=dominant) if dominant else None,
+        "roofline_step": roof_step,
+        "rooflines": kr,
+        "clocks": r["clocks"],
+        "prefill_s": round(r["prefill_s"], 2),
+        "kernel_ms_per_block": {k: round(v[1] / len(r["prof_blocks"]), 3) for k, v in r["breakdown"].items()},
     }
+    if args.workload == "full_b1" and not args.no_b16:
+        # the batch-16 workload in the same run: 16 requests x 4 blocks x 12 steps per bench step
+        s16, w16 = max(1, min(args.steps, 2)), max(1, min(args.warmup, 1))
+        q = _measure_workload(m, args, "full_b16", s16, w16, dev, dist, world)
+        qb = q["blocks"]
+        blk_ms = q["elapsed_max"] / (s16 * qb)
+        kq = kernel_rooflines(q["model"], q["B"], q["n"], q["prof_blocks"], q["touched"], q["breakdown"], peaks,
+                              peak_kind)
+        line["workloads"] = {"full_b16": {
+            "value": round(q["units_all"] / (q["elapsed_max"] / 1e3), 2), "unit": "tokens/s",
+            "steps": s16, "warmup": w16, "ms_per_step": round(q["elapsed_max"] / s16, 3),
+            "us_per_denoise_step": round(q["elapsed_max"] * 1e3 / max(1, q["denoise_steps"]), 1),
+            "config": {"batch": q["B"], "canvas": q["n"], "prompt_len": q["P0"], "blocks_per_step": qb,
+                       "denoise_steps_per_block": q["W"]["sampler"]["max_steps"]},
+            "e2e": {"value": round(q["units_all"] / (q["e2e_max"] / 1e3), 2), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 4 * q["B"] * qb, "d2h_bytes_per_step": 4 * q["B"] * q["n"] * qb},
+            "gpu_launches": int(q["launches"]),
+            "roofline_step": block_roofline(q["model"], q["B"], q["n"], q["timed_blocks"][:qb], q["touched"],
+                                            blk_ms, peaks),
+            "rooflines": kq,
+            "clocks": q["clocks"],
+            "kernel_ms_per_block": {k: round(v[1] / len(q["prof_blocks"]), 3) for k, v in q["breakdown"].items()},
+        }}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(W, line["denoise_steps_per_block"])
+        line["cpu_baseline"] = cpu_baseline(r["W"], line["denoise_steps_per_block"])
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
-    h.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -415,10 +585,12 @@ def run_reference(args):
     steps_per_block = {"full_b1": 7.0, "full_b16": 12.0}[args.workload]
     rates = []
     for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         layer_s, head_row_s = oracle_sample(W, seed_off=0)
+        sample_s = time.perf_counter() - t0
         tps, _, block_s = oracle_tokens_per_s(W, layer_s, head_row_s, steps_per_block)
         if i >= args.warmup:
-            rates.append((tps, block_s))
+            rates.append((tps, block_s, sample_s))
     value = statistics.median(r[0] for r in rates)
     line = {
         "impl": "reference",
@@ -430,6 +602,8 @@ def run_reference(args):
         "config": {"workload": args.workload, "batch": W["batch"], "canvas": W["model"]["canvas"],
                    "prompt_len": W["prompt_len"], "layers": W["model"]["n_layers"],
                    "parallelism": "host cores"},
+        "projected": True,
+        "timed_sample_s_per_step": round(statistics.median(r[2] for r in rates), 2),
         "cpu_baseline": {"value": round(value, 5), "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
                          "sample": "per step: 1 layer on the full canvas + LM head/sampler for 16 positions, "
                                    f"extrapolated at {steps_per_block} denoise steps per block"},

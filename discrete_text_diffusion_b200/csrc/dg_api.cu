@@ -672,9 +672,10 @@ void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
 
 template <typename T>
 void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const int32_t* tokens,
-                  const int32_t* prev, bool head, float* logits, float* hidden_out) {
+                  const int32_t* prev, bool head, float* logits, float* hidden_out, const dg_layer_dump* dump) {
   const dg_config& c = H->c;
   const int Tn = bi.B * nq;
+  const size_t hbytes = (size_t)Tn * c.d_model * sizeof(float);
   const float eps = (float)c.rms_eps;
   T* xn = (T*)H->xn;
   {
@@ -699,6 +700,8 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
   const int ldqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& L = H->lw[l];
+    const bool rec = dump && dump->layer == l;
+    if (rec && dump->hidden_in) cudaMemcpyAsync(dump->hidden_in, H->h, hbytes, cudaMemcpyDeviceToDevice, H->stream);
     const int qs = qkv_gemm(H, l, Tn);
     {
       ProfScope ps(H, PC_ROPE);
@@ -728,6 +731,12 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
       launch_router_permute(H->ids, Tn * c.top_k, c.n_experts, grouped_tile(H, Tn), H->cnt, H->off, H->perm,
                             H->work, H->n_work, H->touched + l, H->stream);
     }
+    if (rec && dump->expert_ids)
+      cudaMemcpyAsync(dump->expert_ids, H->ids, (size_t)Tn * c.top_k * sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                      H->stream);
+    if (rec && dump->expert_wts)
+      cudaMemcpyAsync(dump->expert_wts, H->wts, (size_t)Tn * c.top_k * sizeof(float), cudaMemcpyDeviceToDevice,
+                      H->stream);
     {
       ProfScope ps(H, PC_GATHER);
       launch_gather_rows<T>(xn, H->perm, (T*)H->xp, Tn * c.top_k, c.top_k, c.d_model, H->stream);
@@ -739,9 +748,10 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
       if (hidden_out && l + 1 == c.n_layers) nw = nullptr;
       launch_combine<T>(H->h, (const T*)H->y, H->wts, c.top_k, nw, xn, Tn, c.d_model, eps, H->stream);
     }
+    if (rec && dump->hidden_out) cudaMemcpyAsync(dump->hidden_out, H->h, hbytes, cudaMemcpyDeviceToDevice, H->stream);
   }
   if (hidden_out) {
-    cudaMemcpyAsync(hidden_out, H->h, (size_t)Tn * c.d_model * sizeof(float), cudaMemcpyDeviceToDevice, H->stream);
+    cudaMemcpyAsync(hidden_out, H->h, hbytes, cudaMemcpyDeviceToDevice, H->stream);
     if (head) {
       ProfScope ps(H, PC_NORM);
       launch_rmsnorm<T>(H->h, H->final_norm, xn, Tn, c.d_model, eps, H->stream);
@@ -752,9 +762,9 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
 }
 
 void run_layers(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const int32_t* tokens, const int32_t* prev,
-                bool head, float* logits, float* hidden_out) {
-  if (H->bf16) run_layers_t<__nv_bfloat16>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out);
-  else run_layers_t<float>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out);
+                bool head, float* logits, float* hidden_out, const dg_layer_dump* dump = nullptr) {
+  if (H->bf16) run_layers_t<__nv_bfloat16>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out, dump);
+  else run_layers_t<float>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out, dump);
 }
 
 int make_batch(dg_handle* H, int batch, const int* req, BatchInfo* bi) {
@@ -905,6 +915,17 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
         if (!p || !aligned16(p)) return fail(nullptr, DG_EINVAL, "layer %d: null or unaligned weight", l);
     }
     if (!aligned16(w->embed) || !aligned16(w->w_sc)) return fail(nullptr, DG_EINVAL, "unaligned embed / w_sc");
+    // the router needs finite gate logits: a non-finite bias is refused here
+    std::vector<float> bias_h(c.n_experts);
+    for (int l = 0; l < c.n_layers; ++l) {
+      if (!w->layers[l].router_b) continue;
+      if (cudaMemcpy(bias_h.data(), w->layers[l].router_b, c.n_experts * sizeof(float), cudaMemcpyDeviceToHost) !=
+          cudaSuccess)
+        return fail(nullptr, DG_EINVAL, "layer %d: router_b is not a readable device pointer (%s)", l,
+                    cudaGetErrorString(cudaGetLastError()));
+      for (float b : bias_h)
+        if (!std::isfinite(b)) return fail(nullptr, DG_EINVAL, "layer %d: router_b holds a non-finite value", l);
+    }
   }
   dg_handle* H = new dg_handle();
   H->c = c;
@@ -1112,6 +1133,26 @@ int dg_set_kv(dg_handle* H, int req, int layer, const void* k, const void* v, in
   return check_launch(H, "set_kv");
 }
 
+int dg_get_kv(dg_handle* H, int req, int layer, void* k, void* v, int n) {
+  if (!H) return DG_EINVAL;
+  const dg_config& c = H->c;
+  if (c.n_layers == 0) return fail(H, DG_ESTATE, "sampler-only handle");
+  if (req < 0 || req >= c.max_batch || layer < 0 || layer >= c.n_layers || !k || !v || n < 0)
+    return fail(H, DG_EINVAL, "bad get_kv arguments");
+  if (n > c.max_ctx) return fail(H, DG_ECAPACITY, "n exceeds max_ctx");
+  const size_t slot_off = (size_t)req * c.n_kv_heads * c.max_ctx * c.head_dim * H->esz;
+  const char* kc = (const char*)kc_layer(H, layer) + slot_off;
+  const char* vt = (const char*)vt_layer(H, layer) + slot_off;
+  if (H->bf16)
+    launch_get_kv<__nv_bfloat16>((const __nv_bfloat16*)kc, (const __nv_bfloat16*)vt, (__nv_bfloat16*)k,
+                                 (__nv_bfloat16*)v, c.n_kv_heads, n, c.head_dim, c.max_ctx, H->stream);
+  else
+    launch_get_kv<float>((const float*)kc, (const float*)vt, (float*)k, (float*)v, c.n_kv_heads, n, c.head_dim,
+                         c.max_ctx, H->stream);
+  H->launches += n > 0 ? 1 : 0;
+  return check_launch(H, "get_kv");
+}
+
 int dg_prefill_prompt(dg_handle* H, int batch, const int* req, const int32_t* tokens, int n) {
   if (!H) return DG_EINVAL;
   if (H->c.n_layers == 0) return fail(H, DG_ESTATE, "sampler-only handle");
@@ -1125,11 +1166,8 @@ int dg_prefill_prompt(dg_handle* H, int batch, const int* req, const int32_t* to
   return encode_causal(H, bi, tokens, n, n);
 }
 
-// where a step writes its argmax rows: the caller's buffer, else (the two-round stop needs them) the handle's
-static int32_t* argmax_target(dg_handle* H, const SamplerArgs& a, const dg_step_out* o) {
-  if (o && o->argmax) return o->argmax;
-  return a.stop_mode == DG_STOP_TWO_ROUNDS ? H->amax[0] : nullptr;
-}
+// where a step writes its argmax rows: the caller's buffer (the two-round stop requires one), else nowhere
+static int32_t* argmax_target(const dg_step_out* o) { return (o && o->argmax) ? o->argmax : nullptr; }
 
 int dg_sample(dg_handle* H, const float* logits, int batch, const int* req, int step, const dg_sampler_params* sp,
               int32_t* canvas, const dg_step_out* o) {
@@ -1140,11 +1178,13 @@ int dg_sample(dg_handle* H, const float* logits, int batch, const int* req, int 
   if ((rc = check_sampler_params(H, sp))) return rc;
   if (!logits || !canvas) return fail(H, DG_EINVAL, "null logits or canvas");
   if (!aligned16(logits)) return fail(H, DG_EINVAL, "logits must be 16-byte aligned");
+  if (sp->stop_mode == DG_STOP_TWO_ROUNDS && !(o && o->argmax))
+    return fail(H, DG_EINVAL, "the two-round stop needs o->argmax (the next round's prev_argmax)");
   if ((rc = upload_req(H, bi))) return rc;
   const SamplerArgs a = sampler_args(*sp, step);
   run_sampler(H, logits, bi, a, canvas, (o && o->x_hat) ? o->x_hat : H->xh[0], (o && o->pmax) ? o->pmax : H->pmax,
               (o && o->entropy) ? o->entropy : H->ent, o ? o->keep : nullptr, o ? o->mean_entropy : nullptr,
-              o ? o->stop : nullptr, nullptr, nullptr, 0, argmax_target(H, a, o));
+              o ? o->stop : nullptr, nullptr, nullptr, 0, argmax_target(o));
   return check_launch(H, "sample");
 }
 
@@ -1161,13 +1201,17 @@ int dg_denoise_step(dg_handle* H, const dg_step_args* a, const dg_step_out* o) {
   if (a->step < 1) return fail(H, DG_EINVAL, "step must be >= 1");
   for (int b = 0; b < bi.B; ++b)
     if (bi.len[b] + c.canvas > c.max_ctx) return fail(H, DG_ECAPACITY, "cache + canvas exceeds max_ctx");
+  if (a->dump && (a->dump->layer < 0 || a->dump->layer >= c.n_layers))
+    return fail(H, DG_EINVAL, "dump layer %d out of [0, %d)", a->dump->layer, c.n_layers);
+  if (a->sp.stop_mode == DG_STOP_TWO_ROUNDS && !(o && o->argmax))
+    return fail(H, DG_EINVAL, "the two-round stop needs o->argmax (the next round's prev_argmax)");
   if ((rc = upload_req(H, bi))) return rc;
   float* logits = a->logits_out ? a->logits_out : H->logits;
-  run_layers(H, bi, c.canvas, false, a->canvas, a->prev_pred, true, logits, a->hidden_out);
+  run_layers(H, bi, c.canvas, false, a->canvas, a->prev_pred, true, logits, a->hidden_out, a->dump);
   const SamplerArgs sa = sampler_args(a->sp, a->step);
   run_sampler(H, logits, bi, sa, a->canvas, (o && o->x_hat) ? o->x_hat : H->xh[0],
               (o && o->pmax) ? o->pmax : H->pmax, (o && o->entropy) ? o->entropy : H->ent, o ? o->keep : nullptr,
-              o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0, argmax_target(H, sa, o));
+              o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0, argmax_target(o));
   if (o && o->experts_touched)
     cudaMemcpyAsync(o->experts_touched, H->touched, c.n_layers * sizeof(int32_t), cudaMemcpyDeviceToDevice,
                     H->stream);
@@ -1364,6 +1408,33 @@ int dg_selftest_gemm_split(dg_handle* H, const void* x, const void* w, int T, in
   H->launches += 1;
   *nsplit = p.split;
   return check_launch(H, "selftest split gemm");
+}
+
+int dg_selftest_wait_timeout(dg_handle* H, int limit_us) {
+  if (!H) return DG_EINVAL;
+  if (limit_us < 1 || limit_us > 100000) return fail(H, DG_EINVAL, "limit_us out of [1, 100000]");
+  int rc = cuda_check(H, cudaStreamSynchronize(H->stream), "wait self-test: drain");
+  if (rc) return rc;
+  if ((rc = read_device_error(H))) return rc;
+  launch_wait_timeout_selftest(H->d_err, (unsigned long long)limit_us * 1000ull, H->stream);
+  H->launches += 1;
+  if ((rc = check_launch(H, "wait self-test"))) return rc;
+  return dg_synchronize(H);
+}
+
+int dg_selftest_router(dg_handle* H, const float* logits, const float* bias, int T, int E, int k, int tile,
+                       const dg_router_out* o) {
+  if (!H) return DG_EINVAL;
+  if (!logits || !o || !o->ids || !o->wts || !o->cnt || !o->off || !o->perm || !o->work || !o->n_work ||
+      !o->touched)
+    return fail(H, DG_EINVAL, "null router self-test argument");
+  if (T < 1 || E < 1 || E > 256 || k < 1 || k > 16 || k > E || tile < 1 || tile > 1024)
+    return fail(H, DG_EINVAL, "router self-test shape out of range (T %d, E %d, k %d, tile %d)", T, E, k, tile);
+  if ((long long)T * k > (long long)INT_MAX / 2) return fail(H, DG_EINVAL, "T * k too large");
+  launch_router_topk(logits, 1, bias, o->ids, o->wts, T, E, k, H->stream);
+  launch_router_permute(o->ids, T * k, E, tile, o->cnt, o->off, o->perm, o->work, o->n_work, o->touched, H->stream);
+  H->launches += 2;
+  return check_launch(H, "router self-test");
 }
 
 }  // extern "C"

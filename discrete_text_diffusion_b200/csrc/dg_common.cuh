@@ -21,6 +21,7 @@ constexpr int kErrTimeoutMma = 2;
 constexpr int kErrTimeoutEpi = 3;
 constexpr int kErrTimeoutAttn = 4;
 constexpr int kErrBadToken = 5;
+constexpr int kErrTimeoutSelftest = 6;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 // ------------------------------------------------------------ element types
@@ -125,19 +126,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 #ifndef DG_WAIT_ERR_PERIOD
 #define DG_WAIT_ERR_PERIOD 4096u    // polls between reads of the error flag
 #endif
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* err, int code,
+                                                unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it % DG_WAIT_TIME_PERIOD) == 0) {
       if ((it % DG_WAIT_ERR_PERIOD) == 0 && *(volatile int*)err != 0) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         atomicCAS(err, 0, code);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
+  return mbar_wait_limit(bar, parity, err, code, kWaitLimitNs);
 }
 
 // -------------------------------------------------------------------- TMA

@@ -19,11 +19,23 @@
 #include <mutex>
 
 #include "dg.h"
+#include "dg_common.cuh"
 #include "kernels.h"
 
 using namespace dg;
 
 namespace {
+
+// The request ids travel as a kernel argument, so a call makes no host-to-device copy.
+struct ReqIds {
+  int32_t v[64];
+};
+
+__global__ void store_req_ids_kernel(ReqIds ids, int n, int32_t* dst) {
+  pdl_wait();
+  pdl_trigger();
+  if ((int)threadIdx.x < n) dst[threadIdx.x] = ids.v[threadIdx.x];
+}
 
 constexpr size_t kScratchBytes = size_t(8) << 20;  // 8 MiB per device
 constexpr int kMaxReq = 64;                          // request ids held in the scratch
@@ -72,14 +84,15 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
     return report(err, err_len, DG_EINVAL, "entropy_budget must be finite and >= 0");
   if (sp->stop_mode != DG_STOP_MEAN_ENTROPY && sp->stop_mode != DG_STOP_TWO_ROUNDS)
     return report(err, err_len, DG_EINVAL, "unknown stop_mode %d", sp->stop_mode);
+  if (sp->stop_mode == DG_STOP_TWO_ROUNDS && !(o && o->argmax))
+    return report(err, err_len, DG_EINVAL, "the two-round stop needs o->argmax (the next round's prev_argmax)");
 
-  // scratch layout: request ids | x_hat | pmax | entropy | argmax | chunk partials
+  // scratch layout: request ids | x_hat | pmax | entropy | chunk partials
   const size_t rows = (size_t)batch * n;
   const size_t off_xh = round256(kMaxReq * sizeof(int32_t));
   const size_t off_pm = off_xh + round256(rows * sizeof(int32_t));
   const size_t off_en = off_pm + round256(rows * sizeof(float));
-  const size_t off_am = off_en + round256(rows * sizeof(float));
-  const size_t off_ws = off_am + round256(rows * sizeof(int32_t));
+  const size_t off_ws = off_en + round256(rows * sizeof(float));
   const size_t need = off_ws + round256(sampler_workspace_bytes((int)rows, vocab));
   if (need > kScratchBytes)
     return report(err, err_len, DG_ECAPACITY,
@@ -106,11 +119,10 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* req_dev = reinterpret_cast<int32_t*>(base);
-  int32_t ids[kMaxReq];
-  for (int b = 0; b < batch; ++b) ids[b] = req[b];
-  // a pageable source: the runtime stages it before this call returns
-  e = cudaMemcpyAsync(req_dev, ids, batch * sizeof(int32_t), cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return report(err, err_len, DG_ECUDA, "request id copy: %s", cudaGetErrorString(e));
+  ReqIds ids{};
+  for (int b = 0; b < batch; ++b) ids.v[b] = req[b];
+  e = launch_k(store_req_ids_kernel, dim3(1), dim3(kMaxReq), 0, s, ids, batch, req_dev);
+  if (e != cudaSuccess) return report(err, err_len, DG_ECUDA, "request id store: %s", cudaGetErrorString(e));
 
   int32_t* xh = (o && o->x_hat) ? o->x_hat : reinterpret_cast<int32_t*>(base + off_xh);
   float* pmax = (o && o->pmax) ? o->pmax : reinterpret_cast<float*>(base + off_pm);
@@ -128,9 +140,7 @@ int dg_sample_noalloc(const float* logits, int batch, int n, int vocab, const in
   a.stop_mode = sp->stop_mode;
   a.prev_argmax = sp->prev_argmax;
   a.prev_mean_h = sp->prev_mean_entropy;
-  int32_t* amax = (o && o->argmax) ? o->argmax
-                                   : (sp->stop_mode == DG_STOP_TWO_ROUNDS ? reinterpret_cast<int32_t*>(base + off_am)
-                                                                          : nullptr);
+  int32_t* amax = (o && o->argmax) ? o->argmax : nullptr;
   launch_sampler_rows(logits, (int)rows, n, vocab, req_dev, a, base + off_ws, xh, pmax, ent, s, amax);
   launch_sampler_finish(xh, pmax, ent, batch, n, vocab, req_dev, a, canvas, o ? o->keep : nullptr,
                         o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0, s, amax);

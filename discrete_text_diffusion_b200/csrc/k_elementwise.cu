@@ -631,6 +631,45 @@ void launch_set_kv(const T* k, const T* v, T* kc, T* vt, int hkv, int n, int hd,
   launch_k(set_kv_kernel<T>, dim3(dim3(n, hkv)), dim3(128), 0, s, k, v, kc, vt, n, hd, max_ctx);
 }
 
+// ----------------------------------------------------------------- get_kv
+// Inverse of set_kv: positions [0, n) of one request's cache -> k, v [Hkv, n, hd].
+template <typename T>
+__global__ void get_kv_kernel(const T* __restrict__ kc, const T* __restrict__ vt, T* __restrict__ k,
+                              T* __restrict__ v, int n, int hd, int max_ctx) {
+  pdl_wait();
+  pdl_trigger();
+  const int g = blockIdx.y;
+  const int p = blockIdx.x;
+  for (int j = threadIdx.x; j < hd; j += blockDim.x) {
+    k[((size_t)g * n + p) * hd + j] = kc[((size_t)g * max_ctx + p) * hd + j];
+    v[((size_t)g * n + p) * hd + j] = vt[((size_t)g * hd + j) * max_ctx + p];
+  }
+}
+
+template <typename T>
+void launch_get_kv(const T* kc, const T* vt, T* k, T* v, int hkv, int n, int hd, int max_ctx, cudaStream_t s) {
+  if (n <= 0) return;
+  launch_k(get_kv_kernel<T>, dim3(n, hkv), dim3(128), 0, s, kc, vt, k, v, n, hd, max_ctx);
+}
+
+// ------------------------------------------------------- wait self-test
+// One thread waits on an mbarrier that expects one arrival which never
+// comes; the bounded wait gives up after limit_ns and records the code.
+__global__ void wait_timeout_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait_limit(&bar, 0, err, kErrTimeoutSelftest, limit_ns);
+  }
+}
+
+void launch_wait_timeout_selftest(int* err, unsigned long long limit_ns, cudaStream_t s) {
+  launch_k(wait_timeout_selftest_kernel, dim3(1), dim3(32), 0, s, err, limit_ns);
+}
+
 // ------------------------------------------------------------ instantiation
 #define DG_INST(T)                                                                                          \
   template void launch_embed<T>(const int32_t*, const int32_t*, const T*, float*, T*, int, int, int, int*,    \
@@ -643,7 +682,8 @@ void launch_set_kv(const T* k, const T* v, T* kc, T* vt, int hkv, int n, int hd,
   template void launch_add_rmsnorm<T>(float*, const float*, int, size_t, const float*, T*, int, int, float,   \
                                       cudaStream_t);                                                         \
   template void launch_gather_rows<T>(const T*, const int32_t*, T*, int, int, int, cudaStream_t);            \
-  template void launch_set_kv<T>(const T*, const T*, T*, T*, int, int, int, int, cudaStream_t);
+  template void launch_set_kv<T>(const T*, const T*, T*, T*, int, int, int, int, cudaStream_t);             \
+  template void launch_get_kv<T>(const T*, const T*, T*, T*, int, int, int, int, cudaStream_t);
 DG_INST(float)
 DG_INST(__nv_bfloat16)
 #undef DG_INST

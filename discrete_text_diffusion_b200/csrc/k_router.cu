@@ -32,27 +32,32 @@ __global__ void router_topk_kernel(const float* __restrict__ glog, int nsplit, c
   }
   float sel_v[16];
   int sel_i[16];
+  uint32_t taken = 0;   // bit j: expert lane + 32 j already selected
   for (int r = 0; r < k; ++r) {
-    // best local candidate (lowest id wins ties: j ascending = id ascending)
+    // best local candidate among the experts not yet taken: the first one
+    // seen, then strictly larger values (j ascending = id ascending, so the
+    // lowest id wins ties, -inf included)
     float bv = -INFINITY;
     int bi = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int ex = lane + 32 * j;
-      if (ex < e && (v[j] > bv || (v[j] == bv && ex < bi))) { bv = v[j]; bi = ex; }
+      if (ex < e && !((taken >> j) & 1u) && (bi == 0x7fffffff || v[j] > bv)) { bv = v[j]; bi = ex; }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
     }
+    // every lane takes lane 0's winner, so the removal below agrees with the output
+    bv = __shfl_sync(0xffffffffu, bv, 0);
+    bi = __shfl_sync(0xffffffffu, bi, 0);
     sel_v[r] = bv;
     sel_i[r] = bi;
-    // remove the winner
 #pragma unroll
     for (int j = 0; j < kPer; ++j)
-      if (lane + 32 * j == bi) v[j] = -INFINITY;
+      if (lane + 32 * j == bi) taken |= 1u << j;
   }
   if (lane == 0) {
     const float m = sel_v[0];
@@ -111,24 +116,26 @@ __global__ void router_topk_vec_kernel(const float* __restrict__ glog, int nspli
   }
   float sel_v[16];
   int sel_i[16];
+  uint32_t taken = 0;   // bit j: expert lane * EPL + j already selected
   for (int r = 0; r < k; ++r) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
 #pragma unroll
-    for (int j = 0; j < EPL; ++j)
-      if (v[j] > bv) { bv = v[j]; bi = lane * EPL + j; }   // ascending ids: the first of equals wins
-    if (bi == 0x7fffffff) bi = lane * EPL;                  // all -inf: lowest own id
+    for (int j = 0; j < EPL; ++j)   // ascending ids: the first of equals wins, -inf included
+      if (!((taken >> j) & 1u) && (bi == 0x7fffffff || v[j] > bv)) { bv = v[j]; bi = lane * EPL + j; }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
     }
+    bv = __shfl_sync(0xffffffffu, bv, 0);
+    bi = __shfl_sync(0xffffffffu, bi, 0);
     sel_v[r] = bv;
     sel_i[r] = bi;
 #pragma unroll
     for (int j = 0; j < EPL; ++j)
-      if (lane * EPL + j == bi) v[j] = -INFINITY;
+      if (lane * EPL + j == bi) taken |= 1u << j;
   }
   if (lane == 0) {
     const float m = sel_v[0];

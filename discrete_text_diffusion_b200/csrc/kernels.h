@@ -54,6 +54,13 @@ template <typename T>
 void launch_set_kv(const T* k, const T* v, T* kc, T* vt, int hkv, int n, int hd, int max_ctx,
                    cudaStream_t s);
 
+// Copy positions [0, n) of one request's cache out to [Hkv, n, hd] K/V blocks.
+template <typename T>
+void launch_get_kv(const T* kc, const T* vt, T* k, T* v, int hkv, int n, int hd, int max_ctx,
+                   cudaStream_t s);
+// One thread waits on an mbarrier nothing arrives on; records a timeout after limit_ns.
+void launch_wait_timeout_selftest(int* err, unsigned long long limit_ns, cudaStream_t s);
+
 // ---- router (k_router.cu)
 // Per token: g = glog + bias; top-k (ties -> lower id); softmax over the k.
 // glog holds nsplit partial-sum slices of [n_tok, e] at a stride of n_tok*e

@@ -23,7 +23,8 @@ EXPORTS = (
     "dg_create", "dg_destroy", "dg_last_error", "dg_prefill_prompt", "dg_set_kv", "dg_set_length",
     "dg_get_length", "dg_denoise_step", "dg_sample", "dg_generate_block", "dg_generate_block_host",
     "dg_synchronize", "dg_launch_count", "dg_profile_enable", "dg_profile_read", "dg_profile_reset",
-    "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc", "dg_selftest_gemm_split",
+    "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc", "dg_selftest_gemm_split", "dg_get_kv",
+    "dg_selftest_router", "dg_selftest_wait_timeout",
 )
 
 
@@ -62,10 +63,19 @@ class DgStepOut(C.Structure):
                                           "experts_touched", "argmax")]
 
 
+class DgLayerDump(C.Structure):
+    _fields_ = [("layer", C.c_int), ("hidden_in", C.c_void_p), ("hidden_out", C.c_void_p),
+                ("expert_ids", C.c_void_p), ("expert_wts", C.c_void_p)]
+
+
 class DgStepArgs(C.Structure):
     _fields_ = [("batch", C.c_int), ("req", C.POINTER(C.c_int)), ("canvas", C.c_void_p),
                 ("prev_pred", C.c_void_p), ("step", C.c_int), ("sp", DgSamplerParams),
-                ("logits_out", C.c_void_p), ("hidden_out", C.c_void_p)]
+                ("logits_out", C.c_void_p), ("hidden_out", C.c_void_p), ("dump", C.POINTER(DgLayerDump))]
+
+
+class DgRouterOut(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("ids", "wts", "cnt", "off", "perm", "work", "n_work", "touched")]
 
 
 class DgBlockArgs(C.Structure):
@@ -98,6 +108,9 @@ def lib():
         L.dg_last_error.restype = C.c_char_p
         L.dg_prefill_prompt.argtypes = [P, C.c_int, C.POINTER(C.c_int), P, C.c_int]
         L.dg_set_kv.argtypes = [P, C.c_int, C.c_int, P, P, C.c_int]
+        L.dg_get_kv.argtypes = [P, C.c_int, C.c_int, P, P, C.c_int]
+        L.dg_selftest_router.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(DgRouterOut)]
+        L.dg_selftest_wait_timeout.argtypes = [P, C.c_int]
         L.dg_set_length.argtypes = [P, C.c_int, C.c_int]
         L.dg_get_length.argtypes = [P, C.c_int, C.POINTER(C.c_int)]
         L.dg_denoise_step.argtypes = [P, C.POINTER(DgStepArgs), C.POINTER(DgStepOut)]
@@ -210,6 +223,11 @@ def dg_set_kv(h: Handle, req: int, layer: int, k: torch.Tensor, v: torch.Tensor)
     return h.check(lib().dg_set_kv(h.ptr, req, layer, _ptr(k), _ptr(v), k.shape[1]))
 
 
+def dg_get_kv(h: Handle, req: int, layer: int, k: torch.Tensor, v: torch.Tensor):
+    """Read positions [0, n) of a request's cache of one layer into k, v [Hkv, n, hd]."""
+    return h.check(lib().dg_get_kv(h.ptr, req, layer, _ptr(k), _ptr(v), k.shape[1]))
+
+
 def dg_set_length(h: Handle, req: int, length: int):
     return h.check(lib().dg_set_length(h.ptr, req, length))
 
@@ -239,11 +257,18 @@ def step_out(x_hat=None, pmax=None, entropy=None, keep=None, mean_entropy=None, 
                        (x_hat, pmax, entropy, keep, mean_entropy, stop, experts_touched, argmax)])
 
 
+def layer_dump(layer, hidden_in=None, hidden_out=None, expert_ids=None, expert_wts=None):
+    """A dg_layer_dump: record one layer of the next forward pass into these device tensors."""
+    return DgLayerDump(layer, *[None if t is None else t.data_ptr()
+                                for t in (hidden_in, hidden_out, expert_ids, expert_wts)])
+
+
 def dg_denoise_step(h: Handle, req, canvas, prev_pred, step, sp: DgSamplerParams, out: DgStepOut,
-                    logits_out=None, hidden_out=None):
+                    logits_out=None, hidden_out=None, dump: DgLayerDump = None):
     a = DgStepArgs(len(req), _ints(req), canvas.data_ptr(), None if prev_pred is None else prev_pred.data_ptr(),
                    step, sp, None if logits_out is None else logits_out.data_ptr(),
-                   None if hidden_out is None else hidden_out.data_ptr())
+                   None if hidden_out is None else hidden_out.data_ptr(),
+                   None if dump is None else C.pointer(dump))
     return h.check(lib().dg_denoise_step(h.ptr, C.byref(a), C.byref(out)))
 
 
@@ -329,6 +354,19 @@ def dg_selftest_philox(h: Handle, ctr, key, out, out_curand=None):
 def dg_selftest_gemm(h: Handle, x, w, out):
     """out[T, M] fp32 = x[T, K] @ w[M, K]^T through the tensor-core GEMM."""
     return h.check(lib().dg_selftest_gemm(h.ptr, _ptr(x), _ptr(w), x.shape[0], w.shape[0], x.shape[1], _ptr(out)))
+
+
+def dg_selftest_wait_timeout(h: Handle, limit_us: int) -> int:
+    """Run the wait self-test; returns the status code (DG_ETIMEOUT when the wait gave up as designed)."""
+    return int(lib().dg_selftest_wait_timeout(h.ptr, int(limit_us)))
+
+
+def dg_selftest_router(h: Handle, logits, bias, k: int, tile: int, out: dict):
+    """Router self-test on logits [T, E] fp32 (+ bias [E] or None); out: dict of device tensors
+    ids, wts, cnt, off, perm, work, n_work, touched."""
+    T, E = logits.shape
+    o = DgRouterOut(*[out[n].data_ptr() for n, _ in DgRouterOut._fields_])
+    return h.check(lib().dg_selftest_router(h.ptr, _ptr(logits), _ptr(bias), T, E, k, tile, C.byref(o)))
 
 
 def dg_selftest_gemm_split(h: Handle, x, w, part):

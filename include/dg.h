@@ -154,6 +154,16 @@ typedef struct dg_step_out {
                                 round's prev_argmax for DG_STOP_TWO_ROUNDS */
 } dg_step_out;
 
+/* A record of one layer of a forward pass, for layer-wise checks.  Rows are
+ * the pass's B*N canvas positions in batch order (row b*N + i). */
+typedef struct dg_layer_dump {
+  int layer;             /* layer index, 0 .. n_layers-1 */
+  float* hidden_in;      /* [B*N, d] fp32 residual stream entering the layer, or NULL */
+  float* hidden_out;     /* [B*N, d] fp32 residual stream leaving it (after the MoE residual), or NULL */
+  int32_t* expert_ids;   /* [B*N, k] the router's experts in this layer, selection order, or NULL */
+  float* expert_wts;     /* [B*N, k] their softmax weights, or NULL */
+} dg_layer_dump;
+
 /* One denoising step ([P1 一/二/四]). */
 typedef struct dg_step_args {
   int batch;                   /* B <= max_batch */
@@ -165,6 +175,7 @@ typedef struct dg_step_args {
   float* logits_out;           /* [B, N, V] fp32 to receive the logits (16-byte aligned), or NULL */
   float* hidden_out;           /* [B*N, d] fp32 residual stream before the final
                                   norm, or NULL */
+  const dg_layer_dump* dump;   /* HOST pointer: record one layer of this pass, or NULL */
 } dg_step_args;
 
 /* One block ([P1 一/四], [P2], [P3]). */
@@ -225,6 +236,13 @@ int dg_prefill_prompt(dg_handle* h, int batch, const int* req, const int32_t* to
  */
 int dg_set_kv(dg_handle* h, int req, int layer, const void* k, const void* v, int n);
 
+/*
+ * Test hook: read positions [0, n) of one layer's cache for request req into
+ * k, v: [Hkv, n, hd] in the handle's dtype (K as RoPE'd, V as projected).
+ * Does not change P.  DG_ECAPACITY if n > max_ctx.
+ */
+int dg_get_kv(dg_handle* h, int req, int layer, void* k, void* v, int n);
+
 /* Set / read a request's cache length P (host-side state; set checks capacity). */
 int dg_set_length(dg_handle* h, int req, int length);
 int dg_get_length(const dg_handle* h, int req, int* length);
@@ -249,7 +267,9 @@ int dg_denoise_step(dg_handle* h, const dg_step_args* a, const dg_step_out* o);
  * mean entropy and stop = mean < stop_threshold.
  * logits must be 16-byte aligned (DG_EINVAL otherwise); an unknown keep_mode
  * or stop_mode, or a negative or non-finite entropy_budget, is DG_EINVAL.
- * With DG_STOP_TWO_ROUNDS the stop follows that mode's definition.
+ * With DG_STOP_TWO_ROUNDS the stop follows that mode's definition, and o->argmax
+ * is required (DG_EINVAL without it): pass it back as the next round's
+ * prev_argmax.  dg_denoise_step follows the same rule.
  */
 int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int step,
               const dg_sampler_params* sp, int32_t* canvas, const dg_step_out* o);
@@ -273,9 +293,8 @@ int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int 
  *   n: canvas length, 1..1024.
  *   step, sp: as for dg_sample; sp->keep_k <= n.
  *   canvas: device [batch, n]; in: unused, out: the re-noised canvas.
- *   o: as for dg_sample, or NULL.  x_hat / pmax / entropy (and the argmax a
- *      two-round stop needs) that o does not request are kept in the
- *      scratch; experts_touched is ignored.
+ *   o: as for dg_sample, or NULL.  x_hat / pmax / entropy that o does not
+ *      request are kept in the scratch; experts_touched is ignored.
  *   stream: a cudaStream_t of the current device (NULL = legacy default).
  *   err: buffer of err_len bytes for a message (may be NULL).
  *
@@ -291,8 +310,10 @@ int dg_sample(dg_handle* h, const float* logits, int batch, const int* req, int 
  *   - Every call on a device shares the one scratch.  Calls on a device must
  *     therefore be ordered: the same stream, or streams ordered by events.
  *     Overlapping calls race on the scratch and give wrong results.
- *   - The request ids are copied from pageable host memory, so the call may
- *     wait for earlier work on the stream.
+ *   - The request ids travel to the device as a kernel argument: the call
+ *     makes no host-to-device copy and does not wait for the stream.
+ *   - DG_STOP_TWO_ROUNDS needs o->argmax (DG_EINVAL without it): that row is
+ *     the next round's prev_argmax, which the shared scratch cannot keep.
  *   - Returns DG_OK, DG_EINVAL (bad argument), DG_ECAPACITY (too large) or
  *     DG_ECUDA (a launch or runtime call failed).
  */
@@ -380,6 +401,41 @@ int dg_selftest_gemm(dg_handle* h, const void* x, const void* w, int T, int M, i
  */
 int dg_selftest_gemm_split(dg_handle* h, const void* x, const void* w, int T, int M, int K, float* part,
                            int max_split, int* nsplit);
+
+/*
+ * Test hook for the bounded device waits: one kernel waits on a shared-memory
+ * barrier that nothing arrives on, gives up after limit_us microseconds of wall
+ * time (1 .. 100000), records the timeout and returns.  The call synchronises
+ * and returns what any synchronising call then reports: DG_ETIMEOUT, with the
+ * device error flag cleared, so the handle stays usable.
+ */
+int dg_selftest_wait_timeout(dg_handle* h, int limit_us);
+
+/* Outputs of the router self-test (all device pointers, all required). */
+typedef struct dg_router_out {
+  int32_t* ids;      /* [T, k] selected experts, in selection order (logit desc, id asc) */
+  float* wts;        /* [T, k] softmax of the k selected biased logits */
+  int32_t* cnt;      /* [E] items routed to each expert */
+  int32_t* off;      /* [E + 1] exclusive prefix sum of cnt */
+  int32_t* perm;     /* [T * k] item t*k+s at position off[e] + (its rank among expert e's items, by item index) */
+  int32_t* work;     /* [3 * (E + ceil(T * k / tile))] (expert, first position, rows <= tile) tiles, experts
+                        ascending */
+  int32_t* n_work;   /* [1] number of work tiles */
+  int32_t* touched;  /* [1] number of experts with cnt > 0 */
+} dg_router_out;
+
+/*
+ * Test hook: the router of one layer ([P1 二]: 128 experts, 8 per token) run
+ * by the kernels the layers use, on caller logits.  logits [T, E] fp32 (the
+ * gate projection x W_r^T), bias [E] fp32 or NULL, both 16-byte aligned for the
+ * vector form (any alignment works).  g = logits + bias; top-k by g with ties
+ * to the lower id (no expert twice, -inf included); softmax over the k
+ * selected; then the counting sort into expert order, the work list and the
+ * distinct-expert count.  E <= 256, k <= min(E, 16), 1 <= tile <= 1024.
+ * Uses the handle's stream; h may be a sampler-only handle.
+ */
+int dg_selftest_router(dg_handle* h, const float* logits, const float* bias, int T, int E, int k, int tile,
+                       const dg_router_out* o);
 
 #ifdef __cplusplus
 }

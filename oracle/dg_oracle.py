@@ -195,6 +195,16 @@ def router(x, w_router, b_router, top_k):
     g = x @ w_router.T
     if b_router is not None:
         g = g + np.asarray(b_router, np.float64)
+    ids, w, margin = router_select(g, top_k)
+    return ids, w, g, margin
+
+
+def router_select(g, top_k):
+    """The selection step of R-router on gate logits g [T, E] (bias included):
+    the top_k experts by logit, ties to the lower id (-inf logits rank last,
+    among themselves by id), and the softmax over the selected logits.
+    Returns (ids [T,k] in selection order, weights [T,k], margin [T])."""
+    g = np.asarray(g, np.float64)
     n_e = g.shape[1]
     idx = np.arange(n_e)
     ids = np.empty((g.shape[0], top_k), dtype=np.int64)
@@ -203,11 +213,34 @@ def router(x, w_router, b_router, top_k):
         order = np.lexsort((idx, -g[t]))          # logit descending, then id ascending
         ids[t] = order[:top_k]
         if top_k < n_e:
-            margin[t] = g[t, order[top_k - 1]] - g[t, order[top_k]]
+            a, b = g[t, order[top_k - 1]], g[t, order[top_k]]
+            margin[t] = 0.0 if a == b else a - b          # -inf next to -inf is an exact tie
     sel = np.take_along_axis(g, ids, axis=1)
     e = np.exp(sel - sel.max(axis=1, keepdims=True))
     w = e / e.sum(axis=1, keepdims=True)
-    return ids, w, g, margin
+    return ids, w, margin
+
+
+def expert_order(ids, n_experts, tile):
+    """The routed (token, slot) items grouped by expert, as the experts process
+    them ([P1 二]: each token goes to its top-k experts of 128).  Item t*k+s is
+    token t's s-th choice ids[t, s].
+
+    Returns cnt [E] (items per expert), off [E+1] (exclusive prefix sum of cnt),
+    perm [T*k] (the items of expert 0, then expert 1, ...; inside an expert by
+    ascending item index, so tokens ascending), the work tiles [(expert, first
+    position in perm, rows)] that cut each expert's run into pieces of at most
+    `tile` rows (experts ascending), and the number of experts touched.
+    """
+    items = np.asarray(ids).reshape(-1)
+    cnt = np.array([int(np.sum(items == e)) for e in range(n_experts)], dtype=np.int64)
+    off = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int64)
+    perm = np.empty(items.shape[0], dtype=np.int64)
+    for e in range(n_experts):
+        perm[off[e]:off[e + 1]] = np.nonzero(items == e)[0]
+    work = [(e, int(off[e]) + r0, int(min(tile, cnt[e] - r0)))
+            for e in range(n_experts) for r0 in range(0, int(cnt[e]), tile)]
+    return cnt, off, perm, work, int(np.sum(cnt > 0))
 
 
 def moe(x, layer, top_k):

@@ -46,6 +46,7 @@ _STRUCTS = {
     "dg_config": B.DgConfig, "dg_layer_weights": B.DgLayerWeights, "dg_weights": B.DgWeights,
     "dg_sampler_params": B.DgSamplerParams, "dg_step_out": B.DgStepOut, "dg_step_args": B.DgStepArgs,
     "dg_block_args": B.DgBlockArgs, "dg_profile_entry": B.DgProfileEntry,
+    "dg_layer_dump": B.DgLayerDump, "dg_router_out": B.DgRouterOut,
 }
 
 
@@ -183,3 +184,53 @@ def test_bench_algorithmic_counts_match_brute_force():
     # gate+up bytes: touched experts' two [F, d] bf16 matrices, the rows read, the bf16 SwiGLU rows written
     d, f = model["d_model"], model["d_ff"]
     assert bench.moe_up_bytes(model, 10, 3) == 3 * 2 * f * d * 2 + 10 * d * 2 + 10 * f * 2
+
+
+def test_bench_pass_cost_matches_weight_tensors_and_product_shapes():
+    """bench.pass_cost's bytes against the sizes of the synthetic weight tensors
+    (bf16) plus the KV traffic, and its flops against the products of one layer
+    written out shape by shape."""
+    import bench
+    from discrete_text_diffusion_b200 import synth
+    model = dict(n_layers=2, d_model=64, n_heads=4, n_kv_heads=2, head_dim=16, n_experts=6, top_k=2, d_ff=32,
+                 vocab=100, canvas=8, rope_base=10000.0, rms_eps=1e-6)
+    w = synth.make_weights(model, seed=0, dtype="bf16", router_bias=True)
+    L0 = w["layers"][0]
+    touched = 3
+    attn = sum(L0[k].numel() for k in ("wq", "wk", "wv", "wo")) * 2
+    router = L0["router_w"].numel() * 2
+    expert = (L0["w_gate"][0].numel() + L0["w_up"][0].numel() + L0["w_down"][0].numel()) * 2
+    B, n, P = 2, model["canvas"], 11
+    kv = 2 * model["n_kv_heads"] * model["head_dim"] * 2           # K and V bf16 per position
+    want_b = model["n_layers"] * (attn + router + touched * expert + B * P * kv + 2 * B * n * kv) \
+        + w["embed"].numel() * 2 + w["w_sc"].numel() * 2
+    d, hq, hkv, hd, F, E, k, V = 64, 4, 2, 16, 32, 6, 2, 100
+    T = B * n
+    mm = lambda m_, k_, n_: 2 * m_ * k_ * n_
+    layer = mm(T, d, hq * hd) + 2 * mm(T, d, hkv * hd) + mm(T, hq * hd, d) + mm(T, d, E) \
+        + T * k * (2 * mm(1, d, F) + mm(1, F, d))
+    attn_fl = B * hq * n * (P + n) * (mm(1, hd, 1) + mm(1, 1, hd))
+    want_f = model["n_layers"] * (layer + attn_fl) + mm(T, d, V) + mm(T, d, d)
+    b, f = bench.pass_cost(model, B, n, P, touched, causal=False, head=True, self_cond=True)
+    assert b == want_b and f == want_f
+    # the causal hand-off: query i sees P + i + 1 keys, no head, no self-conditioning
+    b2, f2 = bench.pass_cost(model, B, n, P, touched, causal=True, head=False, self_cond=False)
+    attn_c = B * hq * sum(P + i + 1 for i in range(n)) * (mm(1, hd, 1) + mm(1, 1, hd))
+    assert f2 == model["n_layers"] * (layer + attn_c)
+    assert b2 == want_b - w["embed"].numel() * 2 - w["w_sc"].numel() * 2
+
+
+def test_bench_block_roofline_sums_pass_bounds():
+    import bench
+    model = dict(n_layers=1, d_model=64, n_heads=2, n_kv_heads=1, head_dim=64, n_experts=4, top_k=1, d_ff=64,
+                 vocab=64, canvas=4)
+    peaks = {"hbm_gbs": 1.0, "bf16_tflops": 1.0, "bf16_tflops_sustained": 1.0}
+    r = bench.block_roofline(model, 1, 4, [(10, 3)], 2, 1000.0, peaks)
+    want = 0.0
+    for t in (1, 2, 3):
+        b, f = bench.pass_cost(model, 1, 4, 10, 2, False, True, t > 1)
+        want += max(b / 1e9, f / 1e12)
+    b, f = bench.pass_cost(model, 1, 4, 10, 2, True, False, False)
+    want += max(b / 1e9, f / 1e12)
+    assert abs(r["bound_ms_per_block"] - round(want * 1e3, 3)) < 1e-6
+    assert abs(r["frac"] - round(want / 1.0, 4)) < 1e-6

@@ -16,6 +16,11 @@ test_gpu_layer.py.)
 - Keep count and keep set; kept positions hold x_hat and the others the Philox
   re-noise token; the mean entropy and the stop flag.
 - Determinism of whole blocks, and the KV length after each hand-off.
+- Layer by layer at layers 0, 14 and 29: the step records the residual stream
+  entering and leaving the layer and the router's experts; the oracle runs the
+  same layer on the GPU's own input and the request's cache as the GPU holds
+  it (read back with dg_get_kv), on the canvas step of full_b1 (cache 8192)
+  and of full_b16 (cache 4096, and 4352 after one hand-off).
 """
 import gc
 
@@ -111,6 +116,127 @@ def _check_step(dg, W, w, h, req, step, block, temperature, scale, keep_k, stop,
         if stop >= 0 and abs(mh - stop) > 1e-5:
             assert bool(got["stop"][bi]) == (mh < stop)
     return got
+
+
+PIN_LAYERS = (0, 14, 29)
+ROUTER_MARGIN = 0.02      # router decisions closer than this are rounding-order ties (bf16 router input)
+
+
+class _Experts:
+    """One layer's stacked expert matrix [E, out, in] on the device, handed to
+    the oracle one expert at a time (as float32 numpy, exact for bf16)."""
+
+    def __init__(self, t):
+        self.t = t
+        self.cache = {}
+
+    def __getitem__(self, e):
+        e = int(e)
+        if e not in self.cache:
+            self.cache[e] = to_np(self.t[e].float())
+        return self.cache[e]
+
+
+def _oracle_layer_weights(w, li):
+    L = w["layers"][li]
+    out = {k: (None if v is None else to_np(v.float())) for k, v in L.items()
+           if k not in ("w_gate", "w_up", "w_down")}
+    for k in ("w_gate", "w_up", "w_down"):
+        out[k] = _Experts(L[k])
+    return out
+
+
+def _layer_pins(dg, W, w, h, req, block, check, layers=PIN_LAYERS):
+    """One canvas step per pinned layer, recording that layer; each request in
+    `check` is compared with the oracle's layer on the GPU's input.  Returns the
+    fraction of checked tokens excluded as router near-ties."""
+    M = W["model"]
+    n, d, k = M["canvas"], M["d_model"], M["top_k"]
+    B = len(req)
+    seed = W["sampler"]["seed"]
+    canvas0 = np.stack([O.init_canvas(seed, n, M["vocab"], block, r) for r in req]).astype(np.int32)
+    excluded, total = 0, 0
+    for li in layers:
+        hin = torch.empty((B * n, d), device="cuda")
+        hout = torch.empty((B * n, d), device="cuda")
+        ids = torch.empty((B * n, k), dtype=torch.int32, device="cuda")
+        wts = torch.empty((B * n, k), device="cuda")
+        sp = dg.sampler_params(temperature=1.0, keep_k=n // 2, seed=seed, block=block)
+        dg.dg_denoise_step(h, req, torch.from_numpy(canvas0).cuda(), None, 1, sp, dg.step_out(),
+                           dump=dg.layer_dump(li, hin, hout, ids, wts))
+        dg.dg_synchronize(h)
+        om = O.OracleModel(dict(M), {"layers": {li: _oracle_layer_weights(w, li)}})
+        for bi, r in enumerate(req):
+            if r not in check:
+                continue
+            P = dg.dg_get_length(h, r)
+            kc = torch.empty((M["n_kv_heads"], P, M["head_dim"]), dtype=torch.bfloat16, device="cuda")
+            vc = torch.empty_like(kc)
+            dg.dg_get_kv(h, r, li, kc, vc)
+            dg.dg_synchronize(h)
+            om.set_kv(r, li, to_np(kc.float()), to_np(vc.float()))
+            rows = slice(bi * n, (bi + 1) * n)
+            x_in = to_np(hin[rows]).astype(np.float64)
+            tr = {}
+            ref, _, _ = om.layer(x_in, li, r, P + np.arange(n), causal=False, trace=tr)
+            got = to_np(hout[rows]).astype(np.float64)
+            gids = to_np(ids[rows])
+            same = np.array([set(a) == set(b) for a, b in zip(gids.tolist(), tr["router_ids"].tolist())])
+            # a token routed differently must be a near-tie of the oracle's router
+            assert (tr["router_margin"][~same] < ROUTER_MARGIN).all(), \
+                f"layer {li} req {r}: experts differ at margins {tr['router_margin'][~same]}"
+            excluded += int((~same).sum())
+            total += n
+            err = float(np.max(np.abs(got[same] - ref[same])) / np.max(np.abs(ref)))
+            assert err < TOL_BF16, f"layer {li} req {r}: output max-abs-rel {err}"
+            # the layer's own contribution, out - in (the input is shared, so this isolates the layer)
+            dref = ref - x_in
+            derr = float(np.max(np.abs((got - x_in)[same] - dref[same])) / np.max(np.abs(dref)))
+            assert derr < TOL_BF16, f"layer {li} req {r}: layer-delta max-abs-rel {derr}"
+            gw = to_np(wts[rows])
+            wmap = [dict(zip(a, b)) for a, b in zip(gids.tolist(), gw.tolist())]
+            _, wref, _, _ = O.router(tr["moe_in"], om.weights["layers"][li]["router_w"],
+                                     om.weights["layers"][li]["router_b"], k)
+            for t in np.nonzero(same)[0][:64]:
+                for e, wv in zip(tr["router_ids"][t], wref[t]):
+                    assert abs(wmap[t][int(e)] - wv) < 2e-2 * max(wv, 1e-3) + 1e-3
+    frac = excluded / max(1, total)
+    print(f"router near-ties excluded: {excluded}/{total} = {frac:.4f}")
+    assert frac < 0.10
+    return frac
+
+
+@pytest.mark.gpu
+@pytest.mark.slow
+def test_full_b1_layer_pins(dg):
+    """full_b1: 30 layers over an 8192-token cache, layers 0, 14, 29 against the oracle."""
+    W, w, h = _setup(dg, "full_b1")
+    try:
+        _layer_pins(dg, W, w, h, [0], 0, check=[0])
+    finally:
+        _release(h, w)
+
+
+@pytest.mark.gpu
+@pytest.mark.slow
+def test_full_b16_layer_pins_before_and_after_hand_off(dg):
+    """full_b16: 4096 canvas tokens per step (the grouped GEMMs at 32768 expert
+    rows), two requests checked per layer, at cache 4096 and after one block's
+    hand-off at 4352."""
+    W, w, h = _setup(dg, "full_b16")
+    S, n, P0, B = W["sampler"], W["model"]["canvas"], W["prompt_len"], W["batch"]
+    req = list(range(B))
+    try:
+        _layer_pins(dg, W, w, h, req, 0, check=[0, 9])
+        a = dg.block_args(req, S["max_steps"], S["schedule_steps"], temperature=S["temperature"],
+                          logit_scale_growth=S["logit_scale_growth"], stop_threshold=S["stop_threshold"],
+                          seed=S["seed"], block=0)
+        out = torch.zeros((B, n), dtype=torch.int32, device="cuda")
+        dg.dg_generate_block(h, a, out)
+        assert all(dg.dg_get_length(h, r) == P0 + n for r in req)
+        _layer_pins(dg, W, w, h, req, 1, check=[5, 15])
+    finally:
+        _release(h, w)
 
 
 @pytest.mark.gpu

@@ -22,6 +22,7 @@ from tests import test_oracle_pins as P
 _philox, _router, _attention = O.philox4x32_10, O.router, O.attention
 _position_stats, _anneal = O.position_stats, O.anneal_temperature
 _quantize = N.quantize
+_expert_order = O.expert_order
 
 
 def _rope_sign(x, pos, base):
@@ -71,6 +72,15 @@ def _router_high_ties(x, w, b, k):
     sel = np.take_along_axis(g, ids, axis=1)
     e = np.exp(sel - sel.max(axis=1, keepdims=True))
     return ids, e / e.sum(axis=1, keepdims=True), g, np.full(g.shape[0], np.inf)
+
+
+def _select_high_ties(g, k):
+    g = np.asarray(g, np.float64)
+    idx = np.arange(g.shape[1])
+    ids = np.stack([np.lexsort((-idx, -row))[:k] for row in g])                  # ties -> higher id
+    sel = np.take_along_axis(g, ids, axis=1)
+    e = np.exp(sel - sel.max(axis=1, keepdims=True))
+    return ids, e / e.sum(axis=1, keepdims=True), np.full(g.shape[0], np.inf)
 
 
 def _moe_unweighted(x, layer, top_k):
@@ -187,6 +197,18 @@ def _pack_swapped(codes):
     return (c[..., 1::2] & 0xF) | ((c[..., 0::2] & 0xF) << 4)
 
 
+def _expert_order_tokens_descending(ids, n_experts, tile):
+    cnt, off, perm, work, touched = _expert_order(ids, n_experts, tile)
+    for e in range(n_experts):
+        perm[off[e]:off[e + 1]] = perm[off[e]:off[e + 1]][::-1].copy()      # tokens in the wrong order
+    return cnt, off, perm, work, touched
+
+
+def _expert_order_tile_overrun(ids, n_experts, tile):
+    cnt, off, perm, work, touched = _expert_order(ids, n_experts, tile)
+    return cnt, off, perm, [(e, p0, min(tile, rows + 1)) for e, p0, rows in work], touched   # off by one
+
+
 KAT = P._kat_rows()
 
 CASES = {
@@ -207,6 +229,13 @@ CASES = {
     "router softmax over all": (O, "router", _router_softmax_all,
                                 [P.test_router_ties_go_to_lower_id_and_weights_sum_to_one]),
     "router ties": (O, "router", _router_high_ties, [P.test_router_ties_go_to_lower_id_and_weights_sum_to_one]),
+    "select ties": (O, "router_select", _select_high_ties,
+                    [P.test_router_select_brute_force_with_ties_and_minus_infinity,
+                     P.test_router_ties_go_to_lower_id_and_weights_sum_to_one]),
+    "expert order tokens descending": (O, "expert_order", _expert_order_tokens_descending,
+                                       [lambda: P.test_expert_order_brute_force(1, 40, 3, 9, 4)]),
+    "expert tile overrun": (O, "expert_order", _expert_order_tile_overrun,
+                            [lambda: P.test_expert_order_brute_force(1, 40, 3, 9, 4)]),
     "moe weights dropped": (O, "moe", _moe_unweighted, [P.test_moe_with_all_experts_is_the_dense_softmax_mixture]),
     "swiglu branch": (O, "swiglu_expert", _swiglu_swapped, [P.test_moe_single_expert_is_a_swiglu_mlp]),
     "entropy without log S": (O, "position_stats", _stats_no_log_s, [P.test_uniform_logits_give_log_v_entropy]),

@@ -222,6 +222,53 @@ def test_router_ties_go_to_lower_id_and_weights_sum_to_one():
     assert np.allclose(w[0], e / e.sum()) and abs(w.sum() - 1) < 1e-15
 
 
+@pytest.mark.parametrize("seed,T,k,E,tile", [(0, 7, 2, 5, 3), (1, 40, 3, 9, 4), (2, 1, 1, 1, 1), (3, 25, 4, 30, 2)])
+def test_expert_order_brute_force(seed, T, k, E, tile):
+    """The permutation against a sort by (expert, item index) written as a
+    plain Python key sort; counts, offsets and work tiles against direct counts."""
+    rng = np.random.default_rng(seed)
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
+    cnt, off, perm, work, touched = O.expert_order(ids, E, tile)
+    items = ids.reshape(-1).tolist()
+    want = sorted(range(len(items)), key=lambda i: (items[i], i))
+    assert perm.tolist() == want
+    assert cnt.tolist() == [items.count(e) for e in range(E)]
+    assert off[0] == 0 and all(off[e + 1] - off[e] == cnt[e] for e in range(E)) and off[E] == T * k
+    assert touched == len(set(items))
+    covered = []
+    for e, p0, rows in work:
+        assert 1 <= rows <= tile and off[e] <= p0 and p0 + rows <= off[e + 1]
+        assert all(items[perm[p]] == e for p in range(p0, p0 + rows))
+        covered += list(range(p0, p0 + rows))
+    assert covered == list(range(T * k))          # tiles in expert order, no gap, no overlap
+    # only each expert's last tile may be short
+    for (e, p0, rows), nxt in zip(work, work[1:] + [(None, None, None)]):
+        if nxt[0] == e:
+            assert rows == tile
+
+
+def test_router_select_brute_force_with_ties_and_minus_infinity():
+    """Selection on given logits against enumeration of every k-subset: the
+    chosen set has the largest sum of ranks under (value desc, id asc), listed
+    in that order; -inf values rank last, among themselves by id."""
+    import itertools
+    rng = np.random.default_rng(31)
+    for trial in range(40):
+        E, k = int(rng.integers(2, 7)), 0
+        k = int(rng.integers(1, E + 1))
+        g = rng.choice([-np.inf, -1.0, 0.0, 0.5, 2.0], size=(1, E))
+        if not np.isfinite(g).any():
+            g[0, 0] = 0.0
+        ids, w, margin = O.router_select(g, k)
+        key = lambda e: (-g[0, e], e)                      # python tuples: -(-inf) = inf sorts last
+        ranked = sorted(range(E), key=key)
+        best = min(itertools.combinations(range(E), k), key=lambda c: sorted(ranked.index(e) for e in c))
+        assert ids[0].tolist() == sorted(best, key=key)
+        assert len(set(ids[0].tolist())) == k
+        fin = np.isfinite(g[0, ids[0]])
+        assert np.all(w[0][~fin] == 0) and abs(w[0].sum() - 1) < 1e-12
+
+
 def test_moe_is_token_order_invariant():
     m = _tiny_model(seed=11, e=6, k=2)
     L = m.weights["layers"][0]

@@ -78,6 +78,30 @@ def test_noalloc_sampler_matches_dg_sample_two_calls_in_a_row(dg):
 
 
 @pytest.mark.gpu
+def test_noalloc_sampler_leaves_free_device_memory_unchanged(dg):
+    """The property the entry point exists for: once the device is set up (the
+    first call), calls take no device memory.  Free memory is read with
+    cudaMemGetInfo around repeated calls, with every output buffer made first."""
+    B, n, V = 2, W["canvas"], W["vocab"]
+    logits, _, _ = synth.peaked_logits(B, n, V, seed=W["seed"] + 92, peak_max=W["peak_max"])
+    logits = logits.cuda()
+    sp = dg.sampler_params(temperature=W["temperature"], keep_k=64, stop_threshold=W["stop_threshold"], seed=5)
+    outs = _outs(B, n)
+    canvas = torch.zeros((B, n), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    o = dg.step_out(**outs)
+    dg.dg_sample_noalloc(logits, [0, 1], 1, sp, canvas, o, stream=stream)     # set-up call
+    stream.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for step in range(2, 7):
+        dg.dg_sample_noalloc(logits, [0, 1], step, sp, canvas, o, stream=stream)
+        dg.dg_sample_noalloc(logits, [0, 1], step, sp, canvas, None, stream=stream)
+    stream.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"free device memory changed by {free0 - free1} bytes across calls"
+
+
+@pytest.mark.gpu
 def test_noalloc_sampler_argmax_ragged_vocab(dg):
     B, n, V = 3, 37, 5001
     g = torch.Generator().manual_seed(5)
