@@ -325,7 +325,36 @@ def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, pe
 
 # -------------------------------------------------------------------- ours
 
-def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clocks=True):
+def _measure_ar(m, h, W, dev, warmup=4, steps=32):
+    """AR mode on the same handle ([P1 五]: one canvas step against one AR step):
+    one token per step appended causally at the end of the prompt's cache, the
+    logits of the next token and its greedy choice.  Device-timed with CUDA
+    events around `steps` consecutive steps."""
+    import torch
+    model = W["model"]
+    P0 = W["prompt_len"]
+    m.dg_set_length(h, 0, P0)
+    tok = torch.zeros(1, dtype=torch.int32, device=dev)
+    logits = torch.empty((1, model["vocab"]), device=dev)
+    for _ in range(warmup):
+        m.dg_ar_step(h, [0], tok, logits, tok)
+    m.dg_synchronize(h)
+    m.dg_set_length(h, 0, P0)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = m.dg_launch_count(h)
+    e0.record(stream)
+    for _ in range(steps):
+        m.dg_ar_step(h, [0], tok, logits, tok)
+    e1.record(stream)
+    m.dg_synchronize(h)
+    ms = e0.elapsed_time(e1)
+    return {"steps": steps, "warmup": warmup, "us_per_token": round(ms * 1e3 / steps, 1),
+            "tokens_per_s": round(steps / (ms / 1e3), 1), "launches_per_token": (m.dg_launch_count(h) - l0) // steps,
+            "cache_from": P0}
+
+
+def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clocks=True, with_ar=False):
     """Build the workload's model, time `steps` bench steps after `warmup`, then
     an end-to-end pass and one profiled block.  Returns a dict of results."""
     import torch
@@ -427,13 +456,16 @@ def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clock
     breakdown = m.dg_profile_read(h)
     prof_blocks = list(block_log)
     m.dg_profile_enable(h, False)
+    ar = None
+    if B == 1 and with_ar:
+        ar = _measure_ar(m, h, W, dev)
     h.close()
     del w
     torch.cuda.empty_cache()
     return dict(W=W, model=model, B=B, n=n, P0=P0, blocks=blocks, elapsed_max=elapsed_max, units_all=units_all,
                 e2e_max=e2e_max, launches=launches, clocks=clocks, denoise_steps=denoise_steps,
                 timed_blocks=timed_blocks, breakdown=breakdown, prof_blocks=prof_blocks, touched=touched_mean,
-                prefill_s=prefill_s, steps=steps, warmup=warmup)
+                prefill_s=prefill_s, steps=steps, warmup=warmup, ar=ar)
 
 
 def run_ours(args):
@@ -446,7 +478,8 @@ def run_ours(args):
     dist = init_dist("nccl")
     dev = torch.device("cuda", local)
     peaks, peak_kind = load_peaks()
-    r = _measure_workload(m, args, args.workload, args.steps, args.warmup, dev, dist, world)
+    r = _measure_workload(m, args, args.workload, args.steps, args.warmup, dev, dist, world,
+                          with_ar=args.workload == "full_b1")
     model, B, n, P0, blocks = r["model"], r["B"], r["n"], r["P0"], r["blocks"]
     block_ms = r["elapsed_max"] / (args.steps * blocks)
     roof_step = block_roofline(model, B, n, r["timed_blocks"][:blocks], r["touched"], block_ms, peaks)
@@ -481,7 +514,16 @@ def run_ours(args):
         "prefill_s": round(r["prefill_s"], 2),
         "kernel_ms_per_block": {k: round(v[1] / len(r["prof_blocks"]), 3) for k, v in r["breakdown"].items()},
     }
-    if args.workload == "full_b1" and not args.no_b16:
+    if r["ar"]:
+        # AR mode on the same weights and cache: the pages' canvas-step / AR-step ratio
+        ar = r["ar"]
+        P = ar["cache_from"] + ar["steps"] // 2
+        b, f = pass_cost(model, 1, 1, P, model["top_k"], True, True, False)
+        bound_us = max(b / (peaks["hbm_gbs"] * 1e9), f / (peaks.get("bf16_tflops_sustained", 1400.0) * 1e12)) * 1e6
+        ar.update({"bound_us_per_token": round(bound_us, 1), "frac": round(bound_us / ar["us_per_token"], 4),
+                   "canvas_step_over_ar_step": round(line["us_per_denoise_step"] / ar["us_per_token"], 2),
+                   "experts_per_token": model["top_k"]})
+        line["ar_decode"] = ar
         # the batch-16 workload in the same run: 16 requests x 4 blocks x 12 steps per bench step
         s16, w16 = max(1, min(args.steps, 2)), max(1, min(args.warmup, 1))
         q = _measure_workload(m, args, "full_b16", s16, w16, dev, dist, world)

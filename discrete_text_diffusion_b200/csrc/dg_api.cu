@@ -631,6 +631,15 @@ void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
   a.max_ctx = c.max_ctx;
   a.causal = causal ? 1 : 0;
   a.bi = bi;
+  if (H->attn_tc && nq == 1) {
+    // one new token per request (AR decode): the single-token kernel, GQA heads sharing K/V
+    ProfScope ps(H, PC_ATTN, 2);
+    if (launch_attn_decode((const __nv_bfloat16*)H->q, (const __nv_bfloat16*)kc_layer(H, l),
+                           (const __nv_bfloat16*)vt_layer(H, l), (__nv_bfloat16*)H->attn, a, H->part_o, H->part_ml,
+                           H->part_rows_cap, H->num_sms, H->stream) != 0)
+      H->bad_launch = true;
+    return;
+  }
   if (H->attn_tc) {
     // Split the keys: one CTA per SM, so the time is about waves x (key tiles
     // per CTA + a fixed cost of ~2 tiles); each split adds partial-output
@@ -1408,6 +1417,33 @@ int dg_selftest_gemm_split(dg_handle* H, const void* x, const void* w, int T, in
   H->launches += 1;
   *nsplit = p.split;
   return check_launch(H, "selftest split gemm");
+}
+
+int dg_ar_step(dg_handle* H, int batch, const int* req, const int32_t* tokens, float* logits, int32_t* next_token) {
+  if (!H) return DG_EINVAL;
+  const dg_config& c = H->c;
+  if (c.n_layers == 0) return fail(H, DG_ESTATE, "sampler-only handle");
+  BatchInfo bi;
+  int rc = make_batch(H, batch, req, &bi);
+  if (rc) return rc;
+  if (!tokens || !logits) return fail(H, DG_EINVAL, "null tokens or logits");
+  if (!aligned16(logits)) return fail(H, DG_EINVAL, "logits must be 16-byte aligned");
+  for (int b = 0; b < bi.B; ++b)
+    if (bi.len[b] + 1 > c.max_ctx) return fail(H, DG_ECAPACITY, "cache full: P + 1 exceeds max_ctx");
+  if ((rc = upload_req(H, bi))) return rc;
+  // causal encode of one token per request at position P, then the tied LM head on it
+  run_layers(H, bi, 1, true, tokens, nullptr, true, logits, nullptr);
+  if (next_token) {
+    SamplerArgs a{};
+    a.temperature = 0.f;   // argmax, ties to the lower index
+    a.logit_scale = 1.f;
+    a.stop_threshold = -1.f;
+    ProfScope ps(H, PC_SAMPLER, 2);
+    launch_sampler_rows(logits, bi.B, 1, c.vocab, H->req_dev, a, H->sws, next_token, H->pmax, H->ent, H->stream);
+  }
+  if ((rc = check_launch(H, "ar step"))) return rc;
+  for (int b = 0; b < bi.B; ++b) H->len[bi.slot[b]] += 1;
+  return DG_OK;
 }
 
 int dg_selftest_wait_timeout(dg_handle* H, int limit_us) {

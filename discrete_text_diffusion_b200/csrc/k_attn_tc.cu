@@ -410,6 +410,14 @@ size_t attn_tc_partial_floats(int n_split, int B, int hq, int nq_pad, int hd) {
   return (size_t)n_split * B * hq * nq_pad * hd;
 }
 
+void launch_attn_combine(const float* part_o, const float* part_ml, __nv_bfloat16* out, int n_split, int B, int hq,
+                         int nq, cudaStream_t s) {
+  const int rows = B * hq * nq;
+  if (rows <= 0) return;
+  launch_k(attn_combine_kernel, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, part_o, part_ml, out, n_split, B, hq,
+           nq);
+}
+
 void launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, __nv_bfloat16* out,
                     const AttnTcArgs& t, cudaStream_t s) {
   const AttnArgs& a = t.a;
@@ -425,11 +433,7 @@ void launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
   P.scale_log2 = 1.4426950408889634f / sqrtf((float)a.hd);
   dim3 grid(P.n_qtiles * t.n_split, a.hq, a.B);
   launch_k(attn_tc_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmem, s, tq, tk, tv, out, P);
-  if (t.n_split > 1) {
-    const int rows = a.B * a.hq * a.nq;
-    launch_k(attn_combine_kernel, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, t.part_o, t.part_ml, out, t.n_split, a.B, a.hq,
-                                                                 a.nq);
-  }
+  if (t.n_split > 1) launch_attn_combine(t.part_o, t.part_ml, out, t.n_split, a.B, a.hq, a.nq, s);
 }
 
 }  // namespace dg

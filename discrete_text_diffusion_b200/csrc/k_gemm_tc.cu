@@ -100,6 +100,12 @@ int gemm_tc_smem_bytes(const TcGemm& p, int* stages) {
   return L.smem_bytes;
 }
 
+// silu(g) * u for an output rounded to bf16 right after: the hardware exp2
+// and the approximate divide (their few-ulp error is far below bf16's 2^-9).
+__device__ __forceinline__ float swiglu_bf16(float gt, float up) {
+  return __fdividef(gt, 1.f + __expf(-gt)) * up;
+}
+
 struct TcKParams {
   TcGemm g;
   int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, n_ttiles, ksub;
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
               for (int j = 0; j < 32; ++j) {
                 if (c0 + j < rows) {
                   const float gt = __uint_as_float(v[j]), up = __uint_as_float(u[j]);
-                  out_b[(size_t)(row0 + c0 + j) * g.ld_out + m] = __float2bfloat16_rn(gt / (1.f + expf(-gt)) * up);
+                  out_b[(size_t)(row0 + c0 + j) * g.ld_out + m] = __float2bfloat16_rn(swiglu_bf16(gt, up));
                 }
               }
             }
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float gt = __uint_as_float(v[j]), up = __uint_as_float(u[j]);
-            stg_b[j * kBM + r] = __float2bfloat16_rn(gt / (1.f + expf(-gt)) * up);
+            stg_b[j * kBM + r] = __float2bfloat16_rn(swiglu_bf16(gt, up));
           }
         } else if (tstore) {
           tmem_ld_wait();

@@ -173,6 +173,17 @@ struct AttnTcArgs {
 void launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     __nv_bfloat16* out, const AttnTcArgs& a, cudaStream_t s);
 size_t attn_tc_partial_floats(int n_split, int B, int hq, int nq_pad, int hd);
+// Merge KV-split partials (unnormalised O [split][B*Hq*nq][256], (max log2, sum)) into
+// out [B*nq, Hq*256] bf16.
+void launch_attn_combine(const float* part_o, const float* part_ml, __nv_bfloat16* out, int n_split, int B, int hq,
+                         int nq, cudaStream_t s);
+// Single-token attention (AR decode, k_attn_decode.cu): bf16, hd 256, nq 1, Hq/Hkv in {1,2,4,8};
+// q [B][Hq][1][hd]; keys are the cache [0, len] of each request.  Split partials in
+// part_o / part_ml (capacity part_rows_cap split rows), then the combine.  Returns -1
+// (nothing launched) for another shape.
+int launch_attn_decode(const __nv_bfloat16* q, const __nv_bfloat16* kc, const __nv_bfloat16* vt,
+                       __nv_bfloat16* out, const AttnArgs& a, float* part_o, float* part_ml, size_t part_rows_cap,
+                       int num_sms, cudaStream_t s);
 
 // ---- self test
 void launch_philox_selftest(const uint32_t* ctr, const uint32_t* key, uint32_t* out, uint32_t* out_curand,

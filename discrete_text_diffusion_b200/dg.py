@@ -24,7 +24,7 @@ EXPORTS = (
     "dg_get_length", "dg_denoise_step", "dg_sample", "dg_generate_block", "dg_generate_block_host",
     "dg_synchronize", "dg_launch_count", "dg_profile_enable", "dg_profile_read", "dg_profile_reset",
     "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc", "dg_selftest_gemm_split", "dg_get_kv",
-    "dg_selftest_router", "dg_selftest_wait_timeout",
+    "dg_selftest_router", "dg_selftest_wait_timeout", "dg_ar_step",
 )
 
 
@@ -111,6 +111,7 @@ def lib():
         L.dg_get_kv.argtypes = [P, C.c_int, C.c_int, P, P, C.c_int]
         L.dg_selftest_router.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(DgRouterOut)]
         L.dg_selftest_wait_timeout.argtypes = [P, C.c_int]
+        L.dg_ar_step.argtypes = [P, C.c_int, C.POINTER(C.c_int), P, P, P]
         L.dg_set_length.argtypes = [P, C.c_int, C.c_int]
         L.dg_get_length.argtypes = [P, C.c_int, C.POINTER(C.c_int)]
         L.dg_denoise_step.argtypes = [P, C.POINTER(DgStepArgs), C.POINTER(DgStepOut)]
@@ -312,6 +313,12 @@ def dg_generate_block_host(h: Handle, a: DgBlockArgs, out_tokens_host: torch.Ten
     steps = C.c_int()
     h.check(lib().dg_generate_block_host(h.ptr, C.byref(a), _ptr(out_tokens_host), C.byref(steps)))
     return steps.value
+
+
+def dg_ar_step(h: Handle, req, tokens, logits, next_token=None):
+    """AR mode: append tokens [B] (int32, device) causally; logits [B, V] fp32 of the next token;
+    next_token [B] int32 (argmax) or None."""
+    return h.check(lib().dg_ar_step(h.ptr, len(req), _ints(req), _ptr(tokens), _ptr(logits), _ptr(next_token)))
 
 
 def dg_synchronize(h: Handle):

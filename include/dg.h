@@ -340,6 +340,23 @@ int dg_generate_block(dg_handle* h, const dg_block_args* a, int32_t* out_tokens,
 int dg_generate_block_host(dg_handle* h, const dg_block_args* a, int32_t* out_tokens_host,
                            int* steps_used);
 
+/*
+ * AR mode ([P1 七]: the same weights load as an autoregressive model; [P1 五]
+ * compares the canvas step with one AR step).  For each request: encode
+ * tokens[b] causally at position P (its K/V appended, P += 1), then write the
+ * logits of the token that follows it: final norm and tied LM head.  No canvas
+ * and no self-conditioning.
+ *   tokens: [B] device int32 in [0, V) (out-of-range tokens are replaced by 0
+ *           and reported as DG_EINVAL by the next synchronising call).
+ *   logits: [B, V] device fp32, 16-byte aligned.
+ *   next_token: [B] device int32, the argmax of the logits (ties -> lower
+ *           index), or NULL.
+ * bf16 handles with head_dim 256 run the single-token attention kernel (one
+ * pass over the cache per KV head, all its query heads together).
+ * DG_ECAPACITY if any P + 1 > max_ctx.
+ */
+int dg_ar_step(dg_handle* h, int batch, const int* req, const int32_t* tokens, float* logits, int32_t* next_token);
+
 /* Synchronise the handle's stream and report device-side timeouts. */
 int dg_synchronize(dg_handle* h);
 
