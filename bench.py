@@ -314,12 +314,25 @@ def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, pe
         add("moe_up", "gemm_tc_kernel (grouped gate/up + SwiGLU)", "tensor", 2.0 * rows * 2 * F * d)
         add("moe_down", "gemm_tc_kernel (grouped down, scatter)", "tensor", 2.0 * rows * F * d)
     if "dense_gemm" in breakdown:
-        # QKV and O every pass, W_sc every step after the first: weights once each
+        # QKV and O every pass, W_sc every step after the first: weights once each (bytes), or
+        # every token through them (flops), whichever bound is slower
         nl, _ = breakdown["dense_gemm"]
-        byt = (passes * L * ((hq + 2 * hkv) * hd * d + d * hq * hd) + (steps - len(blocks)) * d * d) * 2
-        add("dense_gemm", "gemm_tc_kernel (split-K QKV / O / self-cond)", "hbm", byt / nl)
-    add("lm_head", "gemm_tc_kernel (tied LM head)", "hbm", V * d * 2 + T * V * 4)
-    add("sampler_rows", "sampler_pass1 + sampler_pass2", "hbm", 4.0 * V * T)
+        wts = passes * L * ((hq + 2 * hkv) * hd * d + d * hq * hd) + (steps - len(blocks)) * d * d
+        byt, fl = wts * 2.0, 2.0 * wts * T
+        if fl / (tfs * 1e12) > byt / (hbm * 1e9):
+            add("dense_gemm", "gemm_tc_kernel (QKV / O / self-cond)", "tensor", fl / nl)
+        else:
+            add("dense_gemm", "gemm_tc_kernel (split-K QKV / O / self-cond)", "hbm", byt / nl)
+    # the block loop runs the fused head: the LM head writes 16-byte statistics per token and
+    # 32-entry vocabulary group instead of logits; the sampler reads them and recomputes one group
+    groups = (V + 31) // 32
+    lm_fl = 2.0 * T * d * V
+    lm_b = V * d * 2 + T * groups * 16
+    if lm_fl / (tfs * 1e12) > lm_b / (hbm * 1e9):
+        add("lm_head", "gemm_tc_kernel (tied LM head + sampler statistics)", "tensor", lm_fl)
+    else:
+        add("lm_head", "gemm_tc_kernel (tied LM head + sampler statistics)", "hbm", lm_b)
+    add("sampler_rows", "sampler_pass2_fused (merge + one-group recompute)", "hbm", T * groups * 16.0 + T * 32 * d * 2.0)
     return out
 
 

@@ -177,6 +177,8 @@ struct dg_handle {
   void* hb = nullptr;
   void* y = nullptr;            // expert outputs [T*k, d] in (token, slot) order, activation type
   float* logits = nullptr;
+  VocabStat* vstats = nullptr;  // fused LM head -> sampler: per-token statistics of 32-entry vocabulary groups
+  int n_groups = 0;
   float2* rope = nullptr;
   // tensor-core attention (bf16, head dim 256)
   bool attn_tc = false;
@@ -679,9 +681,36 @@ void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
                                     (const __nv_bfloat16*)vt_layer(H, l), (__nv_bfloat16*)H->attn, a, H->stream);
 }
 
+// The tied LM head with the sampler's first pass in its epilogue: per token and
+// 32-entry vocabulary group, (max, first arg-max, sum exp, sum exp * z) of
+// z = logit * s / T into H->vstats; the logits themselves are never written.
+void lm_head_stats(dg_handle* H, int T, const SamplerArgs& sa) {
+  const dg_config& c = H->c;
+  ProfScope ps(H, PC_LMHEAD);
+  TcGemm g{};
+  g.mode = 0;
+  g.M = c.vocab;
+  g.K = c.d_model;
+  g.T = T;
+  g.ntile = pick_ntile((c.vocab + 127) / 128, T, H->num_sms);
+  g.seg1 = g.seg2 = INT_MAX;
+  g.epi = EPI_VOCAB_STATS;
+  g.out = H->vstats;
+  g.ld_out = 0;
+  g.err = H->d_err;
+  g.ksub = ksub_for(0, g.ntile);
+  g.ctas_per_sm = ctas_for(g.ntile);
+  g.argmax_mode = sa.temperature == 0.f ? 1 : 0;
+  g.zscale = g.argmax_mode ? sa.logit_scale : sa.logit_scale / sa.temperature;
+  g.n_groups = H->n_groups;
+  const CUtensorMap& a = pick(H->m_embed, g.ksub);
+  run_tc(H, a, a, a, bmap(H, H->xn, c.d_model, H->T_max, g.ntile, g.ksub), g);
+}
+
 template <typename T>
 void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const int32_t* tokens,
-                  const int32_t* prev, bool head, float* logits, float* hidden_out, const dg_layer_dump* dump) {
+                  const int32_t* prev, bool head, float* logits, float* hidden_out, const dg_layer_dump* dump,
+                  const SamplerArgs* fused) {
   const dg_config& c = H->c;
   const int Tn = bi.B * nq;
   const size_t hbytes = (size_t)Tn * c.d_model * sizeof(float);
@@ -766,14 +795,16 @@ void run_layers_t(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const 
       launch_rmsnorm<T>(H->h, H->final_norm, xn, Tn, c.d_model, eps, H->stream);
     }
   }
-  if (head) dense_gemm(H, PC_LMHEAD, H->xn, H->embed, &H->m_embed, Tn, c.vocab, c.d_model, EPI_STORE_F32,
-                       logits, c.vocab);
+  if (head && fused) lm_head_stats(H, Tn, *fused);
+  else if (head) dense_gemm(H, PC_LMHEAD, H->xn, H->embed, &H->m_embed, Tn, c.vocab, c.d_model, EPI_STORE_F32,
+                            logits, c.vocab);
 }
 
 void run_layers(dg_handle* H, const BatchInfo& bi, int nq, bool causal, const int32_t* tokens, const int32_t* prev,
-                bool head, float* logits, float* hidden_out, const dg_layer_dump* dump = nullptr) {
-  if (H->bf16) run_layers_t<__nv_bfloat16>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out, dump);
-  else run_layers_t<float>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out, dump);
+                bool head, float* logits, float* hidden_out, const dg_layer_dump* dump = nullptr,
+                const SamplerArgs* fused = nullptr) {
+  if (H->bf16) run_layers_t<__nv_bfloat16>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out, dump, fused);
+  else run_layers_t<float>(H, bi, nq, causal, tokens, prev, head, logits, hidden_out, dump, nullptr);
 }
 
 int make_batch(dg_handle* H, int batch, const int* req, BatchInfo* bi) {
@@ -839,11 +870,16 @@ int check_sampler_params(dg_handle* H, const dg_sampler_params* sp) {
 }
 
 // sampler over logits rows of the batch, then keep / re-noise / stop
+// logits == nullptr: the fused form, from the LM head's group statistics in H->vstats
 void run_sampler(dg_handle* H, const float* logits, const BatchInfo& bi, const SamplerArgs& a, int32_t* canvas,
                  int32_t* xh, float* pmax, float* ent, int32_t* keep, float* meanh, int32_t* stop, int32_t* done,
                  int32_t* out_tokens, int final_step, int32_t* argmax) {
   const int n = H->c.canvas;
-  {
+  if (!logits) {
+    ProfScope ps(H, PC_SAMPLER, 1);
+    launch_sampler_fused_rows(H->vstats, H->n_groups, (const __nv_bfloat16*)H->xn, (const __nv_bfloat16*)H->embed,
+                              H->c.d_model, bi.B * n, n, H->c.vocab, H->req_dev, a, xh, pmax, ent, H->stream, argmax);
+  } else {
     ProfScope ps(H, PC_SAMPLER, 2);
     launch_sampler_rows(logits, bi.B * n, n, H->c.vocab, H->req_dev, a, H->sws, xh, pmax, ent, H->stream, argmax);
   }
@@ -983,6 +1019,10 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
     H->hb = dalloc<char>((size_t)T * c.top_k * c.d_ff * H->esz, &ok);
     H->y = dalloc<char>((size_t)T * c.top_k * c.d_model * H->esz, &ok);
     H->logits = dalloc<float>((size_t)nrow * c.vocab, &ok);
+    if (c.dtype == DG_BF16) {
+      H->n_groups = (c.vocab + 31) / 32;
+      H->vstats = dalloc<VocabStat>((size_t)nrow * H->n_groups, &ok);
+    }
     H->rope = dalloc<float2>((size_t)c.max_ctx * (c.head_dim / 2), &ok);
     H->tok_ws = dalloc<int32_t>((size_t)T, &ok);
     if (c.dtype == DG_BF16) {
@@ -1100,7 +1140,7 @@ void dg_destroy(dg_handle* H) {
                 H->off, H->perm, H->work, H->n_work, H->touched, H->xp, H->hb, H->y, H->logits, H->rope, H->sws,
                 H->xh[0], H->xh[1], H->pmax, H->ent, H->keep, H->meanh, H->stop, H->done, H->canvas, H->out_tok,
                 H->req_dev, H->tok_ws, H->d_err, H->part_o, H->part_ml, H->kpart, H->amax[0], H->amax[1],
-                H->mh2[0], H->mh2[1]};
+                H->mh2[0], H->mh2[1], H->vstats};
   for (void* p : ps)
     if (p) cudaFree(p);
   if (H->h_done) cudaFreeHost(H->h_done);
@@ -1215,9 +1255,12 @@ int dg_denoise_step(dg_handle* H, const dg_step_args* a, const dg_step_out* o) {
   if (a->sp.stop_mode == DG_STOP_TWO_ROUNDS && !(o && o->argmax))
     return fail(H, DG_EINVAL, "the two-round stop needs o->argmax (the next round's prev_argmax)");
   if ((rc = upload_req(H, bi))) return rc;
-  float* logits = a->logits_out ? a->logits_out : H->logits;
-  run_layers(H, bi, c.canvas, false, a->canvas, a->prev_pred, true, logits, a->hidden_out, a->dump);
   const SamplerArgs sa = sampler_args(a->sp, a->step);
+  // without a logits buffer from the caller, the LM head feeds the sampler directly (no logits written)
+  const bool fused = H->vstats && !a->logits_out;
+  float* logits = fused ? nullptr : (a->logits_out ? a->logits_out : H->logits);
+  run_layers(H, bi, c.canvas, false, a->canvas, a->prev_pred, true, logits, a->hidden_out, a->dump,
+             fused ? &sa : nullptr);
   run_sampler(H, logits, bi, sa, a->canvas, (o && o->x_hat) ? o->x_hat : H->xh[0],
               (o && o->pmax) ? o->pmax : H->pmax, (o && o->entropy) ? o->entropy : H->ent, o ? o->keep : nullptr,
               o ? o->mean_entropy : nullptr, o ? o->stop : nullptr, nullptr, nullptr, 0, argmax_target(o));
@@ -1277,9 +1320,12 @@ static int generate_block_impl(dg_handle* H, const dg_block_args* a, int32_t* ou
     sp.prev_argmax = (two_rounds && t > 1) ? H->amax[(t - 1) & 1] : nullptr;
     sp.prev_mean_entropy = (two_rounds && t > 1) ? H->mh2[(t - 1) & 1] : nullptr;
     if ((rc = check_sampler_params(H, &sp))) return rc;
-    run_layers(H, bi, n, false, H->canvas, prev, true, H->logits, nullptr);
+    const SamplerArgs sa = sampler_args(sp, t);
+    const bool fused = H->vstats != nullptr;
+    run_layers(H, bi, n, false, H->canvas, prev, true, fused ? nullptr : H->logits, nullptr, nullptr,
+               fused ? &sa : nullptr);
     int32_t* xh = H->xh[t & 1];
-    run_sampler(H, H->logits, bi, sampler_args(sp, t), H->canvas, xh, H->pmax, H->ent, H->keep,
+    run_sampler(H, fused ? nullptr : H->logits, bi, sa, H->canvas, xh, H->pmax, H->ent, H->keep,
                 two_rounds ? H->mh2[t & 1] : H->meanh, H->stop, H->done, out_dev, t == a->max_steps ? 1 : 0,
                 two_rounds ? H->amax[t & 1] : nullptr);
     if ((rc = check_launch(H, "block step"))) return rc;

@@ -151,6 +151,9 @@ __device__ __forceinline__ void tc_item(const TcKParams& P, int item, int nst, i
   }
 }
 
+// kStats: the LM head's sampler-statistics epilogue (EPI_VOCAB_STATS), compiled
+// as its own instantiation so that its registers do not weigh on the other modes.
+template <bool kStats>
 __global__ void __launch_bounds__(kTcThreads, 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap ta1,
                    const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb,
@@ -318,6 +321,49 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       for (int c0 = 0; c0 < rows; c0 += kEpiRows) {
         uint32_t v[32];
         tmem_ld32(tbase + (uint32_t)c0, v);
+        if constexpr (kStats) {
+          // sampler statistics instead of logits.  The chunk (32 tokens x 128
+          // vocabulary rows) goes through the staging tile, XOR-swizzled so
+          // that both the row-wise writes and the column-wise reads are free of
+          // bank conflicts; then thread (warp q, lane t) reduces token t over
+          // its 32-row group m0 + 32q .. +31 on its own, in vocabulary order.
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[j * kBM + (r ^ j)] = __uint_as_float(v[j]);
+          named_barrier_sync(1, 128);
+          const int t = lane, grp = (m0 >> 5) + q;
+          float z[32];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int row = 32 * q + i;
+            z[i] = m0 + row < g.M ? stg[t * kBM + (row ^ t)] * g.zscale : -INFINITY;
+            mx = fmaxf(mx, z[i]);
+          }
+          named_barrier_sync(1, 128);   // the tile is rewritten by the next chunk
+          VocabStat rec;
+          rec.m = mx;
+          rec.idx = m0 + 32 * q;
+          rec.s = 0.f;
+          rec.a = 0.f;
+#pragma unroll
+          for (int i = 31; i >= 0; --i)
+            if (z[i] == mx) rec.idx = m0 + 32 * q + i;   // the first row holding the max
+          if (g.argmax_mode) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rec.s += z[i] == mx ? 1.f : 0.f;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float dz = z[i] - mx;
+              const float e = expf(dz);                 // padding rows: exp(-inf) = 0
+              rec.s += e;
+              rec.a += e > 0.f ? e * dz : 0.f;
+            }
+          }
+          if (c0 + t < rows && grp < g.n_groups)
+            reinterpret_cast<VocabStat*>(g.out)[(size_t)(row0 + c0 + t) * g.n_groups + grp] = rec;
+          continue;
+        }
         if (!staged) {
           // direct form: each thread writes its row m, one token column at a time
           const int m = m0 + r;
@@ -448,7 +494,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 static void set_smem_attr() {
   static bool done = false;
   if (!done) {
-    cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     done = true;
   }
 }
@@ -487,7 +534,7 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   const CUtensorMap& s0 = P.box_levels > 0 ? bsub[0] : b;
   const CUtensorMap& s1 = P.box_levels > 1 ? bsub[1] : b;
   const CUtensorMap& s2 = P.box_levels > 2 ? bsub[2] : b;
-  launch_k(gemm_tc_kernel, dim3(grid), dim3(kTcThreads), L.smem_bytes, s, a0, a1, a2, b, s0, s1, s2,
+  launch_k(g.epi == EPI_VOCAB_STATS ? gemm_tc_kernel<true> : gemm_tc_kernel<false>, dim3(grid), dim3(kTcThreads), L.smem_bytes, s, a0, a1, a2, b, s0, s1, s2,
            g.tma_out ? *tout : b, P);
   return 0;
 }

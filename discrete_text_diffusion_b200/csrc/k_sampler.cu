@@ -290,6 +290,180 @@ void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const 
                                           part, x_hat, pmax, ent, argmax);
 }
 
+// Pass 2 on the LM head's per-group statistics (the fused form): one CTA per
+// row.  Thread t merges groups [t*per, (t+1)*per) in order (fp64), the block
+// merges the threads in order: the max M and its first index, S = sum of the
+// group masses s_g exp(m_g - M), and the entropy term.  The inclusive scan of
+// the threads' masses finds the thread, then the group, whose prefix first
+// exceeds u*S; only that group's 32 logits are recomputed (the final-norm row
+// times 32 embedding rows, fp32 accumulation) and walked in vocabulary order.
+// The recomputed logits can differ from the GEMM's in the last bits, so a
+// crossing that falls short inside the group takes the group's last positive
+// entry, as a crossing that falls short anywhere does.
+constexpr int kFusedThreads = 256;
+constexpr int kGroup = 32;
+
+__global__ void __launch_bounds__(kFusedThreads)
+    sampler_pass2_fused(const VocabStat* __restrict__ st, int n_groups, const __nv_bfloat16* __restrict__ xn,
+                        const __nv_bfloat16* __restrict__ emb, int d, int n, int vocab, float scale, int argmax_mode,
+                        const int* __restrict__ req_ids, uint64_t seed, uint32_t step, uint32_t block,
+                        int32_t* __restrict__ x_hat, float* __restrict__ pmax, float* __restrict__ ent,
+                        int32_t* __restrict__ argmax) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ double scan[kFusedThreads];
+  __shared__ double red_a[kFusedThreads / 32];
+  __shared__ float red_m[kFusedThreads / 32];
+  __shared__ int red_i[kFusedThreads / 32];
+  __shared__ int red_l[kFusedThreads / 32];
+  __shared__ float sh_z[kGroup];
+  __shared__ int sh_g;
+  __shared__ double sh_P0;
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int b = row / n, i = row - b * n;
+  const VocabStat* pr = st + (size_t)row * n_groups;
+  const int per = (n_groups + kFusedThreads - 1) / kFusedThreads;
+  const int g0 = min(n_groups, tid * per), g1 = min(n_groups, g0 + per);
+  // the max and its first index (groups in vocabulary order: strict > keeps the earlier one)
+  float Mt = -INFINITY;
+  int It = 0x7fffffff;
+  for (int g = g0; g < g1; ++g) {
+    const float m = pr[g].m;
+    if (m > Mt) { Mt = m; It = pr[g].idx; }
+  }
+  float M = warp_max(Mt);
+  if (lane == 0) red_m[w] = M;
+  __syncthreads();
+  M = red_m[0];
+  for (int x = 1; x < kFusedThreads / 32; ++x) M = fmaxf(M, red_m[x]);
+  int I = Mt == M ? It : 0x7fffffff;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) I = min(I, __shfl_xor_sync(0xffffffffu, I, o));
+  if (lane == 0) red_i[w] = I;
+  // this thread's mass (relative to M), entropy term and last group with mass, in group order
+  double wt = 0.0, at = 0.0;
+  int lastg = -1;
+  for (int g = g0; g < g1; ++g) {
+    const VocabStat p = pr[g];
+    if (argmax_mode) {
+      if (p.m == M) wt += (double)p.s;
+    } else {
+      const double f = exp((double)p.m - (double)M);
+      const double c = (double)p.s * f;
+      wt += c;
+      at += ((double)p.a + ((double)p.m - (double)M) * (double)p.s) * f;
+      if (c > 0.0) lastg = g;
+    }
+  }
+  int L = lastg;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L = max(L, __shfl_xor_sync(0xffffffffu, L, o));
+  double a_w = warp_sum_d(at);
+  if (lane == 0) { red_a[w] = a_w; red_l[w] = L; }
+  scan[tid] = wt;
+  __syncthreads();
+  I = red_i[0];
+  for (int x = 1; x < kFusedThreads / 32; ++x) I = min(I, red_i[x]);
+  for (int o = 1; o < kFusedThreads; o <<= 1) {
+    const double add = tid >= o ? scan[tid - o] : 0.0;
+    __syncthreads();
+    scan[tid] += add;
+    __syncthreads();
+  }
+  const double S = scan[kFusedThreads - 1];
+  if (argmax_mode) {
+    if (tid == 0) {
+      x_hat[row] = I;
+      if (argmax) argmax[row] = I;
+      pmax[row] = (float)(1.0 / S);
+      ent[row] = (float)log(S);
+    }
+    return;
+  }
+  double A = 0.0;
+  int lastpos = -1;
+  for (int x = 0; x < kFusedThreads / 32; ++x) { A += red_a[x]; lastpos = max(lastpos, red_l[x]); }
+  const Philox4 wd = sampler_words(seed, (uint32_t)i, step, block, (uint32_t)req_ids[b]);
+  const double target = (double)unit_uniform(wd.w[0]) * S;
+  if (tid == 0) {
+    sh_g = 0x7fffffff;
+    if (argmax) argmax[row] = I;
+    pmax[row] = (float)(1.0 / S);
+    ent[row] = (float)(log(S) - A / S);
+  }
+  __syncthreads();
+  const double before = scan[tid] - wt;
+  if (before <= target && before + wt > target) {
+    double cum = before;
+    int gs = -1, glast = -1;
+    double p0 = 0.0, p0_last = 0.0;
+    for (int g = g0; g < g1; ++g) {
+      const VocabStat p = pr[g];
+      const double c = (double)p.s * exp((double)p.m - (double)M);
+      if (c > 0.0) { glast = g; p0_last = cum; }
+      if (cum + c > target) { gs = g; p0 = cum; break; }
+      cum += c;
+    }
+    if (gs < 0) { gs = glast; p0 = p0_last; }   // the thread's sum crossed, the group walk fell short
+    sh_g = gs;
+    sh_P0 = p0;
+  }
+  __syncthreads();
+  if (sh_g == 0x7fffffff) {
+    // no crossing (rounding): the last group with mass, walked to its last positive entry
+    if (tid == 0) { sh_g = lastpos; sh_P0 = INFINITY; }
+    __syncthreads();
+  }
+  const int gsel = sh_g;
+  // recompute the group's logits: warp w takes rows 4w .. 4w+3 of the group
+  const __nv_bfloat16* x = xn + (size_t)row * d;
+  for (int u = 0; u < kGroup / (kFusedThreads / 32); ++u) {
+    const int v = gsel * kGroup + w * (kGroup / (kFusedThreads / 32)) + u;
+    float acc = 0.f;
+    if (v < vocab) {
+      const __nv_bfloat16* er = emb + (size_t)v * d;
+      for (int k = lane * 8; k < d; k += 32 * 8) {
+        const uint4 xa = *reinterpret_cast<const uint4*>(x + k);
+        const uint4 ea = *reinterpret_cast<const uint4*>(er + k);
+        const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xa);
+        const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&ea);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 xf = __bfloat1622float2(x2[q]), ef = __bfloat1622float2(e2[q]);
+          acc = fmaf(xf.x, ef.x, acc);
+          acc = fmaf(xf.y, ef.y, acc);
+        }
+      }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) sh_z[w * (kGroup / (kFusedThreads / 32)) + u] = v < vocab ? acc * scale : -INFINITY;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double cum = sh_P0;
+    int pick = -1, last = -1;
+    for (int j = 0; j < kGroup; ++j) {
+      const float e = expf(sh_z[j] - M);
+      if (e > 0.f) last = j;
+      cum += (double)e;
+      if (pick < 0 && cum > target) pick = j;
+    }
+    if (pick < 0) pick = last >= 0 ? last : 0;
+    x_hat[row] = gsel * kGroup + pick;
+  }
+}
+
+void launch_sampler_fused_rows(const VocabStat* stats, int n_groups, const __nv_bfloat16* xn,
+                               const __nv_bfloat16* embed, int d, int rows, int n, int vocab, const int* req_ids,
+                               const SamplerArgs& a, int32_t* x_hat, float* pmax, float* ent, cudaStream_t s,
+                               int32_t* argmax) {
+  if (rows <= 0) return;
+  const int argmax_mode = a.temperature == 0.f;
+  const float scale = argmax_mode ? a.logit_scale : a.logit_scale / a.temperature;
+  launch_k(sampler_pass2_fused, dim3(rows), dim3(kFusedThreads), 0, s, stats, n_groups, xn, embed, d, n, vocab, scale,
+           argmax_mode, req_ids, a.seed, a.step, a.block, x_hat, pmax, ent, argmax);
+}
+
 // Pass 3: per canvas.  Top-k keep: rank_i = #{j : pmax_j > pmax_i or
 // (pmax_j == pmax_i and j < i)}, kept iff rank_i < keep_k.  Entropy budget:
 // r_i = #{j : H_j < H_i or (H_j == H_i and j < i)} orders the positions by

@@ -75,6 +75,17 @@ void launch_router_permute(const int32_t* ids, int n_items, int e, int tile, int
                            int32_t* perm, int32_t* work, int32_t* n_work, int32_t* touched,
                            cudaStream_t s);
 
+// Sampler statistics of one token over one group of 32 consecutive vocabulary
+// entries, z = logit * scale: the group max, the first index holding it, and
+// sum exp(z - m), sum exp(z - m)(z - m) (fp32 over the 32 terms).  In arg-max
+// mode (temperature 0) s counts the entries equal to m and a is 0.
+struct VocabStat {
+  float m;
+  int idx;
+  float s;
+  float a;
+};
+
 // ---- sampler (k_sampler.cu)
 struct SamplerArgs {
   float temperature, logit_scale, stop_threshold;
@@ -94,6 +105,15 @@ size_t sampler_workspace_bytes(int rows, int vocab);
 void launch_sampler_rows(const float* logits, int rows, int n, int vocab, const int* req_ids,
                          const SamplerArgs& a, void* ws, int32_t* x_hat, float* pmax, float* ent,
                          cudaStream_t s, int32_t* argmax = nullptr);
+// The sampler rows from the LM head's per-group statistics instead of logits:
+// merges each row's n_groups VocabStat records in vocabulary order (fp64), draws
+// the Philox inverse-CDF sample, and recomputes only the 32 logits of the group
+// holding u*S from the final-norm rows xn [rows, d] and the tied embedding
+// [V, d] (bf16).  Same outputs as launch_sampler_rows.
+void launch_sampler_fused_rows(const VocabStat* stats, int n_groups, const __nv_bfloat16* xn,
+                               const __nv_bfloat16* embed, int d, int rows, int n, int vocab, const int* req_ids,
+                               const SamplerArgs& a, int32_t* x_hat, float* pmax, float* ent, cudaStream_t s,
+                               int32_t* argmax = nullptr);
 // Per canvas: keep set, re-noise, mean entropy, stop; optional block-loop outputs.
 // argmax: this round's argmax rows (required by stop_mode 1).
 void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float* ent, int B, int n,
@@ -102,7 +122,9 @@ void launch_sampler_finish(const int32_t* x_hat, const float* pmax, const float*
                            int final_step, cudaStream_t s, const int32_t* argmax = nullptr);
 
 // ---- GEMMs
-enum Epi { EPI_STORE_F32 = 0, EPI_ADD_F32 = 1, EPI_STORE_ACT = 2, EPI_SWIGLU_ACT = 3, EPI_SCATTER_ACT = 4 };
+enum Epi { EPI_STORE_F32 = 0, EPI_ADD_F32 = 1, EPI_STORE_ACT = 2, EPI_SWIGLU_ACT = 3, EPI_SCATTER_ACT = 4,
+           EPI_VOCAB_STATS = 5 };
+
 
 // SIMT fp32/generic path: out[t, n] (op)= sum_k x[t,k] w[n,k].
 template <typename T>
@@ -138,6 +160,11 @@ struct TcGemm {
                      // writes its partial sums at out + s * split_stride (floats)
   size_t split_stride;
   int tma_out;       // set by the launcher: the output goes out through TMA stores
+  // EPI_VOCAB_STATS (dense, the tied LM head): out is VocabStat [T][n_groups] with
+  // n_groups = ceil(M / 32); the logits are scaled by zscale (argmax_mode: counts of maxima)
+  float zscale;
+  int argmax_mode;
+  int n_groups;
 };
 // Returns 0, or -1 when the tile does not fit a two-stage pipeline (nothing launched).
 // b: token map with boxes of ntile rows.  bsub (grouped modes, or NULL): maps of the
