@@ -10,7 +10,9 @@ to the prompt, so every step does the same work.  Weights (49 GB) exceed L2.
 
 With full_b1 the same run then measures the batch-16 workload (full_b16: 16
 requests with 4096-token prompts, 4 blocks of 12 fixed steps per bench step)
-and reports it under "workloads" (skip with --no-b16).  The JSON line carries
+and full_b1 again with NVFP4 expert weights, and reports them under
+"workloads" (skip with --no-b16 / --no-nvfp4); full_b1 also times AR-mode
+decode on the same weights ("ar_decode").  The JSON line carries
 the block-level roofline ("roofline_step": the sum over the block's passes of
 max(bytes / HBM, flops / bf16 peak) against the measured block time), the
 dominant kernel's roofline and every major kernel class's, from one extra
@@ -54,6 +56,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["full_b1", "full_b16"], default="full_b1")
     ap.add_argument("--no-b16", action="store_true", help="with full_b1: skip the batch-16 companion measurement")
+    ap.add_argument("--no-nvfp4", action="store_true", help="with full_b1: skip the NVFP4-expert companion")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
@@ -204,7 +207,7 @@ def moe_down_bytes(model, n_rows, touched):
     return touched * f * d * 2 + n_rows * f * 2 + n_rows * d * 2
 
 
-def pass_cost(model, batch, canvas, prompt, touched, causal, head, self_cond):
+def pass_cost(model, batch, canvas, prompt, touched, causal, head, self_cond, expert_bytes=2.0):
     """Algorithmic (bytes, flops) of one forward pass over batch x canvas tokens
     at cache length `prompt`: every weight read once (experts only if touched,
     `touched` distinct experts per layer), the KV cache read once and the
@@ -212,13 +215,14 @@ def pass_cost(model, batch, canvas, prompt, touched, causal, head, self_cond):
     causal: the hand-off pass (query i sees prompt + i + 1 keys) instead of the
     bidirectional canvas step.  head: the LM head; self_cond: the W_sc product.
     Activations and logits between kernels are not counted (a fused path need
-    not write them)."""
+    not write them).  expert_bytes: bytes per expert weight (2 for bf16; 0.5625
+    for NVFP4: half a byte of code and a sixteenth of a byte of block scale)."""
     d, hq, hkv, hd = model["d_model"], model["n_heads"], model["n_kv_heads"], model["head_dim"]
     E, k, F, V, L = model["n_experts"], model["top_k"], model["d_ff"], model["vocab"], model["n_layers"]
     T = batch * canvas
     attn_w = ((hq + 2 * hkv) * hd * d + d * hq * hd) * 2
     router_w = E * d * 2
-    expert_w = 3 * F * d * 2
+    expert_w = 3 * F * d * expert_bytes
     kv_pos = hkv * hd * 2 * 2                      # K and V, bf16, per position per layer
     byt = L * (attn_w + router_w + touched * expert_w + batch * prompt * kv_pos + 2 * T * kv_pos)
     if head:
@@ -235,7 +239,7 @@ def pass_cost(model, batch, canvas, prompt, touched, causal, head, self_cond):
     return float(byt), float(fl)
 
 
-def block_roofline(model, batch, canvas, blocks, touched, block_ms, peaks, sustained=True):
+def block_roofline(model, batch, canvas, blocks, touched, block_ms, peaks, sustained=True, expert_bytes=2.0):
     """Roofline of whole blocks (denoise steps + hand-off): the bound time is the
     sum over passes of max(bytes / HBM, flops / bf16 peak); frac = bound / measured."""
     hbm = peaks["hbm_gbs"] * 1e9
@@ -243,13 +247,13 @@ def block_roofline(model, batch, canvas, blocks, touched, block_ms, peaks, susta
     bound_s, byt_all, fl_all, steps_all, hbm_s, tc_s = 0.0, 0.0, 0.0, 0, 0.0, 0.0
     for prompt, steps in blocks:
         for t in range(1, steps + 1):
-            b, f = pass_cost(model, batch, canvas, prompt, touched, False, True, t > 1)
+            b, f = pass_cost(model, batch, canvas, prompt, touched, False, True, t > 1, expert_bytes)
             bound_s += max(b / hbm, f / tf)
             hbm_s += b / hbm
             tc_s += f / tf
             byt_all += b
             fl_all += f
-        b, f = pass_cost(model, batch, canvas, prompt, touched, True, False, False)
+        b, f = pass_cost(model, batch, canvas, prompt, touched, True, False, False, expert_bytes)
         bound_s += max(b / hbm, f / tf)
         hbm_s += b / hbm
         tc_s += f / tf
@@ -272,7 +276,7 @@ def block_roofline(model, batch, canvas, blocks, touched, block_ms, peaks, susta
                         "between kernels not counted"}
 
 
-def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, peak_kind):
+def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, peak_kind, expert_bytes=2.0):
     """Per-kernel-class roofline from one profiled block (every class timed on
     the library's stream).  Returns {class: roofline} with algorithmic bytes or
     flops per launch over the class's mean launch time."""
@@ -308,8 +312,12 @@ def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, pe
         nl, _ = breakdown["attention"]
         add("attention", "attn_tc_kernel (+ split combine)", "tensor", attention_flops(model, batch, canvas, blocks) / nl)
     if batch == 1:
-        add("moe_up", "gemm_tc_kernel (grouped gate/up + SwiGLU)", "hbm", moe_up_bytes(model, rows, touched))
-        add("moe_down", "gemm_tc_kernel (grouped down, scatter)", "hbm", moe_down_bytes(model, rows, touched))
+        wb = expert_bytes / 2.0      # the weight terms of the byte counts scale with the storage
+        up_b = moe_up_bytes(model, rows, touched) - touched * 2 * F * d * 2 * (1 - wb)
+        down_b = moe_down_bytes(model, rows, touched) - touched * F * d * 2 * (1 - wb)
+        kname = "gemm_fp4_kernel" if expert_bytes < 2.0 else "gemm_tc_kernel"
+        add("moe_up", f"{kname} (grouped gate/up + SwiGLU)", "hbm", up_b)
+        add("moe_down", f"{kname} (grouped down, scatter)", "hbm", down_b)
     else:
         add("moe_up", "gemm_tc_kernel (grouped gate/up + SwiGLU)", "tensor", 2.0 * rows * 2 * F * d)
         add("moe_down", "gemm_tc_kernel (grouped down, scatter)", "tensor", 2.0 * rows * F * d)
@@ -367,7 +375,25 @@ def _measure_ar(m, h, W, dev, warmup=4, steps=32):
             "cache_from": P0}
 
 
-def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clocks=True, with_ar=False):
+def quantize_experts(m, w):
+    """Replace every layer's bf16 expert stacks by NVFP4 (codes, tiled block
+    scales, per-matrix scales) with the library's device quantiser."""
+    import torch
+    for L in w["layers"]:
+        for name in ("w_gate", "w_up", "w_down"):
+            x = L[name]
+            n, rows, K = x.shape
+            codes = torch.empty((n, rows, K // 2), dtype=torch.uint8, device=x.device)
+            scales = torch.empty(m.nvfp4_scales_shape(n, rows, K), dtype=torch.uint8, device=x.device)
+            g = torch.empty(n, dtype=torch.float32, device=x.device)
+            m.dg_quantize_nvfp4(x, codes, scales, g)
+            torch.cuda.synchronize(x.device)
+            L[name], L[name + "_sf"], L[name + "_g"] = codes, scales, g
+            del x
+    torch.cuda.empty_cache()
+
+
+def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clocks=True, with_ar=False, nvfp4=False):
     """Build the workload's model, time `steps` bench steps after `warmup`, then
     an end-to-end pass and one profiled block.  Returns a dict of results."""
     import torch
@@ -380,7 +406,10 @@ def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clock
     max_ctx = ((P0 + blocks * n + 63) // 64) * 64
     max_tokens = max(B * n, min(8192, B * P0))
     w = synth.make_weights(model, seed=W["seed"], dtype=W["dtype"], router_bias=W["router_bias"], device=dev)
-    h = m.dg_create(model, w, dtype=W["dtype"], max_batch=B, max_ctx=max_ctx, max_tokens=max_tokens)
+    if nvfp4:
+        quantize_experts(m, w)
+    h = m.dg_create(model, w, dtype=W["dtype"], max_batch=B, max_ctx=max_ctx, max_tokens=max_tokens,
+                    expert_format=m.DG_EXPERT_NVFP4 if nvfp4 else m.DG_EXPERT_DTYPE)
     req = list(range(B))
     prompt = synth.uniform_tokens(P0, model["vocab"], seed=W["seed"] + 1, batch=B, device=dev)
     t0 = time.time()
@@ -559,6 +588,29 @@ def run_ours(args):
             "clocks": q["clocks"],
             "kernel_ms_per_block": {k: round(v[1] / len(q["prof_blocks"]), 3) for k, v in q["breakdown"].items()},
         }}
+    if args.workload == "full_b1" and not args.no_nvfp4:
+        # the same workload with NVFP4 expert weights (quantised on the device by the library)
+        q = _measure_workload(m, args, "full_b1", max(1, min(args.steps, 3)), max(1, min(args.warmup, 2)), dev,
+                              dist, world, nvfp4=True)
+        ew = 0.5 + 1.0 / 16.0
+        blk_ms = q["elapsed_max"] / q["steps"]
+        line.setdefault("workloads", {})["full_b1_nvfp4"] = {
+            "value": round(q["units_all"] / (q["elapsed_max"] / 1e3), 2), "unit": "tokens/s",
+            "steps": q["steps"], "warmup": q["warmup"], "ms_per_step": round(blk_ms, 3),
+            "us_per_denoise_step": round(q["elapsed_max"] * 1e3 / max(1, q["denoise_steps"]), 1),
+            "denoise_steps_per_block": round(q["denoise_steps"] / q["steps"], 2),
+            "config": {"expert_weights": "NVFP4 (E2M1 codes, E4M3 scales per 16, fp32 per matrix)",
+                       "expert_bytes_per_weight": ew},
+            "e2e": {"value": round(q["units_all"] / (q["e2e_max"] / 1e3), 2), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4 * n},
+            "gpu_launches": int(q["launches"]),
+            "roofline_step": block_roofline(q["model"], 1, n, q["timed_blocks"][:1], q["touched"], blk_ms, peaks,
+                                            expert_bytes=ew),
+            "rooflines": kernel_rooflines(q["model"], 1, n, q["prof_blocks"], q["touched"], q["breakdown"], peaks,
+                                          peak_kind, expert_bytes=ew),
+            "clocks": q["clocks"],
+            "kernel_ms_per_block": {k: round(v[1] / len(q["prof_blocks"]), 3) for k, v in q["breakdown"].items()},
+        }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(r["W"], line["denoise_steps_per_block"])
     if dist is not None:

@@ -97,6 +97,19 @@ bool tmap_chunks4(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// uint8 codes of n_mats stacked [rows][K/2] matrices: dims (K/2, rows, n_mats), box (32 bytes, 128 rows, 1),
+// no swizzle (the dequantising threads read them row by row).
+bool tmap_codes(CUtensorMap* m, const void* ptr, uint64_t half_k, uint64_t rows, uint64_t n_mats) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {half_k, rows, n_mats};
+  cuuint64_t strides[2] = {half_k, half_k * rows};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 enum ProfClass {
   PC_EMBED, PC_DENSE, PC_ROPE, PC_ATTN, PC_NORM, PC_ROUTER, PC_GATHER, PC_MOE_UP, PC_MOE_DOWN, PC_COMBINE,
   PC_LMHEAD, PC_SAMPLER, PC_FINISH, PC_COUNT
@@ -120,6 +133,7 @@ struct WMap {
 };
 struct LayerMaps {
   WMap wq, wk, wv, wo, router, gate, up, down;
+  CUtensorMap gate_c, up_c, down_c;   // NVFP4 expert codes
 };
 struct BMapEntry {
   const void* p;
@@ -136,6 +150,7 @@ struct OMapEntry {
 struct dg_handle {
   dg_config c{};
   bool bf16 = false;
+  bool fp4 = false;     // expert weights stored as NVFP4
   size_t esz = 4;
   cudaStream_t stream = nullptr;
   int num_sms = 148;
@@ -554,7 +569,59 @@ int qkv_gemm(dg_handle* H, int l, int T) {
   return 0;
 }
 
+void moe_gemms_fp4(dg_handle* H, int l, int T) {
+  const dg_config& c = H->c;
+  const dg_layer_weights& L = H->lw[l];
+  const LayerMaps& M = H->lmaps[l];
+  const int tile = grouped_tile(H, T);
+  const uint64_t rows = (uint64_t)H->T_max * c.top_k;
+  Fp4Gemm g{};
+  g.ntile = tile;
+  g.work = H->work;
+  g.n_work = H->n_work;
+  g.n_work_max = c.n_experts + (T * c.top_k + tile - 1) / tile;
+  g.err = H->d_err;
+  CUtensorMap bsub[3];
+  {
+    ProfScope ps(H, PC_MOE_UP);
+    g.mode = 1;
+    g.M = c.d_ff;
+    g.K = c.d_model;
+    g.out = H->hb;
+    g.ld_out = c.d_ff;
+    g.sf0 = L.w_gate_sf;
+    g.sf1 = L.w_up_sf;
+    g.g0 = L.w_gate_g;
+    g.g1 = L.w_up_g;
+    const CUtensorMap* b = bmap(H, H->xp, c.d_model, rows, tile, 1);
+    if (!b || !grouped_bsub(H, H->xp, c.d_model, rows, 1, bsub) ||
+        launch_gemm_fp4(M.gate_c, M.up_c, *b, bsub, g, H->num_sms, H->stream) != 0)
+      H->bad_launch = true;
+  }
+  {
+    ProfScope ps(H, PC_MOE_DOWN);
+    g.mode = 2;
+    g.M = c.d_model;
+    g.K = c.d_ff;
+    g.out = H->y;
+    g.ld_out = c.d_model;
+    g.row_map = H->perm;
+    g.sf0 = L.w_down_sf;
+    g.sf1 = nullptr;
+    g.g0 = L.w_down_g;
+    g.g1 = nullptr;
+    const CUtensorMap* b = bmap(H, H->hb, c.d_ff, rows, tile, 1);
+    if (!b || !grouped_bsub(H, H->hb, c.d_ff, rows, 1, bsub) ||
+        launch_gemm_fp4(M.down_c, M.down_c, *b, bsub, g, H->num_sms, H->stream) != 0)
+      H->bad_launch = true;
+  }
+}
+
 void moe_gemms(dg_handle* H, int l, int T) {
+  if (H->fp4) {
+    moe_gemms_fp4(H, l, T);
+    return;
+  }
   const dg_config& c = H->c;
   const dg_layer_weights& L = H->lw[l];
   const int tile = grouped_tile(H, T);
@@ -950,6 +1017,10 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
     if (!(c.rms_eps > 0) || !(c.rope_base > 1)) return fail(nullptr, DG_EINVAL, "bad rms_eps / rope_base");
     if (c.dtype == DG_BF16 && (c.d_model % 64 || c.d_ff % 64 || c.head_dim % 64))
       return fail(nullptr, DG_EINVAL, "bf16 needs d_model, d_ff, head_dim multiples of 64");
+    if (c.expert_format != DG_EXPERT_DTYPE && c.expert_format != DG_EXPERT_NVFP4)
+      return fail(nullptr, DG_EINVAL, "unknown expert_format %d", c.expert_format);
+    if (c.expert_format == DG_EXPERT_NVFP4 && c.dtype != DG_BF16)
+      return fail(nullptr, DG_EINVAL, "NVFP4 experts need a bf16 handle");
     if (!w || !w->embed || !w->w_sc || !w->final_norm || !w->layers)
       return fail(nullptr, DG_EINVAL, "null weight pointer");
     if (!aligned16(w->final_norm)) return fail(nullptr, DG_EINVAL, "unaligned final_norm");
@@ -958,6 +1029,11 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
       const void* ps[] = {L.attn_norm, L.wq, L.wk, L.wv, L.wo, L.ffn_norm, L.router_w, L.w_gate, L.w_up, L.w_down};
       for (const void* p : ps)
         if (!p || !aligned16(p)) return fail(nullptr, DG_EINVAL, "layer %d: null or unaligned weight", l);
+      if (c.expert_format == DG_EXPERT_NVFP4) {
+        const void* qs[] = {L.w_gate_sf, L.w_up_sf, L.w_down_sf, L.w_gate_g, L.w_up_g, L.w_down_g};
+        for (const void* p : qs)
+          if (!p || !aligned16(p)) return fail(nullptr, DG_EINVAL, "layer %d: null or unaligned NVFP4 scales", l);
+      }
     }
     if (!aligned16(w->embed) || !aligned16(w->w_sc)) return fail(nullptr, DG_EINVAL, "unaligned embed / w_sc");
     // the router needs finite gate logits: a non-finite bias is refused here
@@ -980,6 +1056,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
     return fail(nullptr, DG_EINVAL, "max_tokens < max_batch * canvas");
   }
   H->bf16 = c.dtype == DG_BF16;
+  H->fp4 = model && c.expert_format == DG_EXPERT_NVFP4;
   H->esz = H->bf16 ? 2 : 4;
   H->stream = (cudaStream_t)stream;
   cudaGetDevice(&H->dev);
@@ -1096,9 +1173,15 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
         dense(M.wv, L.wv, d, kw);
         dense(M.wo, L.wo, qw, d);
         dense(M.router, L.router_w, d, E);
-        experts(M.gate, L.w_gate, d, F);
-        experts(M.up, L.w_up, d, F);
-        experts(M.down, L.w_down, F, d);
+        if (H->fp4) {
+          tm &= tmap_codes(&M.gate_c, L.w_gate, d / 2, F, E);
+          tm &= tmap_codes(&M.up_c, L.w_up, d / 2, F, E);
+          tm &= tmap_codes(&M.down_c, L.w_down, F / 2, d, E);
+        } else {
+          experts(M.gate, L.w_gate, d, F);
+          experts(M.up, L.w_up, d, F);
+          experts(M.down, L.w_down, F, d);
+        }
       }
       tm &= tmap_chunks(&H->m_embed.k1, H->embed, d, c.vocab, d, 128, 1);
       tm &= tmap_chunks(&H->m_embed.k2, H->embed, d, c.vocab, d, 128, 2);

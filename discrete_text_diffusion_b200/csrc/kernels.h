@@ -177,6 +177,31 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
                    const CUtensorMap* tout = nullptr);
 int gemm_tc_smem_bytes(const TcGemm& p, int* stages);
 
+// NVFP4 grouped expert GEMMs (k_gemm_fp4.cu): modes 1 (gate/up + SwiGLU) and 2
+// (down + scatter) of the bf16 grouped GEMM, with the weights as E2M1 codes
+// (c0 / c1: uint8 maps (K/2 bytes, M rows, E) with boxes of 32 bytes x 128
+// rows), tiled E4M3 scales and per-expert fp32 scales.  b / bsub: the token
+// maps, as for launch_gemm_tc.  Returns -1 (nothing launched) for an
+// unsupported shape.
+struct Fp4Gemm {
+  int mode;
+  int M, K;
+  int ntile;
+  const int32_t* work;
+  const int32_t* n_work;
+  int n_work_max;
+  void* out;
+  int ld_out;
+  const int32_t* row_map;
+  int* err;
+  const uint8_t* sf0;
+  const uint8_t* sf1;
+  const float* g0;
+  const float* g1;
+};
+int launch_gemm_fp4(const CUtensorMap& c0, const CUtensorMap& c1, const CUtensorMap& b, const CUtensorMap* bsub,
+                    const Fp4Gemm& g, int num_sms, cudaStream_t s);
+
 // ---- attention
 struct AttnArgs {
   int B, nq, hq, hkv, hd, max_ctx;

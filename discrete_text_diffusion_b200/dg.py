@@ -24,7 +24,7 @@ EXPORTS = (
     "dg_get_length", "dg_denoise_step", "dg_sample", "dg_generate_block", "dg_generate_block_host",
     "dg_synchronize", "dg_launch_count", "dg_profile_enable", "dg_profile_read", "dg_profile_reset",
     "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc", "dg_selftest_gemm_split", "dg_get_kv",
-    "dg_selftest_router", "dg_selftest_wait_timeout", "dg_ar_step",
+    "dg_selftest_router", "dg_selftest_wait_timeout", "dg_ar_step", "dg_quantize_nvfp4",
 )
 
 
@@ -32,12 +32,14 @@ class DgConfig(C.Structure):
     _fields_ = [("n_layers", C.c_int), ("d_model", C.c_int), ("n_heads", C.c_int), ("n_kv_heads", C.c_int),
                 ("head_dim", C.c_int), ("n_experts", C.c_int), ("top_k", C.c_int), ("d_ff", C.c_int),
                 ("vocab", C.c_int), ("canvas", C.c_int), ("max_batch", C.c_int), ("max_ctx", C.c_int),
-                ("max_tokens", C.c_int), ("dtype", C.c_int), ("rope_base", C.c_double), ("rms_eps", C.c_double)]
+                ("max_tokens", C.c_int), ("dtype", C.c_int), ("rope_base", C.c_double), ("rms_eps", C.c_double),
+                ("expert_format", C.c_int)]
 
 
 class DgLayerWeights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "router_w",
-                                          "router_b", "w_gate", "w_up", "w_down")]
+                                          "router_b", "w_gate", "w_up", "w_down", "w_gate_sf", "w_up_sf",
+                                          "w_down_sf", "w_gate_g", "w_up_g", "w_down_g")]
 
 
 class DgWeights(C.Structure):
@@ -51,6 +53,9 @@ class DgSamplerParams(C.Structure):
                 ("entropy_budget", C.c_float), ("stop_mode", C.c_int), ("prev_argmax", C.c_void_p),
                 ("prev_mean_entropy", C.c_void_p)]
 
+
+DG_EXPERT_DTYPE = 0
+DG_EXPERT_NVFP4 = 1
 
 DG_KEEP_TOPK = 0
 DG_KEEP_ENTROPY_BUDGET = 1
@@ -112,6 +117,7 @@ def lib():
         L.dg_selftest_router.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(DgRouterOut)]
         L.dg_selftest_wait_timeout.argtypes = [P, C.c_int]
         L.dg_ar_step.argtypes = [P, C.c_int, C.POINTER(C.c_int), P, P, P]
+        L.dg_quantize_nvfp4.argtypes = [P, C.c_int, C.c_int, C.c_int, P, P, P, P, C.c_char_p, C.c_size_t]
         L.dg_set_length.argtypes = [P, C.c_int, C.c_int]
         L.dg_get_length.argtypes = [P, C.c_int, C.POINTER(C.c_int)]
         L.dg_denoise_step.argtypes = [P, C.POINTER(DgStepArgs), C.POINTER(DgStepOut)]
@@ -173,20 +179,24 @@ class Handle:
             pass
 
 
-def _cfg(model: dict, *, dtype: str, max_batch: int, max_ctx: int, max_tokens: int = 0) -> DgConfig:
+def _cfg(model: dict, *, dtype: str, max_batch: int, max_ctx: int, max_tokens: int = 0,
+         expert_format: int = DG_EXPERT_DTYPE) -> DgConfig:
     m = model
     return DgConfig(m.get("n_layers", 0), m.get("d_model", 0), m.get("n_heads", 0), m.get("n_kv_heads", 0),
                     m.get("head_dim", 0), m.get("n_experts", 0), m.get("top_k", 0), m.get("d_ff", 0),
                     m["vocab"], m["canvas"], max_batch, max_ctx, max_tokens,
                     DG_BF16 if dtype == "bf16" else DG_FP32, float(m.get("rope_base", 10000.0)),
-                    float(m.get("rms_eps", 1e-6)))
+                    float(m.get("rms_eps", 1e-6)), expert_format)
 
 
 def dg_create(model: dict, weights, *, dtype: str, max_batch: int, max_ctx: int, max_tokens: int = 0,
-              stream=None) -> Handle:
+              stream=None, expert_format: int = DG_EXPERT_DTYPE) -> Handle:
     """dg_create.  weights: dict of device tensors (synth.make_weights layout) or None
-    for a sampler-only handle (model['n_layers'] == 0)."""
-    cfg = _cfg(model, dtype=dtype, max_batch=max_batch, max_ctx=max_ctx, max_tokens=max_tokens)
+    for a sampler-only handle (model['n_layers'] == 0).  With expert_format
+    DG_EXPERT_NVFP4 each layer's w_gate / w_up / w_down are the codes and the layer
+    also holds w_gate_sf ... w_down_g (see dg_quantize_nvfp4)."""
+    cfg = _cfg(model, dtype=dtype, max_batch=max_batch, max_ctx=max_ctx, max_tokens=max_tokens,
+               expert_format=expert_format)
     keep = [weights]
     wp = None
     if weights is not None:
@@ -319,6 +329,23 @@ def dg_ar_step(h: Handle, req, tokens, logits, next_token=None):
     """AR mode: append tokens [B] (int32, device) causally; logits [B, V] fp32 of the next token;
     next_token [B] int32 (argmax) or None."""
     return h.check(lib().dg_ar_step(h.ptr, len(req), _ints(req), _ptr(tokens), _ptr(logits), _ptr(next_token)))
+
+
+def nvfp4_scales_shape(n_mats: int, rows: int, K: int):
+    """Shape of the tiled block scales dg_quantize_nvfp4 writes: [n_mats, K/64, rows_pad, 4]."""
+    return (n_mats, K // 64, (rows + 127) // 128 * 128, 4)
+
+
+def dg_quantize_nvfp4(w, codes, scales, g, stream=None):
+    """w [n_mats, rows, K] bf16 -> codes [n_mats, rows, K/2] uint8, scales (nvfp4_scales_shape) uint8,
+    g [n_mats] float32, all on the device."""
+    n_mats, rows, K = w.shape
+    err = C.create_string_buffer(256)
+    sptr = None if stream is None else C.c_void_p(stream.cuda_stream)
+    rc = lib().dg_quantize_nvfp4(_ptr(w), n_mats, rows, K, _ptr(codes), _ptr(scales), _ptr(g), sptr, err, len(err))
+    if rc != 0:
+        raise DgError(rc, err.value.decode())
+    return rc
 
 
 def dg_synchronize(h: Handle):

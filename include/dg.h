@@ -79,7 +79,23 @@ typedef struct dg_config {
   int dtype;         /* DG_BF16 or DG_FP32 */
   double rope_base;  /* RoPE base (10000) */
   double rms_eps;    /* RMSNorm epsilon */
+  int expert_format; /* DG_EXPERT_DTYPE (0: experts in the handle's dtype) or DG_EXPERT_NVFP4 (bf16 handles) */
 } dg_config;
+
+/* Storage of the expert weights ([P2] 推荐的部署与优化方案 and [P4] MoE 26B参数架构分析:
+ * the model ships NVFP4 weights for Blackwell).
+ * DG_EXPERT_NVFP4: each expert matrix [out, in] (in a multiple of 64) is
+ *   - codes: [out, in/2] bytes of FP4 E2M1 codes, element 2j in the low nibble
+ *     of byte j (OCP MX E2M1: 1 sign, 2 exponent, 1 mantissa bit);
+ *   - block scales: one E4M3 code per 16 consecutive elements of a row, stored
+ *     tiled as [in/64][out_pad][4] bytes, out_pad = out rounded up to 128
+ *     (entry [k/64][row][(k%64)/16]; padding rows are 0);
+ *   - g: one fp32 scale per matrix;
+ *   value = E2M1(code) * E4M3(scale) * g.  dg_quantize_nvfp4 produces it.
+ * Activations stay bf16: the kernels expand the codes to bf16 (exact: at most
+ * 6 significant bits) ahead of the bf16 tensor-core product and apply g to
+ * the fp32 accumulator. */
+enum { DG_EXPERT_DTYPE = 0, DG_EXPERT_NVFP4 = 1 };
 
 /* One layer's weights (all borrowed device pointers). */
 typedef struct dg_layer_weights {
@@ -94,6 +110,13 @@ typedef struct dg_layer_weights {
   const void* w_gate;      /* [E, F, d] */
   const void* w_up;        /* [E, F, d] */
   const void* w_down;      /* [E, d, F] */
+  /* DG_EXPERT_NVFP4 only (w_gate / w_up / w_down then hold the codes [E, out, in/2]): */
+  const uint8_t* w_gate_sf;  /* block scales [E][d/64][F_pad][4] */
+  const uint8_t* w_up_sf;    /* [E][d/64][F_pad][4] */
+  const uint8_t* w_down_sf;  /* [E][F/64][d_pad][4] */
+  const float* w_gate_g;     /* [E] per-matrix fp32 scales */
+  const float* w_up_g;       /* [E] */
+  const float* w_down_g;     /* [E] */
 } dg_layer_weights;
 
 typedef struct dg_weights {
@@ -427,6 +450,25 @@ int dg_selftest_gemm_split(dg_handle* h, const void* x, const void* w, int T, in
  * device error flag cleared, so the handle stays usable.
  */
 int dg_selftest_wait_timeout(dg_handle* h, int limit_us);
+
+/*
+ * NVFP4 quantisation of n_mats bf16 matrices w [n_mats][rows][K] (K a multiple
+ * of 64, rows >= 1), the storage of DG_EXPERT_NVFP4, computed on the device
+ * without allocating.  Per matrix: g = fp32(amax / (6 * 448)) (1 for an
+ * all-zero matrix); per block of 16 elements of a row: scale code
+ * s = E4M3(amax_b / (6 g)); element code q = E2M1(w / (E4M3(s) g)), both
+ * rounded to nearest with ties to the even code and saturated (a block whose
+ * scale is 0 gets codes 0).  Quotients are formed in fp64.
+ *   codes:  [n_mats][rows][K/2] bytes (element 2j in the low nibble)
+ *   scales: [n_mats][K/64][rows_pad][4] bytes, rows_pad = rows rounded up to
+ *           128; padding rows are written as 0
+ *   g:      [n_mats] fp32
+ * All device pointers; stream: a cudaStream_t (NULL = legacy default).
+ * Returns DG_OK, DG_EINVAL (bad shape, null or unaligned pointer: w and codes
+ * 16-byte aligned) or DG_ECUDA; err (err_len bytes, may be NULL) gets the message.
+ */
+int dg_quantize_nvfp4(const void* w, int n_mats, int rows, int K, uint8_t* codes, uint8_t* scales, float* g,
+                      void* stream, char* err, size_t err_len);
 
 /* Outputs of the router self-test (all device pointers, all required). */
 typedef struct dg_router_out {
