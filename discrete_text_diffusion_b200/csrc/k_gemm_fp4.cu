@@ -9,17 +9,20 @@
 // has at most 6 significant bits and lies in [2^-10, 2688], so it is exact in
 // bf16, and the per-matrix scale is applied to the fp32 accumulator.
 //
-// 320 threads per CTA:
-//   warp 0 lane 0: producer.  Per 64-wide K stage: one TMA box of the codes
-//     (128 rows x 32 bytes) per weight operand and one 512-byte bulk copy of
-//     their scales (tiled [K/64][rows_pad][4]) into a raw area, signalled on
-//     raw_full; the token box (bf16, 128-byte swizzle) straight into the stage.
+// 480 threads per CTA:
+//   warp 0 lane 0: token producer: the token box (bf16, 128-byte swizzle) of
+//     each 64-wide K stage into the stage ring.
 //   warp 1 lane 0: tcgen05.mma issuer (M = 128, N = token rows, K = 16).
 //   warps 2-5: epilogue (TMEM -> scale by g -> SwiGLU or scatter).
-//   warps 6-9: dequantisation.  Thread t expands row t of each weight operand
-//     (64 codes, 4 scales) into 64 bf16 in the 128-byte-swizzled K-major tile
-//     the MMA reads, then arrives on the stage's full barrier (which also
-//     carries the token TMA's bytes).
+//   warp 6 lane 0: code producer: one TMA box of codes (128 rows x 32 bytes)
+//     and one 512-byte bulk copy of their scales (tiled [K/64][rows_pad][4])
+//     per weight operand and stage, into a deeper ring of raw slots, so that
+//     the HBM reads of the weights run well ahead of the MMA.
+//   warps 7-14: dequantisation.  Two threads per tile row expand 32 codes each
+//     through a 256-entry table (a code byte -> its two E2M1 values as bf16x2)
+//     and one bf16x2 multiply by the block scale, into the 128-byte-swizzled
+//     K-major tile the MMA reads; then they free the raw slot and arrive on
+//     the stage's full barrier (which also carries the token box's bytes).
 // Weight bytes per 128 x 64 tile: 4 KB of codes + 512 B of scales instead of
 // 16 KB of bf16.
 #include <cuda_bf16.h>
@@ -35,13 +38,14 @@ namespace {
 
 constexpr int kFBM = 128;
 constexpr int kFBK = 64;
-constexpr int kFThreads = 320;
+constexpr int kFThreads = 480;
+constexpr int kDeqThreads = 256;
 constexpr int kTileBytes = kFBM * kFBK * 2;   // 16 KB bf16 weight tile
 constexpr int kCodeBytes = kFBM * kFBK / 2;   // 4 KB of codes
 constexpr int kSfBytes = kFBM * 4;            // 512 B of scales
 constexpr int kMaxSmemF = 232448;
-constexpr int kSmemPerSmF = 233472;
 constexpr int kEpiRowsF = 32;
+constexpr int kRawSlots = 8;
 
 struct Fp4Params {
   int mode;               // 1 gate/up, 2 down
@@ -57,8 +61,8 @@ struct Fp4Params {
   const uint8_t* sf1;     // scales of operand 1 (up)
   const float* g0;        // per-expert fp32 scales
   const float* g1;
-  int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, box_levels, vec;
-  int off_b, off_raw;     // byte offsets inside a stage: token tile, raw codes / scales
+  int stages, stage_bytes, raw_bytes, acc_cols, n_acc_buf, tmem_cols, n_mtiles, box_levels, vec;
+  int off_b;              // byte offset of the token tile inside a stage
 };
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -94,26 +98,38 @@ __global__ void __launch_bounds__(kFThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* stage0 = base;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + P.stages * P.stage_bytes);
-  uint64_t* full = bars;                      // tokens' bytes + 128 dequantisation arrivals
-  uint64_t* empty = bars + P.stages;          // the MMA has read the stage
-  uint64_t* raw_full = bars + 2 * P.stages;   // codes and scales have landed
-  uint64_t* acc_full = bars + 3 * P.stages;
+  uint8_t* stage0 = base;                                         // [stages][stage_bytes]
+  uint8_t* raw0 = base + P.stages * P.stage_bytes;                // [kRawSlots][raw_bytes]
+  uint32_t* lut = reinterpret_cast<uint32_t*>(raw0 + kRawSlots * P.raw_bytes);   // 256 bf16x2
+  uint64_t* bars = reinterpret_cast<uint64_t*>(lut + 256);
+  uint64_t* full = bars;                          // token bytes + 256 dequantisation arrivals
+  uint64_t* empty = full + P.stages;              // the MMA has read the stage
+  uint64_t* raw_full = empty + P.stages;          // codes and scales landed
+  uint64_t* raw_empty = raw_full + kRawSlots;     // the dequantisation has read them
+  uint64_t* acc_full = raw_empty + kRawSlots;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  __nv_bfloat16* stg_b = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(bars) + 512);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = P.err;
   const int n_a = P.mode == 1 ? 2 : 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < P.stages; ++s) {
-      mbar_init(&full[s], 1 + 128);
+      mbar_init(&full[s], 1 + kDeqThreads);
       mbar_init(&empty[s], 1);
-      mbar_init(&raw_full[s], 1);
+    }
+    for (int r = 0; r < kRawSlots; ++r) {
+      mbar_init(&raw_full[r], 1);
+      mbar_init(&raw_empty[r], kDeqThreads);
     }
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
     fence_mbar_init();
+  }
+  // byte of two E2M1 codes (element 2j low nibble) -> bf16x2 of their values
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(e2m1_f(i & 0xF), e2m1_f(i >> 4));
+    lut[i] = *reinterpret_cast<const uint32_t*>(&v);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, (uint32_t)P.tmem_cols);
@@ -136,12 +152,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
   const int nkc = P.K / kFBK;
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ token producer
     uint32_t kiter = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-      const int mt = item % P.n_mtiles, w = item / P.n_mtiles;
-      const int m0 = mt * kFBM, e = P.work[3 * w], row0 = P.work[3 * w + 1], rows = P.work[3 * w + 2];
+      const int w = item / P.n_mtiles;
+      const int row0 = P.work[3 * w + 1], rows = P.work[3 * w + 2];
       int lvl;
       const int box = fp4_item_box(P, rows, &lvl);
       const CUtensorMap* bm = box == P.ntile ? &tb : (lvl == 0 ? &tbs0 : lvl == 1 ? &tbs1 : &tbs2);
@@ -149,18 +165,30 @@ __global__ void __launch_bounds__(kFThreads, 1)
         const int s = kiter % P.stages;
         const uint32_t ph = (kiter / P.stages) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
-        uint8_t* st = stage0 + (size_t)s * P.stage_bytes;
-        uint8_t* rw = st + P.off_raw;
-        mbar_expect_tx(&raw_full[s], (uint32_t)(n_a * (kCodeBytes + kSfBytes)));
-        tma_load_3d(rw, &tc0, &raw_full[s], j * (kFBK / 2), m0, e);
-        bulk_load(rw + n_a * kCodeBytes, P.sf0 + (((size_t)e * nkc + j) * P.M_pad + m0) * 4, kSfBytes, &raw_full[s]);
-        if (P.mode == 1) {
-          tma_load_3d(rw + kCodeBytes, &tc1, &raw_full[s], j * (kFBK / 2), m0, e);
-          bulk_load(rw + 2 * kCodeBytes + kSfBytes, P.sf1 + (((size_t)e * nkc + j) * P.M_pad + m0) * 4, kSfBytes,
-                    &raw_full[s]);
-        }
         mbar_expect_tx(&full[s], (uint32_t)(box * kFBK * 2));
-        tma_load_3d(st + P.off_b, bm, &full[s], 0, row0, j);
+        tma_load_3d(stage0 + (size_t)s * P.stage_bytes + P.off_b, bm, &full[s], 0, row0, j);
+      }
+    }
+  } else if (warp == 6 && lane == 0) {
+    // ------------------------------------------------------------ code producer
+    uint32_t kiter = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+      const int mt = item % P.n_mtiles, w = item / P.n_mtiles;
+      const int m0 = mt * kFBM, e = P.work[3 * w];
+      for (int j = 0; j < nst; ++j, ++kiter) {
+        const int r = kiter % kRawSlots;
+        const uint32_t ph = (kiter / kRawSlots) & 1u;
+        if (!mbar_wait(&raw_empty[r], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
+        uint8_t* rw = raw0 + (size_t)r * P.raw_bytes;
+        mbar_expect_tx(&raw_full[r], (uint32_t)(n_a * (kCodeBytes + kSfBytes)));
+        tma_load_3d(rw, &tc0, &raw_full[r], j * (kFBK / 2), m0, e);
+        bulk_load(rw + n_a * kCodeBytes, P.sf0 + (((size_t)e * nkc + j) * P.M_pad + m0) * 4, kSfBytes, &raw_full[r]);
+        if (P.mode == 1) {
+          tma_load_3d(rw + kCodeBytes, &tc1, &raw_full[r], j * (kFBK / 2), m0, e);
+          bulk_load(rw + 2 * kCodeBytes + kSfBytes, P.sf1 + (((size_t)e * nkc + j) * P.M_pad + m0) * 4, kSfBytes,
+                    &raw_full[r]);
+        }
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -172,9 +200,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
       const int w = item / P.n_mtiles;
       const int rows = P.work[3 * w + 2];
       const uint32_t idesc = idesc_bf16(kFBM, (rows + 15) & ~15);
-      int lvl;
-      const int bsub = fp4_item_box(P, rows, &lvl) * kFBK * 2;
-      (void)bsub;
       const int ab = it % P.n_acc_buf;
       const uint32_t use = (uint32_t)(it / P.n_acc_buf);
       if (!mbar_wait(&acc_empty[ab], (use & 1u) ^ 1u, err, kErrTimeoutMma)) break;
@@ -199,50 +224,56 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (!ok) break;
       umma_commit(&acc_full[ab]);
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 7) {
     // ------------------------------------------------------------ dequantisation
-    const int t = threadIdx.x - 192;                 // tile row 0..127
-    const uint32_t r8 = (uint32_t)(t & 7);
+    const int t = threadIdx.x - 224;                  // 0..255
+    const int row = t >> 1, half = t & 1;             // tile row, which 32 of its 64 codes
+    const uint32_t r8 = (uint32_t)(row & 7);
     uint32_t kiter = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
       for (int j = 0; j < nst; ++j, ++kiter) {
+        const int r = kiter % kRawSlots;
         const int s = kiter % P.stages;
-        const uint32_t ph = (kiter / P.stages) & 1u;
-        if (!mbar_wait(&raw_full[s], ph, err, kErrTimeoutTma)) { ok = false; break; }
+        if (!mbar_wait(&raw_full[r], (kiter / kRawSlots) & 1u, err, kErrTimeoutTma)) { ok = false; break; }
+        // the stage's previous contents must have been consumed by the MMA
+        if (!mbar_wait(&empty[s], ((kiter / P.stages) & 1u) ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
+        const uint8_t* rw = raw0 + (size_t)r * P.raw_bytes;
         uint8_t* st = stage0 + (size_t)s * P.stage_bytes;
-        const uint8_t* rw = st + P.off_raw;
+        uint4 cw[2];
+        uint32_t sfw[2];
         for (int a = 0; a < n_a; ++a) {
-          const uint4 c0 = *reinterpret_cast<const uint4*>(rw + a * kCodeBytes + t * 32);
-          const uint4 c1 = *reinterpret_cast<const uint4*>(rw + a * kCodeBytes + t * 32 + 16);
-          const uint32_t sfw = *reinterpret_cast<const uint32_t*>(rw + n_a * kCodeBytes + a * kSfBytes + t * 4);
-          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          uint8_t* tile = st + a * kTileBytes + (t >> 3) * 1024 + r8 * 128;
+          cw[a] = *reinterpret_cast<const uint4*>(rw + a * kCodeBytes + row * 32 + half * 16);
+          sfw[a] = *reinterpret_cast<const uint16_t*>(rw + n_a * kCodeBytes + a * kSfBytes + row * 4 + half * 2);
+        }
+        mbar_arrive(&raw_empty[r]);                    // the raw slot is in registers
+        for (int a = 0; a < n_a; ++a) {
+          uint8_t* tile = st + a * kTileBytes + (row >> 3) * 1024 + r8 * 128;
+          const uint32_t words[4] = {cw[a].x, cw[a].y, cw[a].z, cw[a].w};
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {            // 16-byte chunk: elements 8ch .. 8ch+7
-            const float sc = e4m3_f((sfw >> (8 * (ch >> 1))) & 0xFFu);   // 16 elements per scale
-            const uint32_t word = cw[ch];
+          for (int ch = 0; ch < 4; ++ch) {              // 8 elements: one 16-byte chunk of the bf16 row
+            const __nv_bfloat16 sc1 = __float2bfloat16_rn(e4m3_f((sfw[a] >> (8 * (ch >> 1))) & 0xFFu));
+            const __nv_bfloat162 sc = __halves2bfloat162(sc1, sc1);
             uint32_t pk[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const float lo = e2m1_f((word >> (8 * q)) & 0xFu) * sc;
-              const float hi = e2m1_f((word >> (8 * q + 4)) & 0xFu) * sc;
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);
-              pk[q] = *reinterpret_cast<const uint32_t*>(&b2);
+              const uint32_t v = lut[(words[ch] >> (8 * q)) & 0xFFu];
+              const __nv_bfloat162 p2 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&v), sc);
+              pk[q] = *reinterpret_cast<const uint32_t*>(&p2);
             }
-            *reinterpret_cast<uint4*>(tile + (((uint32_t)ch ^ r8) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            const uint32_t c = (uint32_t)(half * 4 + ch);
+            *reinterpret_cast<uint4*>(tile + ((c ^ r8) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
         fence_proxy_async_smem();
         mbar_arrive(&full[s]);
       }
     }
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const int te = threadIdx.x - 64;
-    __nv_bfloat16* stg_b = reinterpret_cast<__nv_bfloat16*>(base + P.stages * P.stage_bytes + 1024);
     __nv_bfloat16* out_b = reinterpret_cast<__nv_bfloat16*>(P.out);
     int it = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
@@ -337,13 +368,13 @@ int launch_gemm_fp4(const CUtensorMap& c0, const CUtensorMap& c1, const CUtensor
   P.tmem_cols = 32;
   while (P.tmem_cols < P.n_acc_buf * P.acc_cols) P.tmem_cols <<= 1;
   P.off_b = n_a * kTileBytes;
-  P.off_raw = P.off_b + g.ntile * kFBK * 2;
-  P.stage_bytes = (P.off_raw + n_a * (kCodeBytes + kSfBytes) + 1023) & ~1023;
-  const int overhead = 1024 /*align*/ + 1024 /*barriers*/ + (g.mode == 2 ? kEpiRowsF * kFBM * 2 : 0);
-  const int budget = std::min(kMaxSmemF, kSmemPerSmF - 1024);
-  P.stages = std::min(8, (budget - overhead) / P.stage_bytes);
+  P.stage_bytes = (P.off_b + g.ntile * kFBK * 2 + 1023) & ~1023;
+  P.raw_bytes = (n_a * (kCodeBytes + kSfBytes) + 1023) & ~1023;
+  // LUT 1 KB, barriers and the down projection's staging tile (8 KB) after the rings
+  const int overhead = 1024 /*align*/ + 1024 /*lut*/ + 512 /*barriers*/ + kEpiRowsF * kFBM * 2;
+  P.stages = std::min(6, (kMaxSmemF - overhead - kRawSlots * P.raw_bytes) / P.stage_bytes);
   if (P.stages < 2) return -1;
-  const int smem = overhead + P.stages * P.stage_bytes;
+  const int smem = overhead + P.stages * P.stage_bytes + kRawSlots * P.raw_bytes;
   P.n_mtiles = (g.M + kFBM - 1) / kFBM;
   P.box_levels = 0;
   if (bsub)
