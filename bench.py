@@ -45,7 +45,14 @@ CSRC = os.path.join(ROOT, "discrete_text_diffusion_b200", "csrc")
 # DRAM bytes (read + write) per launch measured by ncu for a kernel class, with
 # the source file and the sha256 prefix of that file when it was captured.  A
 # class whose source has changed since reports traffic null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # canvas-step attention over an 8192-position cache (16/8 heads of 256): the bench's launch shape
+    "attention": (71365376 + 2604032, "k_attn_tc.cu", "5e28d2db74c28ed9"),
+    # LM head with the sampler statistics, 256 tokens x 262144 vocabulary: the bench's launch shape
+    "lm_head": (1488360960 + 33390336, "k_gemm_tc.cu", "b6966e2537710892"),
+    # the fused sampler pass over 256 rows: the bench's launch shape
+    "sampler_rows": (80628736 + 1649152, "k_sampler.cu", "d9ce1c2931c1b66c"),
+}
 
 
 def parse_args(argv=None):
@@ -58,6 +65,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-b16", action="store_true", help="with full_b1: skip the batch-16 companion measurement")
     ap.add_argument("--no-nvfp4", action="store_true", help="with full_b1: skip the NVFP4-expert companion")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--launch-list", action="store_true",
+                    help="for a profiler's launch list: after the warm-up run one bench step and stop; prints how "
+                         "many library launches came before it and how many it made")
     return ap.parse_args(argv)
 
 
@@ -450,6 +460,14 @@ def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clock
     for _ in range(warmup):
         one_step()
     m.dg_synchronize(h)
+    if args.launch_list:
+        before = m.dg_launch_count(h)
+        one_step()
+        m.dg_synchronize(h)
+        print(json.dumps({"launch_list": name, "launches_before_step": before,
+                          "launches_in_step": m.dg_launch_count(h) - before, "denoise_steps": steps_seen[-1]}))
+        h.close()
+        raise SystemExit(0)
 
     # the timed region: no profiling events, only the two bracketing events
     stream = torch.cuda.current_stream(dev)

@@ -331,9 +331,15 @@ int pick_ntile(int n_mtiles, int T, int num_sms) {
 // rows (32 .. DG_GROUPED_TILE), so a small item does not pay for a large box.
 // Larger items stream an expert's weights fewer times but leave fewer items
 // to spread over the SMs when the routing concentrates on a few experts.
+#ifndef DG_GROUPED_TILE_LARGE
+#define DG_GROUPED_TILE_LARGE 128   // rows of an expert work item when a pass has >= DG_LARGE_PASS tokens
+#endif
+#ifndef DG_LARGE_PASS
+#define DG_LARGE_PASS 2048
+#endif
 int grouped_tile(const dg_handle* H, int T) {
-  (void)T;
-  return H->bf16 ? DG_GROUPED_TILE : 64;
+  if (!H->bf16) return 64;
+  return T >= DG_LARGE_PASS ? DG_GROUPED_TILE_LARGE : DG_GROUPED_TILE;
 }
 
 // Pipeline shape of a tensor-core GEMM launch.  TMA throughput per CTA is
