@@ -519,12 +519,67 @@ void run_split(dg_handle* H, const CUtensorMap& a0, const CUtensorMap& a1, const
   run_tc(H, a0, a1, a2, b, g, nullptr, tma_out ? &to : nullptr);
 }
 
+// The split-K form on CTA pairs (k_gemm_tc2.cu): the token tile holds every
+// row (64 .. 256), a pair of SMs takes one 256-row weight tile, and K is split
+// into as many slices as keep every pair busy in one wave.  Each SM streams
+// 128 weight rows and half of the token tile per stage, a third less than a
+// single CTA on a 128-row tile, with two 64-column chunks per TMA instruction.
+#ifndef DG_DENSE_PAIR
+#define DG_DENSE_PAIR 1
+#endif
+#ifndef DG_PAIR_KSUB
+#define DG_PAIR_KSUB 2        // chunks per stage of the CTA-pair dense GEMM
+#endif
+SplitPlan pair_plan(int num_sms, int T, int n_out, int K, size_t cap_floats, int seg1, int seg2) {
+  SplitPlan p;
+  if (T < 1 || T > kDenseSplitRows || (size_t)T * n_out > cap_floats) return p;
+  if ((seg1 != INT_MAX && seg1 % 256) || (seg2 != INT_MAX && seg2 % 256)) return p;
+  p.ksub = DG_PAIR_KSUB;
+  p.ntile = 64;
+  while (p.ntile < T) p.ntile <<= 1;
+  const int nst = (K / 64 + p.ksub - 1) / p.ksub;
+  const int items = (n_out + 255) / 256;
+  p.split = 1;
+  while (p.split < kMaxDenseSplit && items * (p.split + 1) <= num_sms / 2 && (p.split + 1) * 2 <= nst &&
+         (size_t)(p.split + 1) * T * n_out <= cap_floats)
+    ++p.split;
+  return p;
+}
+
 // The layers' use of the split-K form: up to three weight maps stacked along
 // M (boundaries seg1, seg2), partials in H->kpart.  Returns the number of
 // slices, or 0 when the call does not take this form (nothing launched).
 int dense_gemm_part(dg_handle* H, int cls, const void* x, const WMap& a0, const WMap& a1, const WMap& a2, int seg1,
                     int seg2, int T, int n_out, int K) {
   if (!H->bf16 || !H->kpart) return 0;
+  if (DG_DENSE_PAIR) {
+    const SplitPlan q = pair_plan(H->num_sms, T, n_out, K, H->kpart_floats, seg1, seg2);
+    if (q.split >= 1) {
+      ProfScope ps(H, cls);
+      const CUtensorMap* b = bmap(H, x, K, H->T_max, q.ntile / 2, q.ksub);
+      TcGemm g{};
+      g.mode = 0;
+      g.M = n_out;
+      g.K = K;
+      g.T = T;
+      g.ntile = q.ntile;
+      g.seg1 = seg1;
+      g.seg2 = seg2;
+      g.epi = EPI_STORE_F32;
+      g.out = H->kpart;
+      g.ld_out = n_out;
+      g.err = H->d_err;
+      g.ksub = q.ksub;
+      g.ksplit = q.split;
+      g.split_stride = (size_t)T * n_out;
+      CUtensorMap to;
+      const bool tma_out = omap(H, H->kpart, n_out, T, q.split, n_out, &to);
+      if (!b || launch_gemm_tc_pair(pick(a0, q.ksub), pick(a1, q.ksub), pick(a2, q.ksub), *b, g, H->num_sms,
+                                    H->stream, tma_out ? &to : nullptr) != 0)
+        H->bad_launch = true;
+      return q.split;
+    }
+  }
   const SplitPlan p = split_plan(H->num_sms, T, n_out, K, H->kpart_floats);
   if (p.split < 1) return 0;
   ProfScope ps(H, cls);
@@ -1552,6 +1607,39 @@ int dg_selftest_gemm_split(dg_handle* H, const void* x, const void* w, int T, in
   H->launches += 1;
   *nsplit = p.split;
   return check_launch(H, "selftest split gemm");
+}
+
+int dg_selftest_gemm_pair(dg_handle* H, const void* x, const void* w, int T, int M, int K, int ntile, int ksplit,
+                          float* part) {
+  if (!H || !x || !w || !part || T < 1 || M < 1 || K < 64 || K % 64 || ksplit < 1 || ksplit > K / 64 ||
+      (ntile != 64 && ntile != 128 && ntile != 256))
+    return H ? fail(H, DG_EINVAL, "bad pair gemm args") : DG_EINVAL;
+  if (!H->bf16) return fail(H, DG_ESTATE, "needs a bf16 handle");
+  if (!aligned16(x) || !aligned16(w)) return fail(H, DG_EINVAL, "unaligned operands");
+  TcGemm g{};
+  g.mode = 0;
+  g.M = M;
+  g.K = K;
+  g.T = T;
+  g.ntile = ntile;
+  g.seg1 = g.seg2 = INT_MAX;
+  g.epi = EPI_STORE_F32;
+  g.out = part;
+  g.ld_out = M;
+  g.err = H->d_err;
+  g.ksplit = ksplit;
+  g.split_stride = (size_t)T * M;
+  g.ksub = DG_PAIR_KSUB;
+  while (g.ksub > 1 && ksplit > (K / 64 + g.ksub - 1) / g.ksub) g.ksub >>= 1;
+  CUtensorMap mx, mw, to;
+  if (!tmap_chunks(&mx, x, K, T, K, (uint32_t)(ntile / 2), (uint32_t)g.ksub) ||
+      !tmap_chunks(&mw, w, K, M, K, 128, (uint32_t)g.ksub))
+    return fail(H, DG_ECUDA, "tensor map encode failed");
+  const bool tma_out = tmap_out3d(&to, part, M, T, ksplit, M);
+  if (launch_gemm_tc_pair(mw, mw, mw, mx, g, H->num_sms, H->stream, tma_out ? &to : nullptr) != 0)
+    return fail(H, DG_EINVAL, "pair GEMM tiling rejected");
+  H->launches += 1;
+  return check_launch(H, "selftest pair gemm");
 }
 
 int dg_ar_step(dg_handle* H, int batch, const int* req, const int32_t* tokens, float* logits, int32_t* next_token) {

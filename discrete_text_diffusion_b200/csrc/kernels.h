@@ -176,6 +176,15 @@ int launch_gemm_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
                    const CUtensorMap* bsub, const TcGemm& p, int num_sms, cudaStream_t s,
                    const CUtensorMap* tout = nullptr);
 int gemm_tc_smem_bytes(const TcGemm& p, int* stages);
+// Dense mode (EPI_STORE_F32, split-K slices as launch_gemm_tc) on CTA pairs
+// (k_gemm_tc2.cu): 256-row weight tiles, each CTA of a pair holding 128 weight
+// rows and half of the token tile.  a0..a2: weight maps with boxes of 128 rows
+// by g.ksub (1, 2 or 4) 64-column chunks; b: token map with boxes of ntile/2
+// rows by g.ksub chunks;
+// tout: fp32 output map as for launch_gemm_tc, or NULL.  seg1 / seg2 must be
+// multiples of 256.  Returns -1 (nothing launched) for another shape.
+int launch_gemm_tc_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
+                        const TcGemm& g, int num_sms, cudaStream_t s, const CUtensorMap* tout);
 
 // NVFP4 grouped expert GEMMs (k_gemm_fp4.cu): modes 1 (gate/up + SwiGLU) and 2
 // (down + scatter) of the bf16 grouped GEMM, with the weights as E2M1 codes

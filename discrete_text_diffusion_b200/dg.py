@@ -23,7 +23,7 @@ EXPORTS = (
     "dg_create", "dg_destroy", "dg_last_error", "dg_prefill_prompt", "dg_set_kv", "dg_set_length",
     "dg_get_length", "dg_denoise_step", "dg_sample", "dg_generate_block", "dg_generate_block_host",
     "dg_synchronize", "dg_launch_count", "dg_profile_enable", "dg_profile_read", "dg_profile_reset",
-    "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc", "dg_selftest_gemm_split", "dg_get_kv",
+    "dg_selftest_philox", "dg_selftest_gemm", "dg_sample_noalloc", "dg_selftest_gemm_split", "dg_selftest_gemm_pair", "dg_get_kv",
     "dg_selftest_router", "dg_selftest_wait_timeout", "dg_ar_step", "dg_quantize_nvfp4",
 )
 
@@ -134,6 +134,7 @@ def lib():
         L.dg_selftest_philox.argtypes = [P, P, P, P, P, C.c_int]
         L.dg_selftest_gemm.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, P]
         L.dg_selftest_gemm_split.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, P, C.c_int, C.POINTER(C.c_int)]
+        L.dg_selftest_gemm_pair.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, P]
         L.dg_sample_noalloc.argtypes = [P, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_int), C.c_int,
                                         C.POINTER(DgSamplerParams), P, C.POINTER(DgStepOut), P, C.c_char_p,
                                         C.c_size_t]
@@ -401,6 +402,12 @@ def dg_selftest_router(h: Handle, logits, bias, k: int, tile: int, out: dict):
     T, E = logits.shape
     o = DgRouterOut(*[out[n].data_ptr() for n, _ in DgRouterOut._fields_])
     return h.check(lib().dg_selftest_router(h.ptr, _ptr(logits), _ptr(bias), T, E, k, tile, C.byref(o)))
+
+
+def dg_selftest_gemm_pair(h: Handle, x, w, part, ntile):
+    """x @ w.T on CTA pairs as part.shape[0] split-K fp32 slices part [ksplit, T, M]."""
+    return h.check(lib().dg_selftest_gemm_pair(h.ptr, _ptr(x), _ptr(w), x.shape[0], w.shape[0], x.shape[1], ntile,
+                                               part.shape[0], _ptr(part)))
 
 
 def dg_selftest_gemm_split(h: Handle, x, w, part):

@@ -443,6 +443,16 @@ int dg_selftest_gemm_split(dg_handle* h, const void* x, const void* w, int T, in
                            int max_split, int* nsplit);
 
 /*
+ * Test hook: the same split-K product on CTA pairs (two SMs compute one
+ * 256-row weight tile, each loading 128 weight rows and half of the token
+ * tile).  ksplit fp32 slices part[s][T][M] sum to x[T, K] * w[M, K]^T; ntile
+ * (token rows of a pair's tile) is 64, 128 or 256 and ksplit is in
+ * [1, K / 64].  Same operand rules as dg_selftest_gemm; DG_EINVAL otherwise.
+ */
+int dg_selftest_gemm_pair(dg_handle* h, const void* x, const void* w, int T, int M, int K, int ntile, int ksplit,
+                          float* part);
+
+/*
  * Test hook for the bounded device waits: one kernel waits on a shared-memory
  * barrier that nothing arrives on, gives up after limit_us microseconds of wall
  * time (1 .. 100000), records the timeout and returns.  The call synchronises
