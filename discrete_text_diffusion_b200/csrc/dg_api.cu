@@ -84,6 +84,20 @@ bool tmap_out3d(CUtensorMap* m, void* ptr, uint64_t cols, uint64_t rows, uint64_
             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// Split-attention partial outputs part_o as (256 columns, nq rows, planes):
+// boxes of 32 columns x 128 rows x 1 plane, 128-byte swizzle, rows past nq
+// clipped by the store.
+bool tmap_attn_part(CUtensorMap* m, void* ptr, uint64_t nq, uint64_t planes) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {256, nq, planes};
+  cuuint64_t strides[2] = {256 * 4, nq * 256 * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 // The same for n2 stacked matrices [n2][rows][cols]: dims (64, rows, cols/64, n2).
 bool tmap_chunks4(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t n2, uint32_t box_rows,
                   uint32_t nz) {
@@ -165,6 +179,11 @@ struct dg_handle {
   WMap m_embed{}, m_wsc{};
   std::vector<BMapEntry> bmaps;   // token-operand maps, built on first use
   std::vector<OMapEntry> omaps;   // fp32 output maps of the TMA-store epilogue, built on first use
+  struct PartMap {
+    int nq, planes;
+    CUtensorMap m;
+  };
+  std::vector<PartMap> part_maps;  // split-attention partial maps by (nq, planes)
   bool bad_launch = false;        // a tensor map or GEMM tiling was rejected
   // KV cache (owned)
   void* kc = nullptr;
@@ -198,7 +217,7 @@ struct dg_handle {
   // tensor-core attention (bf16, head dim 256)
   bool attn_tc = false;
   CUtensorMap m_q{};
-  std::vector<CUtensorMap> m_kc, m_vt;
+  std::vector<CUtensorMap> m_kc, m_vt, m_vt2;   // m_vt: boxes of 64 keys x 256 dims; m_vt2: x 128 dims
   float* part_o = nullptr;
   float* part_ml = nullptr;
   size_t part_rows_cap = 0;   // split-rows capacity of part_o / part_ml
@@ -750,6 +769,9 @@ void moe_gemms(dg_handle* H, int l, int T) {
   }
 }
 
+#ifndef DG_ATTN_PAIR
+#define DG_ATTN_PAIR 1
+#endif
 void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
   const dg_config& c = H->c;
   AttnArgs a{};
@@ -771,13 +793,17 @@ void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
     return;
   }
   if (H->attn_tc) {
+    // Query heads 2y and 2y+1 on one CTA pair when they read the same KV head
+    // (128-key tiles); otherwise one CTA per head (64-key tiles).
+    const bool pair = DG_ATTN_PAIR && attn_tc2_supported(c.n_heads, c.n_kv_heads, c.head_dim);
+    const int ktile = pair ? 128 : 64;
     // Split the keys: one CTA per SM, so the time is about waves x (key tiles
     // per CTA + a fixed cost of ~2 tiles); each split adds partial-output
     // traffic and combine work (charged half a tile).
     int max_len = 0;
     for (int b = 0; b < bi.B; ++b) max_len = std::max(max_len, bi.len[b] + nq);
     const int base = bi.B * c.n_heads * ((nq + 127) / 128);
-    const int tiles = (max_len + 63) / 64;
+    const int tiles = (max_len + ktile - 1) / ktile;
     int n_split = 1;
     double best = 1e30;
     for (int n = 1; n <= std::min(16, std::max(1, tiles / 4)); ++n) {
@@ -797,7 +823,27 @@ void attention(dg_handle* H, int l, const BatchInfo& bi, int nq, bool causal) {
     t.nq_pad = nq;
     t.err = H->d_err;
     ProfScope ps(H, PC_ATTN, n_split > 1 ? 2 : 1);
-    launch_attn_tc(H->m_q, H->m_kc[l], H->m_vt[l], (__nv_bfloat16*)H->attn, t, H->stream);
+    if (pair) {
+      const CUtensorMap* tpo = nullptr;
+      if (n_split > 1) {
+        const int planes = n_split * bi.B * c.n_heads;
+        for (const auto& e : H->part_maps)
+          if (e.nq == nq && e.planes == planes) tpo = &e.m;
+        if (!tpo) {
+          dg_handle::PartMap e;
+          e.nq = nq;
+          e.planes = planes;
+          if (tmap_attn_part(&e.m, H->part_o, (uint64_t)nq, (uint64_t)planes)) {
+            if (H->part_maps.size() >= 16) H->part_maps.clear();
+            H->part_maps.push_back(e);
+            tpo = &H->part_maps.back().m;
+          }
+        }
+      }
+      launch_attn_tc2(H->m_q, H->m_kc[l], H->m_vt2[l], tpo, (__nv_bfloat16*)H->attn, t, H->stream);
+    }
+    else
+      launch_attn_tc(H->m_q, H->m_kc[l], H->m_vt[l], (__nv_bfloat16*)H->attn, t, H->stream);
     return;
   }
   ProfScope ps(H, PC_ATTN);
@@ -1256,10 +1302,12 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* stream, dg_handle
         tm &= tmap_chunks(&H->m_q, H->q, hd, (uint64_t)T * c.n_heads, hd, 128, 4);
         H->m_kc.resize(c.n_layers);
         H->m_vt.resize(c.n_layers);
+        H->m_vt2.resize(c.n_layers);
         const uint64_t kv_rows = (uint64_t)c.max_batch * c.n_kv_heads;
         for (int l = 0; l < c.n_layers; ++l) {
           tm &= tmap_chunks(&H->m_kc[l], kc_layer(H, l), hd, kv_rows * c.max_ctx, hd, 64, 4);
           tm &= tmap_2d(&H->m_vt[l], vt_layer(H, l), (uint64_t)c.max_ctx, kv_rows * hd, (uint64_t)c.max_ctx, 256);
+          tm &= tmap_2d(&H->m_vt2[l], vt_layer(H, l), (uint64_t)c.max_ctx, kv_rows * hd, (uint64_t)c.max_ctx, 128);
         }
       }
       if (!tm) {

@@ -193,10 +193,14 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // the set-up above touches no global memory: it overlaps the previous kernel
-  pdl_wait();
+  // The set-up above touches no global memory: it overlaps the previous
+  // kernel.  So does the dense producer's first weight boxes (below): dense
+  // weights are never written by the launch just before this one.
+  const bool prefetch_a = g.mode == 0;
+  if (!(prefetch_a && warp == 0 && lane == 0)) pdl_wait();
   pdl_trigger();
 
+  // (the prefetching producer has not waited yet; mode 0 reads no n_work)
   const int total = (g.mode == 0) ? P.n_mtiles * P.n_ttiles * (g.ksplit > 1 ? g.ksplit : 1)
                                   : (*g.n_work) * P.n_mtiles;
   const int nk = g.K / kBK;                       // 64-wide K blocks
@@ -212,6 +216,29 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     // the token map a (64, rows, K/64) view with a box of ntile rows x ksub
     // chunks.  A stage always receives whole boxes (chunks past K, rows past
     // the matrix are zero-filled), so the byte count is fixed.
+    // Dense mode: the weight boxes of the first item's first stages go out
+    // before waiting for the previous launch (the ring is empty, so those
+    // stages are free); the token boxes follow once it has finished.
+    int pre = 0;
+    if (prefetch_a) {
+      if ((int)blockIdx.x < total) {
+        int m0, e, row0, rows, j0, j1, ks;
+        tc_item(P, blockIdx.x, nst, m0, e, row0, rows, j0, j1, ks);
+        int lvl;
+        const int box = item_box(P, rows, &lvl);
+        const uint32_t tx = (uint32_t)(ksub * (kABytes + box * kBK * 2));
+        const CUtensorMap* am = &ta0;
+        int am0 = m0;
+        if (m0 >= g.seg2) { am = &ta2; am0 = m0 - g.seg2; }
+        else if (m0 >= g.seg1) { am = &ta1; am0 = m0 - g.seg1; }
+        pre = min(P.stages, j1 - j0);
+        for (int i = 0; i < pre; ++i) {
+          mbar_expect_tx(&full[i], tx);
+          tma_load_3d(stage0 + (size_t)i * P.stage_bytes, am, &full[i], 0, am0, (j0 + i) * ksub);
+        }
+      }
+      pdl_wait();
+    }
     uint32_t kiter = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
       int m0, e, row0, rows, j0, j1, ks;
@@ -230,9 +257,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       for (int j = j0; j < j1; ++j, ++kiter) {
         const int s = kiter % P.stages;
         const uint32_t ph = (kiter / P.stages) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
         const int kb0 = j * ksub;
         uint8_t* st = stage0 + (size_t)s * P.stage_bytes;
+        if (kiter < (uint32_t)pre) {   // weight box already in flight
+          tma_load_3d(st + n_a * ksub * kABytes, bm, &full[s], 0, row0, kb0);
+          continue;
+        }
+        if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
         mbar_expect_tx(&full[s], tx);
         if (g.mode == 0) {
           tma_load_3d(st, am, &full[s], 0, am0, kb0);
@@ -480,7 +511,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);
     }
-    if (tstore && te == 0) bulk_wait_all();
+    if (tstore && te == 0) bulk_wait_read_all();
   }
   tc_fence_before();
   __syncthreads();

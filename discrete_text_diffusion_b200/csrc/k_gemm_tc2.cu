@@ -25,6 +25,7 @@
 #include <algorithm>
 
 #include "dg_common.cuh"
+#include "dg_pair.cuh"
 #include "kernels.h"
 
 namespace dg {
@@ -52,61 +53,6 @@ struct PairParams {
   int stages, stage_bytes, acc_cols, n_acc_buf, tmem_cols, n_mpairs, n_ttiles;
   int tma_out, vec;
 };
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// shared::cluster address of the same shared variable in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
-  return a;
-}
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
-}
-// TMA load into this CTA's shared memory, completing on a barrier of either CTA of the pair
-__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
-                                                 int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_alloc2(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish2() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void umma2_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// arrive on the barrier at this offset in both CTAs of the pair once the MMAs
-// issued so far complete: one commit per CTA's barrier
-__device__ __forceinline__ void umma2_commit_to(uint32_t bar_cluster) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
-               : "memory");
-}
-__device__ __forceinline__ void umma2_commit_both(uint64_t* bar) {
-  umma2_commit_to(smem_u32(bar));
-  umma2_commit_to(map_to_rank(bar, 1));
-}
 
 __device__ __forceinline__ void pair_item(const PairParams& P, int item, int nst, int rank, int& m0, int& row0,
                                           int& rows_pair, int& j0, int& j1, int& ks) {
@@ -161,7 +107,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
   cluster_sync_all();     // both CTAs' barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
+  // the producer waits for the previous launch only after its first weight boxes
+  if (!(warp == 0 && lane == 0)) pdl_wait();
   pdl_trigger();
 
   const int n_items = P.n_mpairs * P.n_ttiles * (P.ksplit > 1 ? P.ksplit : 1);
@@ -174,23 +121,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
+    // The weights are never written by the launch just before this one: the
+    // first item's first stages (free, the ring is empty) receive their
+    // weight boxes before the wait for that launch; the token boxes after it.
+    auto weight_map = [&](int m0, int& am0) -> const CUtensorMap* {
+      const int mp0 = m0 - (int)rank * kPM;
+      if (mp0 >= P.seg2) { am0 = m0 - P.seg2; return &ta2; }
+      if (mp0 >= P.seg1) { am0 = m0 - P.seg1; return &ta1; }
+      am0 = m0;
+      return &ta0;
+    };
+    int pre = 0;
+    if (cid < n_items) {
+      int m0, row0, rows_pair, j0, j1, ks, am0;
+      pair_item(P, cid, nst, (int)rank, m0, row0, rows_pair, j0, j1, ks);
+      const CUtensorMap* am = weight_map(m0, am0);
+      pre = min(P.stages, j1 - j0);
+      for (int i = 0; i < pre; ++i) {
+        if (leader) mbar_expect_tx(&full[i], 2u * (a_bytes + b_bytes));
+        tma_load_3d_pair(stage0 + (size_t)i * P.stage_bytes, am, map_to_rank(&full[i], 0), 0, am0,
+                         (j0 + i) * P.ksub);
+      }
+    }
+    pdl_wait();
     uint32_t kiter = 0;
     bool ok = true;
     for (int item = cid; item < n_items && ok; item += n_clusters) {
-      int m0, row0, rows_pair, j0, j1, ks;
+      int m0, row0, rows_pair, j0, j1, ks, am0;
       pair_item(P, item, nst, (int)rank, m0, row0, rows_pair, j0, j1, ks);
-      const CUtensorMap* am = &ta0;
-      int am0 = m0;
-      if (m0 - (int)rank * kPM >= P.seg2) { am = &ta2; am0 = m0 - P.seg2; }
-      else if (m0 - (int)rank * kPM >= P.seg1) { am = &ta1; am0 = m0 - P.seg1; }
+      const CUtensorMap* am = weight_map(m0, am0);
       for (int j = j0; j < j1; ++j, ++kiter) {
         const int s = kiter % P.stages;
         const uint32_t ph = (kiter / P.stages) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
         uint8_t* st = stage0 + (size_t)s * P.stage_bytes;
         const uint32_t fb = map_to_rank(&full[s], 0);   // the leader's barrier counts both CTAs' bytes
-        if (leader) mbar_expect_tx(&full[s], 2u * (a_bytes + b_bytes));
-        tma_load_3d_pair(st, am, fb, 0, am0, j * P.ksub);
+        if (kiter >= (uint32_t)pre) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, err, kErrTimeoutTma)) { ok = false; break; }
+          if (leader) mbar_expect_tx(&full[s], 2u * (a_bytes + b_bytes));
+          tma_load_3d_pair(st, am, fb, 0, am0, j * P.ksub);
+        }
         tma_load_3d_pair(st + a_bytes, &tb, fb, 0, row0, j * P.ksub);
       }
     }
@@ -284,7 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       tc_fence_before();
       mbar_arrive_cluster(empty_bar + (uint32_t)(ab * sizeof(uint64_t)));
     }
-    if (P.tma_out && te == 0) bulk_wait_all();
+    if (P.tma_out && te == 0) bulk_wait_read_all();
   }
   tc_fence_before();
   __syncthreads();

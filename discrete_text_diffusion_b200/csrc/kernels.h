@@ -234,6 +234,15 @@ struct AttnTcArgs {
 void launch_attn_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     __nv_bfloat16* out, const AttnTcArgs& a, cudaStream_t s);
 size_t attn_tc_partial_floats(int n_split, int B, int hq, int nq_pad, int hd);
+// The same on CTA pairs (k_attn_tc2.cu): query heads 2y and 2y+1 (one KV head)
+// share every K/V byte, 128-key tiles.  tv: V^T map with boxes of 64 keys x
+// 128 dims.  Needs hd == 256 and an even number of query heads per KV head
+// (attn_tc2_supported).  Same partial layout and combine as launch_attn_tc.
+// tpo (or NULL: plain stores): fp32 map over part_o as (256 columns, nq rows,
+// n_split * B * Hq planes) with boxes of 32 x 128 x 1 and 128-byte swizzle.
+bool attn_tc2_supported(int hq, int hkv, int hd);
+void launch_attn_tc2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap* tpo,
+                     __nv_bfloat16* out, const AttnTcArgs& a, cudaStream_t s);
 // Merge KV-split partials (unnormalised O [split][B*Hq*nq][256], (max log2, sum)) into
 // out [B*nq, Hq*256] bf16.
 void launch_attn_combine(const float* part_o, const float* part_ml, __nv_bfloat16* out, int n_split, int B, int hq,
