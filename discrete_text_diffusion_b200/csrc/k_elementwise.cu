@@ -228,15 +228,29 @@ __global__ void __launch_bounds__(kRowThreadsMax) add_rmsnorm_kernel(float* __re
       const int j = threadIdx.x + u * blockDim.x;
       v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j < d4) {
-        float4 a = p4[j];
-        for (int sp0 = 1; sp0 < nsplit; sp0 += 4) {
-          float4 b[4];
+        float4 a;
+        if (VPT == 1 && nsplit <= 8) {
+          // every load of the column in flight at once: one memory latency per row
+          // (one column per thread: wider rows would spill the 8 slices)
+          float4 b[8];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (sp0 + q < nsplit) b[q] = p4[(size_t)(sp0 + q) * s4 + j];
+          for (int q = 0; q < 8; ++q)
+            if (q < nsplit) b[q] = p4[(size_t)q * s4 + j];
+          a = b[0];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (sp0 + q < nsplit) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
+          for (int q = 1; q < 8; ++q)
+            if (q < nsplit) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
+        } else {
+          a = p4[j];
+          for (int sp0 = 1; sp0 < nsplit; sp0 += 4) {
+            float4 b[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (sp0 + q < nsplit) b[q] = p4[(size_t)(sp0 + q) * s4 + j];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (sp0 + q < nsplit) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
+          }
         }
         float4 x = h4[j];
         x.x += a.x; x.y += a.y; x.z += a.z; x.w += a.w;
@@ -354,38 +368,71 @@ __global__ void __launch_bounds__(kRowThreadsMax) combine_reg_kernel(float* __re
   __shared__ float red[32];
   __shared__ float ws[16];
   const int t = blockIdx.x, d4 = d >> 2;
-  if (threadIdx.x < k) ws[threadIdx.x] = wts[(size_t)t * k + threadIdx.x];
-  __syncthreads();
   float4* h4 = reinterpret_cast<float4*>(h + (size_t)t * d);
   const T* yt = y + (size_t)t * k * d;
   float4 v[VPT];
   float ss = 0.f;
+  if (VPT == 1 && k <= 8) {
+    // the slot weights and every slot row of a column in flight at once: one
+    // memory latency per row (the sums keep slot order; one column per thread)
+    float c[8];
 #pragma unroll
-  for (int u = 0; u < VPT; ++u) {
-    const int j = threadIdx.x + u * blockDim.x;
-    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < d4) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < k; s0 += 4) {
-        float4 yv[4];
+    for (int q = 0; q < 8; ++q) c[q] = q < k ? wts[(size_t)t * k + q] : 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (s0 + q < k) yv[q] = load4<T>(yt, (size_t)(s0 + q) * d4 + j);
+    for (int u = 0; u < VPT; ++u) {
+      const int j = threadIdx.x + u * blockDim.x;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < d4) {
+        float4 yv[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (s0 + q < k) {
-            const float c = ws[s0 + q];
-            acc.x += c * yv[q].x;
-            acc.y += c * yv[q].y;
-            acc.z += c * yv[q].z;
-            acc.w += c * yv[q].w;
+        for (int q = 0; q < 8; ++q)
+          if (q < k) yv[q] = load4<T>(yt, (size_t)q * d4 + j);
+        float4 x = h4[j];
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < k) {
+            acc.x += c[q] * yv[q].x;
+            acc.y += c[q] * yv[q].y;
+            acc.z += c[q] * yv[q].z;
+            acc.w += c[q] * yv[q].w;
           }
+        x.x += acc.x; x.y += acc.y; x.z += acc.z; x.w += acc.w;
+        h4[j] = x;
+        v[u] = x;
+        ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
       }
-      float4 x = h4[j];
-      x.x += acc.x; x.y += acc.y; x.z += acc.z; x.w += acc.w;
-      h4[j] = x;
-      v[u] = x;
-      ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+    }
+  } else {
+    if (threadIdx.x < k) ws[threadIdx.x] = wts[(size_t)t * k + threadIdx.x];
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      const int j = threadIdx.x + u * blockDim.x;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < d4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < k; s0 += 4) {
+          float4 yv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (s0 + q < k) yv[q] = load4<T>(yt, (size_t)(s0 + q) * d4 + j);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (s0 + q < k) {
+              const float c = ws[s0 + q];
+              acc.x += c * yv[q].x;
+              acc.y += c * yv[q].y;
+              acc.z += c * yv[q].z;
+              acc.w += c * yv[q].w;
+            }
+        }
+        float4 x = h4[j];
+        x.x += acc.x; x.y += acc.y; x.z += acc.z; x.w += acc.w;
+        h4[j] = x;
+        v[u] = x;
+        ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+      }
     }
   }
   if (norm_w == nullptr) return;
@@ -471,7 +518,10 @@ __global__ void rope_scatter_kernel(const float* __restrict__ qkv, int nsplit, s
 // lane = token, so consecutive lanes store consecutive cache positions.
 constexpr int kRopeTok = 32;
 
-template <typename T>
+// NS = 1 or 2: exactly NS split-K slices and hd <= 256, so a thread's items
+// (at most 4 rotated groups, or 8 V vectors) are all loaded before any is
+// used: one memory latency per CTA.  NS = 0: any slice count, item by item.
+template <typename T, int NS>
 __global__ void __launch_bounds__(256) rope_scatter_tiled_kernel(const float* __restrict__ qkv, int nsplit,
                                                                  size_t split_stride, T* __restrict__ q,
                                                                  T* __restrict__ kc, T* __restrict__ vt,
@@ -486,6 +536,95 @@ __global__ void __launch_bounds__(256) rope_scatter_tiled_kernel(const float* __
   const int half = hd >> 1, g4 = half >> 2;
   const size_t ncol = (size_t)(hq + 2 * hkv) * hd;
   const int ntk = min(kRopeTok, n_tok - t0);
+  if constexpr (NS > 0) {
+    if (head < hq + hkv) {
+      constexpr int kIt = 4;   // kRopeTok * 256 / 8 groups over 256 threads
+      float4 x1[kIt], x2[kIt], a1[kIt], a2[kIt], ca[kIt], cb[kIt];
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) {
+        const int idx = threadIdx.x + it * blockDim.x;
+        if (idx < ntk * g4) {
+          const int tt = idx / g4, j = (idx - tt * g4) * 4;
+          const int t = t0 + tt;
+          const int b = t / nq, pos = bi.len[b] + (t - b * nq);
+          const float* src = qkv + (size_t)t * ncol + (size_t)head * hd;
+          x1[it] = *reinterpret_cast<const float4*>(src + j);
+          x2[it] = *reinterpret_cast<const float4*>(src + half + j);
+          if (NS == 2) {
+            a1[it] = *reinterpret_cast<const float4*>(src + split_stride + j);
+            a2[it] = *reinterpret_cast<const float4*>(src + split_stride + half + j);
+          }
+          const float4* cs4 = reinterpret_cast<const float4*>(rope_cs + (size_t)pos * half + j);
+          ca[it] = cs4[0];
+          cb[it] = cs4[1];
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) {
+        const int idx = threadIdx.x + it * blockDim.x;
+        if (idx < ntk * g4) {
+          const int tt = idx / g4, jg = idx - tt * g4;
+          const int t = t0 + tt;
+          const int b = t / nq, i = t - b * nq;
+          const int pos = bi.len[b] + i;
+          float4 u1 = x1[it], u2 = x2[it];
+          if (NS == 2) {
+            u1.x += a1[it].x; u1.y += a1[it].y; u1.z += a1[it].z; u1.w += a1[it].w;
+            u2.x += a2[it].x; u2.y += a2[it].y; u2.z += a2[it].z; u2.w += a2[it].w;
+          }
+          const float4 c0 = ca[it], c1 = cb[it];  // (cos, sin) of pairs j, j+1 | j+2, j+3
+          const float4 r1 = make_float4(u1.x * c0.x - u2.x * c0.y, u1.y * c0.z - u2.y * c0.w,
+                                        u1.z * c1.x - u2.z * c1.y, u1.w * c1.z - u2.w * c1.w);
+          const float4 r2 = make_float4(u2.x * c0.x + u1.x * c0.y, u2.y * c0.z + u1.y * c0.w,
+                                        u2.z * c1.x + u1.z * c1.y, u2.w * c1.z + u1.w * c1.w);
+          T* dst = head < hq ? q + (((size_t)b * hq + head) * nq + i) * hd
+                             : kc + (((size_t)bi.slot[b] * hkv + (head - hq)) * max_ctx + pos) * hd;
+          store4<T>(dst, jg, r1);
+          store4<T>(dst + half, jg, r2);
+        }
+      }
+      return;
+    }
+    T* tile = reinterpret_cast<T*>(rope_smem);
+    const int ld = hd + 2;
+    const int d4n = hd >> 2;
+    constexpr int kItV = 8;   // kRopeTok * 256 / 4 vectors over 256 threads
+    float4 xv[kItV], av[kItV];
+#pragma unroll
+    for (int it = 0; it < kItV; ++it) {
+      const int idx = threadIdx.x + it * blockDim.x;
+      if (idx < ntk * d4n) {
+        const int tt = idx / d4n, jj = (idx - tt * d4n) * 4;
+        const float* src = qkv + (size_t)(t0 + tt) * ncol + (size_t)head * hd + jj;
+        xv[it] = *reinterpret_cast<const float4*>(src);
+        if (NS == 2) av[it] = *reinterpret_cast<const float4*>(src + split_stride);
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < kItV; ++it) {
+      const int idx = threadIdx.x + it * blockDim.x;
+      if (idx < ntk * d4n) {
+        const int tt = idx / d4n, jj = (idx - tt * d4n) * 4;
+        float4 x = xv[it];
+        if (NS == 2) { x.x += av[it].x; x.y += av[it].y; x.z += av[it].z; x.w += av[it].w; }
+        T* r = tile + tt * ld + jj;
+        r[0] = from_f32<T>(x.x);
+        r[1] = from_f32<T>(x.y);
+        r[2] = from_f32<T>(x.z);
+        r[3] = from_f32<T>(x.w);
+      }
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    if (lane < ntk) {
+      const int t = t0 + lane;
+      const int b = t / nq, i = t - b * nq;
+      const int pos = bi.len[b] + i;
+      T* col = vt + ((size_t)bi.slot[b] * hkv + (head - hq - hkv)) * hd * (size_t)max_ctx + pos;
+      for (int dd = w; dd < hd; dd += nw) col[(size_t)dd * max_ctx] = tile[lane * ld + dd];
+    }
+    return;
+  }
   if (head < hq + hkv) {
     for (int idx = threadIdx.x; idx < ntk * g4; idx += blockDim.x) {
       const int tt = idx / g4, jg = idx - tt * g4, j = jg * 4;
@@ -555,9 +694,16 @@ void launch_rope_scatter(const float* qkv, int nsplit, size_t split_stride, T* q
   if (hd % 8 == 0) {
     dim3 grid((n_tok + kRopeTok - 1) / kRopeTok, hq + 2 * hkv);
     const size_t smem = (size_t)kRopeTok * (hd + 2) * sizeof(T);
-    launch_k(rope_scatter_tiled_kernel<T>, dim3(grid), dim3(256), smem, s, qkv, nsplit, split_stride, q, kc, vt,
-                                                         reinterpret_cast<const float2*>(rope_cs), bi, nq, n_tok,
-                                                         hq, hkv, hd, max_ctx);
+    const float2* cs = reinterpret_cast<const float2*>(rope_cs);
+    if (hd <= 256 && nsplit == 1)
+      launch_k(rope_scatter_tiled_kernel<T, 1>, dim3(grid), dim3(256), smem, s, qkv, nsplit, split_stride, q, kc,
+               vt, cs, bi, nq, n_tok, hq, hkv, hd, max_ctx);
+    else if (hd <= 256 && nsplit == 2)
+      launch_k(rope_scatter_tiled_kernel<T, 2>, dim3(grid), dim3(256), smem, s, qkv, nsplit, split_stride, q, kc,
+               vt, cs, bi, nq, n_tok, hq, hkv, hd, max_ctx);
+    else
+      launch_k(rope_scatter_tiled_kernel<T, 0>, dim3(grid), dim3(256), smem, s, qkv, nsplit, split_stride, q, kc,
+               vt, cs, bi, nq, n_tok, hq, hkv, hd, max_ctx);
     return;
   }
   dim3 grid(n_tok, hq + 2 * hkv);
@@ -578,7 +724,16 @@ __global__ void gather_rows_kernel(const T* __restrict__ xn, const int32_t* __re
     const int nv = d * (int)sizeof(T) / 16;
     const uint4* s4 = reinterpret_cast<const uint4*>(xn + (size_t)src * d);
     uint4* d4 = reinterpret_cast<uint4*>(xp + (size_t)p * d);
-    for (int j = threadIdx.x; j < nv; j += blockDim.x) d4[j] = s4[j];
+    // four vectors per thread in flight before the first store
+    for (int j0 = threadIdx.x; j0 < nv; j0 += 4 * blockDim.x) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (j0 + u * (int)blockDim.x < nv) r[u] = s4[j0 + u * blockDim.x];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (j0 + u * (int)blockDim.x < nv) d4[j0 + u * blockDim.x] = r[u];
+    }
   } else {
     for (int j = threadIdx.x; j < d; j += blockDim.x) xp[(size_t)p * d + j] = xn[(size_t)src * d + j];
   }
