@@ -46,8 +46,8 @@ CSRC = os.path.join(ROOT, "discrete_text_diffusion_b200", "csrc")
 # the source file and the sha256 prefix of that file when it was captured.  A
 # class whose source has changed since reports traffic null.
 NCU_TRAFFIC = {
-    # canvas-step attention over an 8192-position cache (16/8 heads of 256): the bench's launch shape
-    "attention": (71365376 + 2604032, "k_attn_tc.cu", "5e28d2db74c28ed9"),
+    # canvas-step attention over an 8192-position cache (16/8 heads of 256, CTA pairs): the bench's launch shape
+    "attention": (71362304 + 3758080, "k_attn_tc2.cu", "c6dffe33dab64a07"),
     # LM head with the sampler statistics, 256 tokens x 262144 vocabulary: the bench's launch shape
     "lm_head": (1488360960 + 33390336, "k_gemm_tc.cu", "b6966e2537710892"),
     # the fused sampler pass over 256 rows: the bench's launch shape
@@ -320,7 +320,9 @@ def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, pe
 
     if "attention" in breakdown:
         nl, _ = breakdown["attention"]
-        add("attention", "attn_tc_kernel (+ split combine)", "tensor", attention_flops(model, batch, canvas, blocks) / nl)
+        pair = model["n_heads"] % (2 * model["n_kv_heads"]) == 0
+        add("attention", ("attn_tc2_kernel (CTA pairs" if pair else "attn_tc_kernel (") + ", + split combine)", "tensor",
+            attention_flops(model, batch, canvas, blocks) / nl)
     if batch == 1:
         wb = expert_bytes / 2.0      # the weight terms of the byte counts scale with the storage
         up_b = moe_up_bytes(model, rows, touched) - touched * 2 * F * d * 2 * (1 - wb)
@@ -337,10 +339,13 @@ def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, pe
         nl, _ = breakdown["dense_gemm"]
         wts = passes * L * ((hq + 2 * hkv) * hd * d + d * hq * hd) + (steps - len(blocks)) * d * d
         byt, fl = wts * 2.0, 2.0 * wts * T
+        # up to 256 tokens: the split-K form on CTA pairs; more: one CTA per 128-row tile
+        kern = "gemm_tc2_kernel (split-K QKV / O / self-cond, CTA pairs)" if T <= 256 else \
+            "gemm_tc_kernel (QKV / O / self-cond)"
         if fl / (tfs * 1e12) > byt / (hbm * 1e9):
-            add("dense_gemm", "gemm_tc_kernel (QKV / O / self-cond)", "tensor", fl / nl)
+            add("dense_gemm", kern, "tensor", fl / nl)
         else:
-            add("dense_gemm", "gemm_tc_kernel (split-K QKV / O / self-cond)", "hbm", byt / nl)
+            add("dense_gemm", kern, "hbm", byt / nl)
     # the block loop runs the fused head: the LM head writes 16-byte statistics per token and
     # 32-entry vocabulary group instead of logits; the sampler reads them and recomputes one group
     groups = (V + 31) // 32

@@ -697,6 +697,51 @@ void moe_gemms_fp4(dg_handle* H, int l, int T) {
   }
 }
 
+// The grouped GEMMs on CTA pairs (k_moe_tc2.cu): each SM streams 128 weight
+// rows and half of an item's token rows.
+#ifndef DG_MOE_PAIR
+#define DG_MOE_PAIR 1              // bit 0: gate/up on pairs, bit 1: down on pairs (passes below DG_LARGE_PASS)
+#endif
+#ifndef DG_MOE_PAIR_UP_KSUB
+#define DG_MOE_PAIR_UP_KSUB 1      // chunks per stage, gate/up (two weight operands)
+#endif
+#ifndef DG_MOE_PAIR_DOWN_KSUB
+#define DG_MOE_PAIR_DOWN_KSUB 2    // chunks per stage, down
+#endif
+// One part (1: gate/up, 2: down) on pairs; false when that part is not run
+// this way (nothing launched).
+bool moe_gemm_pair(dg_handle* H, int l, int T, int part) {
+  const dg_config& c = H->c;
+  const int tile = grouped_tile(H, T);
+  if (!H->bf16 || tile > 128 || T >= DG_LARGE_PASS || !(DG_MOE_PAIR & part)) return false;
+  const int n_work_max = c.n_experts + (T * c.top_k + tile - 1) / tile;
+  const uint64_t rows = (uint64_t)H->T_max * c.top_k;
+  const LayerMaps& M = H->lmaps[l];
+  TcGemm g{};
+  g.ntile = tile;
+  g.work = H->work;
+  g.n_work = H->n_work;
+  g.n_work_max = n_work_max;
+  g.err = H->d_err;
+  const void* x = part == 1 ? H->xp : H->hb;
+  const uint64_t kdim = part == 1 ? c.d_model : c.d_ff;
+  g.mode = part;
+  g.M = part == 1 ? c.d_ff : c.d_model;
+  g.K = (int)kdim;
+  g.out = part == 1 ? H->hb : H->y;
+  g.ld_out = g.M;
+  g.row_map = part == 1 ? nullptr : H->perm;
+  g.ksub = part == 1 ? DG_MOE_PAIR_UP_KSUB : DG_MOE_PAIR_DOWN_KSUB;
+  const CUtensorMap* b16 = bmap(H, x, kdim, rows, 16, g.ksub);
+  const CUtensorMap* b32 = bmap(H, x, kdim, rows, 32, g.ksub);
+  const CUtensorMap* b64 = bmap(H, x, kdim, rows, 64, g.ksub);
+  const CUtensorMap& a0 = pick(part == 1 ? M.gate : M.down, g.ksub);
+  const CUtensorMap& a1 = pick(part == 1 ? M.up : M.down, g.ksub);
+  if (!b16 || !b32 || !b64 || launch_gemm_tc2_grouped(a0, a1, *b16, *b32, *b64, g, H->num_sms, H->stream) != 0)
+    H->bad_launch = true;
+  return true;
+}
+
 void moe_gemms(dg_handle* H, int l, int T) {
   if (H->fp4) {
     moe_gemms_fp4(H, l, T);
@@ -709,7 +754,8 @@ void moe_gemms(dg_handle* H, int l, int T) {
   const uint64_t rows = (uint64_t)H->T_max * c.top_k;
   {
     ProfScope ps(H, PC_MOE_UP);
-    if (!H->bf16) {
+    if (moe_gemm_pair(H, l, T, 1)) {
+    } else if (!H->bf16) {
       launch_grouped_simt<float>((const float*)H->xp, (const float*)L.w_gate, (const float*)L.w_up, c.d_ff,
                                  c.d_model, H->work, H->n_work, n_work_max, H->perm, true, H->hb, c.d_ff, H->stream);
     } else {
@@ -739,7 +785,8 @@ void moe_gemms(dg_handle* H, int l, int T) {
   }
   {
     ProfScope ps(H, PC_MOE_DOWN);
-    if (!H->bf16) {
+    if (moe_gemm_pair(H, l, T, 2)) {
+    } else if (!H->bf16) {
       launch_grouped_simt<float>((const float*)H->hb, (const float*)L.w_down, nullptr, c.d_model, c.d_ff, H->work,
                                  H->n_work, n_work_max, H->perm, false, H->y, c.d_model, H->stream);
     } else {

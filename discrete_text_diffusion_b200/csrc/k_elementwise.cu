@@ -228,29 +228,15 @@ __global__ void __launch_bounds__(kRowThreadsMax) add_rmsnorm_kernel(float* __re
       const int j = threadIdx.x + u * blockDim.x;
       v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j < d4) {
-        float4 a;
-        if (VPT == 1 && nsplit <= 8) {
-          // every load of the column in flight at once: one memory latency per row
-          // (one column per thread: wider rows would spill the 8 slices)
-          float4 b[8];
+        float4 a = p4[j];
+        for (int sp0 = 1; sp0 < nsplit; sp0 += 4) {
+          float4 b[4];
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (q < nsplit) b[q] = p4[(size_t)q * s4 + j];
-          a = b[0];
+          for (int q = 0; q < 4; ++q)
+            if (sp0 + q < nsplit) b[q] = p4[(size_t)(sp0 + q) * s4 + j];
 #pragma unroll
-          for (int q = 1; q < 8; ++q)
-            if (q < nsplit) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
-        } else {
-          a = p4[j];
-          for (int sp0 = 1; sp0 < nsplit; sp0 += 4) {
-            float4 b[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (sp0 + q < nsplit) b[q] = p4[(size_t)(sp0 + q) * s4 + j];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (sp0 + q < nsplit) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
-          }
+          for (int q = 0; q < 4; ++q)
+            if (sp0 + q < nsplit) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
         }
         float4 x = h4[j];
         x.x += a.x; x.y += a.y; x.z += a.z; x.w += a.w;
@@ -368,71 +354,38 @@ __global__ void __launch_bounds__(kRowThreadsMax) combine_reg_kernel(float* __re
   __shared__ float red[32];
   __shared__ float ws[16];
   const int t = blockIdx.x, d4 = d >> 2;
+  if (threadIdx.x < k) ws[threadIdx.x] = wts[(size_t)t * k + threadIdx.x];
+  __syncthreads();
   float4* h4 = reinterpret_cast<float4*>(h + (size_t)t * d);
   const T* yt = y + (size_t)t * k * d;
   float4 v[VPT];
   float ss = 0.f;
-  if (VPT == 1 && k <= 8) {
-    // the slot weights and every slot row of a column in flight at once: one
-    // memory latency per row (the sums keep slot order; one column per thread)
-    float c[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) c[q] = q < k ? wts[(size_t)t * k + q] : 0.f;
+  for (int u = 0; u < VPT; ++u) {
+    const int j = threadIdx.x + u * blockDim.x;
+    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < d4) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < k; s0 += 4) {
+        float4 yv[4];
 #pragma unroll
-    for (int u = 0; u < VPT; ++u) {
-      const int j = threadIdx.x + u * blockDim.x;
-      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < d4) {
-        float4 yv[8];
+        for (int q = 0; q < 4; ++q)
+          if (s0 + q < k) yv[q] = load4<T>(yt, (size_t)(s0 + q) * d4 + j);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q < k) yv[q] = load4<T>(yt, (size_t)q * d4 + j);
-        float4 x = h4[j];
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q < k) {
-            acc.x += c[q] * yv[q].x;
-            acc.y += c[q] * yv[q].y;
-            acc.z += c[q] * yv[q].z;
-            acc.w += c[q] * yv[q].w;
+        for (int q = 0; q < 4; ++q)
+          if (s0 + q < k) {
+            const float c = ws[s0 + q];
+            acc.x += c * yv[q].x;
+            acc.y += c * yv[q].y;
+            acc.z += c * yv[q].z;
+            acc.w += c * yv[q].w;
           }
-        x.x += acc.x; x.y += acc.y; x.z += acc.z; x.w += acc.w;
-        h4[j] = x;
-        v[u] = x;
-        ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
       }
-    }
-  } else {
-    if (threadIdx.x < k) ws[threadIdx.x] = wts[(size_t)t * k + threadIdx.x];
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < VPT; ++u) {
-      const int j = threadIdx.x + u * blockDim.x;
-      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < d4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s0 = 0; s0 < k; s0 += 4) {
-          float4 yv[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (s0 + q < k) yv[q] = load4<T>(yt, (size_t)(s0 + q) * d4 + j);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (s0 + q < k) {
-              const float c = ws[s0 + q];
-              acc.x += c * yv[q].x;
-              acc.y += c * yv[q].y;
-              acc.z += c * yv[q].z;
-              acc.w += c * yv[q].w;
-            }
-        }
-        float4 x = h4[j];
-        x.x += acc.x; x.y += acc.y; x.z += acc.z; x.w += acc.w;
-        h4[j] = x;
-        v[u] = x;
-        ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
-      }
+      float4 x = h4[j];
+      x.x += acc.x; x.y += acc.y; x.z += acc.z; x.w += acc.w;
+      h4[j] = x;
+      v[u] = x;
+      ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
     }
   }
   if (norm_w == nullptr) return;
