@@ -49,7 +49,7 @@ NCU_TRAFFIC = {
     # canvas-step attention over an 8192-position cache (16/8 heads of 256, CTA pairs): the bench's launch shape
     "attention": (71362304 + 3758080, "k_attn_tc2.cu", "c6dffe33dab64a07"),
     # LM head with the sampler statistics, 256 tokens x 262144 vocabulary: the bench's launch shape
-    "lm_head": (1488360960 + 33390336, "k_gemm_tc.cu", "b6966e2537710892"),
+    "lm_head": (1491159296 + 33348608, "k_gemm_tc.cu", "90fc3c42a9945e1b"),
     # the fused sampler pass over 256 rows: the bench's launch shape
     "sampler_rows": (80628736 + 1649152, "k_sampler.cu", "d9ce1c2931c1b66c"),
 }
@@ -328,7 +328,9 @@ def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, pe
         up_b = moe_up_bytes(model, rows, touched) - touched * 2 * F * d * 2 * (1 - wb)
         down_b = moe_down_bytes(model, rows, touched) - touched * F * d * 2 * (1 - wb)
         kname = "gemm_fp4_kernel" if expert_bytes < 2.0 else "gemm_tc_kernel"
-        add("moe_up", f"{kname} (grouped gate/up + SwiGLU)", "hbm", up_b)
+        # bf16 experts, passes below 2048 tokens: gate/up runs on CTA pairs
+        uname = kname if expert_bytes < 2.0 or T >= 2048 else "gemm_tc2_grouped_kernel"
+        add("moe_up", f"{uname} (grouped gate/up + SwiGLU)", "hbm", up_b)
         add("moe_down", f"{kname} (grouped down, scatter)", "hbm", down_b)
     else:
         add("moe_up", "gemm_tc_kernel (grouped gate/up + SwiGLU)", "tensor", 2.0 * rows * 2 * F * d)
