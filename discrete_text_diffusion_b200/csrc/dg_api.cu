@@ -702,6 +702,9 @@ void moe_gemms_fp4(dg_handle* H, int l, int T) {
 #ifndef DG_MOE_PAIR
 #define DG_MOE_PAIR 1              // bit 0: gate/up on pairs, bit 1: down on pairs (passes below DG_LARGE_PASS)
 #endif
+#ifndef DG_MOE_PAIR_MIN_T
+#define DG_MOE_PAIR_MIN_T 64       // below this many tokens (AR decode) the one-CTA form keeps more SMs busy per item
+#endif
 #ifndef DG_MOE_PAIR_UP_KSUB
 #define DG_MOE_PAIR_UP_KSUB 1      // chunks per stage, gate/up (two weight operands)
 #endif
@@ -713,7 +716,7 @@ void moe_gemms_fp4(dg_handle* H, int l, int T) {
 bool moe_gemm_pair(dg_handle* H, int l, int T, int part) {
   const dg_config& c = H->c;
   const int tile = grouped_tile(H, T);
-  if (!H->bf16 || tile > 128 || T >= DG_LARGE_PASS || !(DG_MOE_PAIR & part)) return false;
+  if (!H->bf16 || tile > 128 || T < DG_MOE_PAIR_MIN_T || T >= DG_LARGE_PASS || !(DG_MOE_PAIR & part)) return false;
   const int n_work_max = c.n_experts + (T * c.top_k + tile - 1) / tile;
   const uint64_t rows = (uint64_t)H->T_max * c.top_k;
   const LayerMaps& M = H->lmaps[l];
