@@ -373,21 +373,46 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   if (row >= rows) return;
   const size_t stride = (size_t)rows;
   float M = -INFINITY;
-  for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[2 * (s * stride + row)]);
   float L = 0.f;
   float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+  if (n_split <= 8) {
+    // every split's (max, sum) and O columns in flight at once: one memory latency per row
+    float2 ml[8];
+    float4 v0[8], v1[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (s < n_split) {
+        ml[s] = *reinterpret_cast<const float2*>(part_ml + 2 * (s * stride + row));
+        const float4* po = reinterpret_cast<const float4*>(part_o + (s * stride + row) * kHd) + 2 * lane;
+        v0[s] = po[0];
+        v1[s] = po[1];
+      }
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (s < n_split) M = fmaxf(M, ml[s].x);
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (s < n_split && ml[s].x != -INFINITY) {
+        const float w = exp2f(ml[s].x - M);
+        L += ml[s].y * w;
+        a0.x += w * v0[s].x; a0.y += w * v0[s].y; a0.z += w * v0[s].z; a0.w += w * v0[s].w;
+        a1.x += w * v1[s].x; a1.y += w * v1[s].y; a1.z += w * v1[s].z; a1.w += w * v1[s].w;
+      }
+  } else {
+    for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[2 * (s * stride + row)]);
 #pragma unroll 4
-  for (int s = 0; s < n_split; ++s) {
-    const float ms = part_ml[2 * (s * stride + row)];
-    const float ls = part_ml[2 * (s * stride + row) + 1];
-    const float4* po = reinterpret_cast<const float4*>(part_o + (s * stride + row) * kHd) + 2 * lane;
-    const float4 v0 = po[0], v1 = po[1];
-    const bool live = ms != -INFINITY;
-    const float w = live ? exp2f(ms - M) : 0.f;
-    if (live) {
-      L += ls * w;
-      a0.x += w * v0.x; a0.y += w * v0.y; a0.z += w * v0.z; a0.w += w * v0.w;
-      a1.x += w * v1.x; a1.y += w * v1.y; a1.z += w * v1.z; a1.w += w * v1.w;
+    for (int s = 0; s < n_split; ++s) {
+      const float ms = part_ml[2 * (s * stride + row)];
+      const float ls = part_ml[2 * (s * stride + row) + 1];
+      const float4* po = reinterpret_cast<const float4*>(part_o + (s * stride + row) * kHd) + 2 * lane;
+      const float4 v0 = po[0], v1 = po[1];
+      const bool live = ms != -INFINITY;
+      const float w = live ? exp2f(ms - M) : 0.f;
+      if (live) {
+        L += ls * w;
+        a0.x += w * v0.x; a0.y += w * v0.y; a0.z += w * v0.z; a0.w += w * v0.w;
+        a1.x += w * v1.x; a1.y += w * v1.y; a1.z += w * v1.z; a1.w += w * v1.w;
+      }
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
