@@ -351,13 +351,15 @@ int pick_ntile(int n_mtiles, int T, int num_sms) {
 // Larger items stream an expert's weights fewer times but leave fewer items
 // to spread over the SMs when the routing concentrates on a few experts.
 #ifndef DG_GROUPED_TILE_LARGE
-#define DG_GROUPED_TILE_LARGE 128   // rows of an expert work item when a pass has >= DG_LARGE_PASS tokens
+#define DG_GROUPED_TILE_LARGE 256   // rows of an expert work item when a pass has >= DG_LARGE_PASS tokens
 #endif
 #ifndef DG_LARGE_PASS
 #define DG_LARGE_PASS 2048
 #endif
 int grouped_tile(const dg_handle* H, int T) {
   if (!H->bf16) return 64;
+  // the 256-row items are for the CTA-pair kernels; the NVFP4 kernel keeps 128
+  if (H->fp4) return DG_GROUPED_TILE;
   return T >= DG_LARGE_PASS ? DG_GROUPED_TILE_LARGE : DG_GROUPED_TILE;
 }
 
@@ -702,6 +704,9 @@ void moe_gemms_fp4(dg_handle* H, int l, int T) {
 #ifndef DG_MOE_PAIR
 #define DG_MOE_PAIR 1              // bit 0: gate/up on pairs, bit 1: down on pairs (passes below DG_LARGE_PASS)
 #endif
+#ifndef DG_MOE_PAIR_LARGE
+#define DG_MOE_PAIR_LARGE 3        // the same bits for passes of DG_LARGE_PASS tokens or more (256-row items)
+#endif
 #ifndef DG_MOE_PAIR_MIN_T
 #define DG_MOE_PAIR_MIN_T 64       // below this many tokens (AR decode) the one-CTA form keeps more SMs busy per item
 #endif
@@ -716,7 +721,9 @@ void moe_gemms_fp4(dg_handle* H, int l, int T) {
 bool moe_gemm_pair(dg_handle* H, int l, int T, int part) {
   const dg_config& c = H->c;
   const int tile = grouped_tile(H, T);
-  if (!H->bf16 || tile > 128 || T < DG_MOE_PAIR_MIN_T || T >= DG_LARGE_PASS || !(DG_MOE_PAIR & part)) return false;
+  const bool large = T >= DG_LARGE_PASS;
+  if (!H->bf16 || tile > 256 || T < DG_MOE_PAIR_MIN_T || !((large ? DG_MOE_PAIR_LARGE : DG_MOE_PAIR) & part))
+    return false;
   const int n_work_max = c.n_experts + (T * c.top_k + tile - 1) / tile;
   const uint64_t rows = (uint64_t)H->T_max * c.top_k;
   const LayerMaps& M = H->lmaps[l];
@@ -738,9 +745,11 @@ bool moe_gemm_pair(dg_handle* H, int l, int T, int part) {
   const CUtensorMap* b16 = bmap(H, x, kdim, rows, 16, g.ksub);
   const CUtensorMap* b32 = bmap(H, x, kdim, rows, 32, g.ksub);
   const CUtensorMap* b64 = bmap(H, x, kdim, rows, 64, g.ksub);
+  const CUtensorMap* b128 = tile > 128 ? bmap(H, x, kdim, rows, 128, g.ksub) : b64;
   const CUtensorMap& a0 = pick(part == 1 ? M.gate : M.down, g.ksub);
   const CUtensorMap& a1 = pick(part == 1 ? M.up : M.down, g.ksub);
-  if (!b16 || !b32 || !b64 || launch_gemm_tc2_grouped(a0, a1, *b16, *b32, *b64, g, H->num_sms, H->stream) != 0)
+  if (!b16 || !b32 || !b64 || !b128 ||
+      launch_gemm_tc2_grouped(a0, a1, *b16, *b32, *b64, *b128, g, H->num_sms, H->stream) != 0)
     H->bad_launch = true;
   return true;
 }

@@ -2,10 +2,10 @@
 // step's few tokens per expert ([P1 五]: 256 tokens spread over the experts).
 //
 // A work item is (expert e, token rows [row0, row0 + rows), 256-row block mb
-// of the expert's weights), rows <= 128.  A cluster of two CTAs computes it
+// of the expert's weights), rows <= 256.  A cluster of two CTAs computes it
 // with M = 256: CTA r holds the weight rows mb*256 + 128r .. +127 and half of
-// the item's token rows (N/2 of N = 32, 64 or 128 >= rows) in its own shared
-// memory; the leader issues the MMAs, which read both CTAs' halves; each CTA's
+// the item's token rows (N/2 of N = 32, 64, 128 or 256 >= rows) in its own
+// shared memory; the leader issues the MMAs, which read both CTAs' halves; each CTA's
 // TMEM holds its 128 accumulator rows for all N tokens and each CTA writes its
 // own output columns.  Per SM and K stage this streams 128 weight rows and
 // N/2 token rows, where one CTA per 128-row tile streams all N: an expert's
@@ -15,10 +15,12 @@
 //     silu(gate) * up as bf16 rows of the activation [T*k, F].
 //   mode 2 (down + scatter): out[row_map[token]] = the bf16 row of d columns
 //     (the token-slot order the combine sums in).
-// Per CTA, 192 threads: warp 0 lane 0 loads its halves (TMA, 128-byte
+// Per CTA, 320 threads: warp 0 lane 0 loads its halves (TMA, 128-byte
 // swizzle, completing on the leader's barrier); warp 1 lane 0 of the leader
-// issues the MMAs and commits to both CTAs' barriers; warps 2-5 are the
-// epilogue (staged in shared memory, 16-byte row stores).  Each TMA load
+// issues the MMAs and commits to both CTAs' barriers; warps 2-9 are the
+// epilogue, two groups of four warps taking alternate 32-token chunks (each
+// staged in shared memory and written as 16-byte row stores), so the
+// epilogue keeps up with the main loop at 256-token items.  Each TMA load
 // writes only its own CTA's shared memory.  Every wait is bounded; both CTAs
 // reach the final cluster barrier before the pair's TMEM is released.
 #include <cuda_bf16.h>
@@ -35,9 +37,10 @@ namespace {
 
 constexpr int kGM = 128;                 // weight rows per CTA
 constexpr int kGK = 64;
-constexpr int kGThreads = 192;
+constexpr int kGEpiGroups = 2;           // epilogue groups of 4 warps, taking alternate 32-token chunks
+constexpr int kGThreads = 64 + kGEpiGroups * 128;
 constexpr int kGABytes = kGM * kGK * 2;  // 16 KB: one 64-column chunk of 128 weight rows
-constexpr int kGBMaxRows = 64;           // token rows per CTA (the pair's N <= 128)
+constexpr int kGBMaxRows = 128;          // token rows per CTA (the pair's N <= 256)
 constexpr int kGMaxSmem = 232448;
 constexpr int kGEpiRows = 32;
 constexpr int kGEpiBytes = kGEpiRows * kGM * 2;   // bf16 staging tile of one 32-token chunk
@@ -53,16 +56,20 @@ struct GPairParams {
   const int32_t* row_map;
   int* err;
   int ksub, stages, stage_bytes, n_a, acc_half, n_acc_buf, acc_cols, tmem_cols;
+  int b_rows;          // token rows per CTA a stage has room for (half of the largest N)
   int vec;
 };
 
-// Token rows of the pair for an item of `rows` rows: 32, 64 or 128 (each CTA half of it).
-__device__ __forceinline__ int pair_n(int rows) { return rows <= 32 ? 32 : rows <= 64 ? 64 : 128; }
+// Token rows of the pair for an item of `rows` rows: 32, 64, 128 or 256 (each CTA half of it).
+__device__ __forceinline__ int pair_n(int rows) {
+  return rows <= 32 ? 32 : rows <= 64 ? 64 : rows <= 128 ? 128 : 256;
+}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     gemm_tc2_grouped_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap ta1,
                             const __grid_constant__ CUtensorMap tb16, const __grid_constant__ CUtensorMap tb32,
-                            const __grid_constant__ CUtensorMap tb64, const GPairParams P) {
+                            const __grid_constant__ CUtensorMap tb64, const __grid_constant__ CUtensorMap tb128,
+                            const GPairParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -82,7 +89,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < P.stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 2 * 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 2 * 4 * kGEpiGroups); }
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -114,7 +121,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
       const int mb = item % P.n_mblk, w = item / P.n_mblk;
       const int e = P.work[3 * w], row0 = P.work[3 * w + 1], rows = P.work[3 * w + 2];
       const int half = pair_n(rows) >> 1;
-      const CUtensorMap* tb = half == 16 ? &tb16 : half == 32 ? &tb32 : &tb64;
+      const CUtensorMap* tb = half == 16 ? &tb16 : half == 32 ? &tb32 : half == 64 ? &tb64 : &tb128;
       const int m0 = mb * 2 * kGM + (int)rank * kGM;
       const int trow = row0 + (int)rank * half;
       const uint32_t tx = 2u * (a_bytes + (uint32_t)(P.ksub * half * kGK * 2));
@@ -176,9 +183,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     // accumulator (weight row m0 + r, one column per token) into a [token][128]
     // bf16 staging tile; then the 128 threads write whole 256-byte output rows
     // with 16-byte stores.
-    const int q = warp & 3;
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
-    const int te = threadIdx.x - 64;
+    const int grp = (warp - 2) >> 2;   // epilogue group
+    const int te = threadIdx.x - 64 - 128 * grp;
+    __nv_bfloat16* gstg = stg + grp * (kGEpiRows * kGM);
     const uint32_t empty_bar = map_to_rank(&acc_empty[0], 0);
     int it = 0;
     for (int item = cid; item < total; item += n_clusters, ++it) {
@@ -190,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
       if (!mbar_wait(&acc_full[ab], use & 1u, err, kErrTimeoutEpi)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * P.acc_cols);
-      for (int c0 = 0; c0 < rows; c0 += kGEpiRows) {
+      for (int c0 = kGEpiRows * grp; c0 < rows; c0 += kGEpiRows * kGEpiGroups) {
         uint32_t v[32];
         tmem_ld32(tbase + (uint32_t)c0, v);
         if (P.mode == 1) {
@@ -198,13 +207,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
           tmem_ld32(tbase + (uint32_t)(P.acc_half + c0), u);
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            stg[j * kGM + r] = __float2bfloat16_rn(
+            gstg[j * kGM + r] = __float2bfloat16_rn(
                 __fdividef(__uint_as_float(v[j]), 1.f + __expf(-__uint_as_float(v[j]))) * __uint_as_float(u[j]));
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) stg[j * kGM + r] = __float2bfloat16_rn(__uint_as_float(v[j]));
+          for (int j = 0; j < 32; ++j) gstg[j * kGM + r] = __float2bfloat16_rn(__uint_as_float(v[j]));
         }
-        named_barrier_sync(1, 128);
+        named_barrier_sync(1 + grp, 128);
         const int nrow = min(kGEpiRows, rows - c0);
 #pragma unroll 4
         for (int it2 = 0; it2 < kGEpiRows * 16 / 128; ++it2) {
@@ -213,7 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
           if (row < nrow && mm < P.M) {
             const int tok = row0 + c0 + row;
             __nv_bfloat16* dst = P.out + (size_t)(P.mode == 2 ? P.row_map[tok] : tok) * P.ld_out + mm;
-            const __nv_bfloat16* src = stg + row * kGM + c8 * 8;
+            const __nv_bfloat16* src = gstg + row * kGM + c8 * 8;
             if (P.vec && mm + 7 < P.M) {
               *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
             } else {
@@ -221,7 +230,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
             }
           }
         }
-        named_barrier_sync(1, 128);   // the staging tile is reused by the next chunk
+        named_barrier_sync(1 + grp, 128);   // the staging tile is reused by the group's next chunk
       }
       tc_fence_before();
       __syncwarp();
@@ -241,8 +250,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
 }  // namespace
 
 int launch_gemm_tc2_grouped(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b16,
-                            const CUtensorMap& b32, const CUtensorMap& b64, const TcGemm& g, int num_sms,
-                            cudaStream_t s) {
+                            const CUtensorMap& b32, const CUtensorMap& b64, const CUtensorMap& b128, const TcGemm& g,
+                            int num_sms, cudaStream_t s) {
   const int ksub = g.ksub >= 1 ? g.ksub : 1;
   if ((g.mode != 1 && g.mode != 2) || g.ntile > 2 * kGBMaxRows || g.K % kGK || (ksub != 1 && ksub != 2))
     return -1;
@@ -259,14 +268,16 @@ int launch_gemm_tc2_grouped(const CUtensorMap& a0, const CUtensorMap& a1, const 
   P.err = g.err;
   P.ksub = ksub;
   P.n_a = g.mode == 1 ? 2 : 1;
-  P.acc_half = 2 * kGBMaxRows;                  // the up accumulator's column offset (mode 1)
-  P.acc_cols = P.n_a * 2 * kGBMaxRows;          // 256 (mode 1) or 128 columns per buffer
-  P.n_acc_buf = 2;
+  const int max_n = g.ntile <= 32 ? 32 : g.ntile <= 64 ? 64 : g.ntile <= 128 ? 128 : 256;   // pair_n(ntile)
+  P.b_rows = max_n / 2;
+  P.acc_half = max_n;                           // the up accumulator's column offset (mode 1)
+  P.acc_cols = P.n_a * max_n;                   // columns per accumulator buffer
+  P.n_acc_buf = 2 * P.acc_cols <= 512 ? 2 : 1;
   P.tmem_cols = 32;
   while (P.tmem_cols < P.n_acc_buf * P.acc_cols) P.tmem_cols <<= 1;
   if (P.tmem_cols > 512) return -1;
-  P.stage_bytes = ksub * (P.n_a * kGABytes + kGBMaxRows * kGK * 2);
-  const int overhead = 1024 + 1024 + kGEpiBytes;
+  P.stage_bytes = ksub * (P.n_a * kGABytes + P.b_rows * kGK * 2);
+  const int overhead = 1024 + 1024 + kGEpiGroups * kGEpiBytes;
   P.stages = std::min(8, (kGMaxSmem - overhead) / P.stage_bytes);
   if (P.stages < 2) return -1;
   const int smem = overhead + P.stages * P.stage_bytes;
@@ -279,7 +290,7 @@ int launch_gemm_tc2_grouped(const CUtensorMap& a0, const CUtensorMap& a1, const 
     attr = true;
   }
   const int clusters = std::min(max_items, num_sms / 2);
-  launch_k(gemm_tc2_grouped_kernel, dim3(2 * clusters), dim3(kGThreads), smem, s, a0, a1, b16, b32, b64, P);
+  launch_k(gemm_tc2_grouped_kernel, dim3(2 * clusters), dim3(kGThreads), smem, s, a0, a1, b16, b32, b64, b128, P);
   return 0;
 }
 

@@ -190,12 +190,13 @@ int launch_gemm_tc_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
 // (k_moe_tc2.cu): 256-row weight blocks, each CTA of a pair holding 128 weight
 // rows and half of the item's token rows.  a0 / a1: expert weight maps (64,
 // rows, K/64, E) with boxes of 128 rows x g.ksub chunks (a1: the up weights,
-// mode 1); b16 / b32 / b64: token maps with boxes of 16 / 32 / 64 rows x
-// g.ksub chunks.  Work items of up to 128 rows (g.ntile <= 128).  Returns -1
-// (nothing launched) for another shape.
+// mode 1); b16 / b32 / b64 / b128: token maps with boxes of 16 / 32 / 64 /
+// 128 rows x g.ksub chunks (b128 is read only when g.ntile > 128).  Work items
+// of up to 256 rows (g.ntile <= 256).  Returns -1 (nothing launched) for
+// another shape.
 int launch_gemm_tc2_grouped(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b16,
-                            const CUtensorMap& b32, const CUtensorMap& b64, const TcGemm& g, int num_sms,
-                            cudaStream_t s);
+                            const CUtensorMap& b32, const CUtensorMap& b64, const CUtensorMap& b128, const TcGemm& g,
+                            int num_sms, cudaStream_t s);
 
 // NVFP4 grouped expert GEMMs (k_gemm_fp4.cu): modes 1 (gate/up + SwiGLU) and 2
 // (down + scatter) of the bf16 grouped GEMM, with the weights as E2M1 codes
