@@ -110,7 +110,10 @@ def aggregate(dist, elapsed_ms: float, units: float, device=None):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+    """nvidia-smi clock / throttle-reason samples every 50 ms.  __enter__ returns
+    once the sampler is running (its first sample written); mark() at the start
+    of the timed region and stop() at its end keep the samples in between, plus
+    the first one after the end when the region is shorter than the interval."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -126,11 +129,34 @@ class ClockSampler:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
+                                          "--format=csv,noheader,nounits", "-lms", "50", "-f", self.path],
                                          stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        self.first = 0
+        self.last = None
+        t0 = time.time()
+        while self.proc is not None and self._count() == 0 and time.time() - t0 < 5.0:
+            time.sleep(0.01)
         return self
+
+    def _count(self):
+        try:
+            with open(self.path) as fh:
+                return sum(1 for line in fh if line.count(",") >= 8)
+        except OSError:
+            return 0
+
+    def mark(self):
+        self.first = self._count()
+
+    def stop(self):
+        self.last = self._count()
+        if self.last == self.first and self.proc is not None:   # region shorter than the interval
+            t0 = time.time()
+            while self._count() == self.first and time.time() - t0 < 1.0:
+                time.sleep(0.005)
+            self.last = self.first + 1
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -148,6 +174,8 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
             os.unlink(self.path)
+        if self.last is not None:
+            rows = rows[self.first:self.last]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -488,11 +516,15 @@ def _measure_workload(m, args, name, steps, warmup, dev, dist, world, with_clock
         clk.__enter__()
     barrier(dist)
     torch.cuda.synchronize(dev)
+    if clk:
+        clk.mark()
     ev0.record(stream)
     for _ in range(steps):
         one_step()
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    if clk:
+        clk.stop()
     barrier(dist)
     if clk:
         clk.__exit__(None, None, None)

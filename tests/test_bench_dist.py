@@ -2,6 +2,7 @@
 elapsed time and the summed units, and only rank 0 prints.  CPU only."""
 import os
 import socket
+import sys
 
 import pytest
 import torch.multiprocessing as mp
@@ -93,3 +94,37 @@ def test_reference_arm_under_torchrun_prints_on_rank_0_only():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1 and '"impl": "reference"' in lines[0]
+
+
+def test_clock_sampler_keeps_samples_of_a_short_region(tmp_path, monkeypatch):
+    """The bench's clock record: with a fake nvidia-smi writing a sample every
+    20 ms, a timed region shorter than the interval still gets one sample
+    (the first after its end), and samples before the region are dropped."""
+    import stat
+    import time
+
+    import bench
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text(
+        "#!" + sys.executable + "\n"
+        "import sys, time\n"
+        "path = sys.argv[sys.argv.index('-f') + 1]\n"
+        "i = 0\n"
+        "while True:\n"
+        "    with open(path, 'a') as fh:\n"
+        "        mhz = 1000 if i == 0 else 1965\n"
+        "        fh.write(f'0, {mhz}, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Active\\n')\n"
+        "    i += 1\n"
+        "    time.sleep(0.02)\n")
+    fake.chmod(fake.stat().st_mode | stat.S_IEXEC)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ["PATH"])
+    clk = bench.ClockSampler(0)
+    clk.__enter__()
+    time.sleep(0.05)          # samples before the region: dropped
+    clk.mark()
+    clk.stop()                # a region shorter than the interval
+    clk.__exit__(None, None, None)
+    s = clk.summary()
+    assert s["samples"] >= 1
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
