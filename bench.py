@@ -355,14 +355,17 @@ def kernel_rooflines(model, batch, canvas, blocks, touched, breakdown, peaks, pe
         wb = expert_bytes / 2.0      # the weight terms of the byte counts scale with the storage
         up_b = moe_up_bytes(model, rows, touched) - touched * 2 * F * d * 2 * (1 - wb)
         down_b = moe_down_bytes(model, rows, touched) - touched * F * d * 2 * (1 - wb)
+        # bf16 experts: gate/up on CTA pairs from 64 tokens per pass, down on pairs from 2048
         kname = "gemm_fp4_kernel" if expert_bytes < 2.0 else "gemm_tc_kernel"
-        # bf16 experts, passes below 2048 tokens: gate/up runs on CTA pairs
-        uname = kname if expert_bytes < 2.0 or T >= 2048 else "gemm_tc2_grouped_kernel"
+        uname = kname if expert_bytes < 2.0 or T < 64 else "gemm_tc2_grouped_kernel"
+        dname = kname if expert_bytes < 2.0 or T < 2048 else "gemm_tc2_grouped_kernel"
         add("moe_up", f"{uname} (grouped gate/up + SwiGLU)", "hbm", up_b)
-        add("moe_down", f"{kname} (grouped down, scatter)", "hbm", down_b)
+        add("moe_down", f"{dname} (grouped down, scatter)", "hbm", down_b)
     else:
-        add("moe_up", "gemm_tc_kernel (grouped gate/up + SwiGLU)", "tensor", 2.0 * rows * 2 * F * d)
-        add("moe_down", "gemm_tc_kernel (grouped down, scatter)", "tensor", 2.0 * rows * F * d)
+        uname = "gemm_tc2_grouped_kernel" if T >= 64 else "gemm_tc_kernel"
+        dname = "gemm_tc2_grouped_kernel" if T >= 2048 else "gemm_tc_kernel"
+        add("moe_up", f"{uname} (grouped gate/up + SwiGLU)", "tensor", 2.0 * rows * 2 * F * d)
+        add("moe_down", f"{dname} (grouped down, scatter)", "tensor", 2.0 * rows * F * d)
     if "dense_gemm" in breakdown:
         # QKV and O every pass, W_sc every step after the first: weights once each (bytes), or
         # every token through them (flops), whichever bound is slower
