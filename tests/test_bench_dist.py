@@ -128,3 +128,25 @@ def test_clock_sampler_keeps_samples_of_a_short_region(tmp_path, monkeypatch):
     assert s["samples"] >= 1
     assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_kernel_rooflines_name_the_kernels_in_use():
+    """The per-class rooflines name the kernel the library runs for the pass
+    size: CTA pairs for attention (16/8 heads), the canvas-size dense split-K
+    and gate/up; the batch-16 passes run both expert projections on pairs."""
+    import bench
+    from discrete_text_diffusion_b200 import synth
+    model = synth.WORKLOADS["full_b16"]["model"]
+    peaks = {"hbm_gbs": 6544.0, "bf16_tflops": 1653.0, "bf16_tflops_sustained": 1396.4}
+    bd = {c: (240, 10.0) for c in ["attention", "moe_up", "moe_down", "dense_gemm", "lm_head", "sampler_rows"]}
+    b1 = bench.kernel_rooflines(model, 1, 256, [(8192, 7)], 14.8, bd, peaks, "measured")
+    b16 = bench.kernel_rooflines(model, 16, 256, [(4096, 12)], 61.5, bd, peaks, "measured")
+    assert b1["attention"]["kernel"].startswith("attn_tc2_kernel")
+    assert b1["dense_gemm"]["kernel"].startswith("gemm_tc2_kernel")
+    assert b1["moe_up"]["kernel"].startswith("gemm_tc2_grouped_kernel")
+    assert b1["moe_down"]["kernel"].startswith("gemm_tc_kernel")
+    assert b16["moe_up"]["kernel"].startswith("gemm_tc2_grouped_kernel")
+    assert b16["moe_down"]["kernel"].startswith("gemm_tc2_grouped_kernel")
+    assert b16["dense_gemm"]["kernel"].startswith("gemm_tc_kernel")
+    for r in list(b1.values()) + list(b16.values()):
+        assert 0 < r["frac"] and r["launches"] == 240
